@@ -1,0 +1,408 @@
+#!/usr/bin/env python3
+"""Benchmark of the fused rotate + int4-quantise hot path (and the W4A4 linear) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--no-extra]
+
+One step = one pass of the hot path over one batch: the fused randomized-Hadamard
+rotate + int4 group-quantise + pack of the Llama-3.2-1B-shaped activation batch
+A[8192, 2048] bf16 (Student-t(4) x 0.5, 0.5% channels x100, G = 32). ``value`` is the
+whole-job throughput in GB/s of algorithmic bytes (bf16 read + packed codes + fp16
+scales written), with inputs resident in HBM; inputs and outputs rotate through six
+buffer sets (258 MB > the 126 MB L2) so every step reads from DRAM.
+
+Also reported: the roofline of that kernel against the measured HBM copy bandwidth, the
+same metric end to end through the C ABI from pinned host memory, the fp64 oracle timed
+on the host cores, SM clocks sampled during the timed region, and (unless --no-extra)
+the other workloads: down_proj K = 8192 int4/int2, HARP K = 11008, and the W4A4 linear
+(prefill TOPS against the int8 tensor peak, decode GB/s).
+
+``--impl reference`` times the fp64 CPU oracle on the same workload (a bounded sample of
+rows per step) and prints the same JSON line with "impl": "reference".
+Under torchrun (N > 1) every rank runs the full batch on its own GPU (weak scaling,
+no data-path collective); time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "rotate+int4-quant GB/s (fraction of HBM peak); W4A4 linear TOPS vs int8 peak"
+WORKLOAD = "llama32_1b"
+INT8_DENSE_SPEC_TOPS = 4500.0
+
+
+def algorithmic_bytes(M: int, K: int, bits: int, G: int, in_bytes: int = 2) -> int:
+    return M * K * in_bytes + M * K * bits // 8 + M * (K // G) * 2
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+def kernel_sources_sha() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "hadamard_butterfly_rotation_b200", "csrc")
+    for f in ("rot_fwht.cu", "rot_internal.cuh"):
+        h.update(open(os.path.join(csrc, f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(name: str):
+    """Per-launch DRAM bytes from a committed ncu summary, if it was taken on the current kernel."""
+    p = os.path.join(ROOT, "profiles", f"{name}.json")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p))
+    if d.get("source_sha") != kernel_sources_sha():
+        return None
+    return d.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons with NVML while the timed region runs."""
+
+    def __init__(self, dev_index: int, period: float = 0.02):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self.period = period
+        self._stop = threading.Event()
+        self._t = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(dev_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self.nv = None
+
+    def _run(self):
+        nv = self.nv
+        names = {
+            "hw_slowdown": getattr(nv, "nvmlClocksEventReasonHwSlowdown", 0x8),
+            "hw_thermal_slowdown": getattr(nv, "nvmlClocksEventReasonHwThermalSlowdown", 0x40),
+            "sw_thermal_slowdown": getattr(nv, "nvmlClocksEventReasonSwThermalSlowdown", 0x20),
+            "sw_power_cap": getattr(nv, "nvmlClocksEventReasonSwPowerCap", 0x4),
+            "hw_power_brake_slowdown": getattr(nv, "nvmlClocksEventReasonHwPowerBrakeSlowdown", 0x80),
+        }
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for k, bit in names.items():
+                    if r & bit:
+                        self.reasons.add(k)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.nv is not None:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._t:
+            self._t.join()
+
+    def summary(self):
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ----------------------------------------------------------------------------- reference arm
+
+def cpu_oracle_throughput(wl, bits, G, seconds: float):
+    """fp64 oracle (dense RHT + quantisation) on the host cores: GB/s of algorithmic bytes."""
+    from oracle import hadamard as Hd
+    from oracle import quant as Q
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max(i.get("num_threads", 1) for i in threadpool_info()) if threadpool_info() else os.cpu_count()
+    except Exception:
+        cores = os.cpu_count()
+    rows = 512
+    done_rows, t0 = 0, time.perf_counter()
+    r0 = 0
+    while True:
+        blk = wl.A[r0:r0 + rows]
+        Q.quantize(Hd.rht_apply(blk, wl.signs), bits, G)
+        done_rows += blk.shape[0]
+        r0 = (r0 + rows) % wl.M
+        if time.perf_counter() - t0 >= seconds:
+            break
+    dt = time.perf_counter() - t0
+    gbs = algorithmic_bytes(done_rows, wl.K, bits, G) / dt / 1e9
+    return gbs, cores, done_rows, dt
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import workloads as W
+    wl = W.make_workload(WORKLOAD)
+    bits, G = wl.quant[0]
+    step_times = []
+    from oracle import hadamard as Hd
+    from oracle import quant as Q
+    rows = 512
+    for i in range(args.warmup + args.steps):
+        r0 = (i * rows) % wl.M
+        t0 = time.perf_counter()
+        Q.quantize(Hd.rht_apply(wl.A[r0:r0 + rows], wl.signs), bits, G)
+        if i >= args.warmup:
+            step_times.append(time.perf_counter() - t0)
+    tot = sum(step_times)
+    gbs = algorithmic_bytes(rows * len(step_times), wl.K, bits, G) / tot / 1e9
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max(i.get("num_threads", 1) for i in threadpool_info())
+    except Exception:
+        cores = os.cpu_count()
+    sample = f"{rows} of {wl.M} rows per step (fp64 dense Sylvester RHT + fp32-decision quantiser)"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(gbs, 4), "unit": "GB/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(1000 * tot / len(step_times), 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": "llama32_1b A[8192,2048] bf16, RHT K=2048, int4 G=32", "rows_per_step": rows},
+        "cpu_baseline": {"value": round(gbs, 4), "unit": "GB/s", "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(gbs, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line))
+    return 0
+
+
+# ----------------------------------------------------------------------------- our arm
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20000)
+    ap.add_argument("--warmup", type=int, default=200)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-extra", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import torch
+    import torch.distributed as dist
+    import workloads as W
+    import hadamard_butterfly_rotation_b200 as hbr
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        torch.cuda.set_device(local)
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    dev = torch.device("cuda", local if world > 1 else 0)
+    torch.cuda.set_device(dev)
+
+    wl = W.make_workload(WORKLOAD, seed=0)
+    bits, G = wl.quant[0]
+    M, K = wl.M, wl.K
+    plan = hbr.Plan.rht(K, wl.signs)
+    A_host = torch.from_numpy(wl.A).to(torch.bfloat16)
+    NSETS = 6
+    A_sets = [A_host.to(dev) for _ in range(NSETS)]
+    outs = [(torch.empty((M, K * bits // 8), dtype=torch.uint8, device=dev),
+             torch.empty((M, K // G), dtype=torch.float16, device=dev)) for _ in range(NSETS)]
+    stream = torch.cuda.current_stream(dev)
+
+    def step(i):
+        c, s = outs[i % NSETS]
+        hbr.rot_quant(A_sets[i % NSETS], plan, bits, G, codes=c, scales=s, stream=stream)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(dev.index) as clk:
+        ev0.record(stream)
+        for i in range(args.steps):
+            step(i)
+        ev1.record(stream)
+        torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    ms = ev0.elapsed_time(ev1)
+    if world > 1:
+        t = torch.tensor([ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    bytes_step = algorithmic_bytes(M, K, bits, G)
+    gbs = bytes_step * args.steps * world / (ms / 1e3) / 1e9
+    per_launch_s = ms / 1e3 / args.steps
+    achieved = bytes_step / per_launch_s / 1e9
+    peaks, peak_kind = load_peaks()
+
+    # end to end through the C ABI from pinned host memory (H2D of A, D2H of codes + scales)
+    A_pin = A_host.pin_memory()
+    c_pin = torch.empty((M, K * bits // 8), dtype=torch.uint8).pin_memory()
+    s_pin = torch.empty((M, K // G), dtype=torch.float16).pin_memory()
+    dA, (dc, ds) = A_sets[0], outs[0]
+
+    def e2e_step():
+        dA.copy_(A_pin, non_blocking=True)
+        hbr.rot_quant(dA, plan, bits, G, codes=dc, scales=ds, stream=stream)
+        c_pin.copy_(dc, non_blocking=True)
+        s_pin.copy_(ds, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    e_steps = 20
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e_ms = e0.elapsed_time(e1) / e_steps
+    if world > 1:
+        t = torch.tensor([e_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e_ms = float(t.item())
+    e2e_gbs = bytes_step * world / (e_ms / 1e3) / 1e9
+
+    extra = {}
+    if not args.no_extra and rank == 0:
+        extra = run_extra(hbr, W, dev, stream, peaks)
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+
+    cpu = None
+    if world == 1:
+        gb, cores, rows_done, dt = cpu_oracle_throughput(wl, bits, G, args.cpu_seconds)
+        cpu = {"value": round(gb, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
+               "sample": f"{rows_done} rows of A[8192,2048] ({dt:.1f} s, blocks of 512 rows): fp64 dense "
+                         "Sylvester RHT + quantiser"}
+    line = {
+        "metric": METRIC, "value": round(gbs, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 6), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": "llama32_1b: A[8192,2048] bf16, RHT K=2048 (signs + FWHT + 1/sqrt(K)), "
+                               "int4 G=32, packed codes + fp16 scales",
+                   "global_batch": M * world, "l2": "6 rotating input/output sets (258 MB > 126 MB L2)",
+                   "parallelism": f"dp{world} (independent rows)"},
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": profiled_traffic("rot_quant_llama32_1b"),
+                     "peak_source": f"{peak_kind} HBM copy bandwidth (MEASURED_PEAKS.json hbm_gbs)"},
+        "cpu_baseline": cpu,
+        "e2e": {"value": round(e2e_gbs, 2), "unit": "GB/s", "h2d_bytes_per_step": M * K * 2,
+                "d2h_bytes_per_step": M * K * bits // 8 + M * (K // G) * 2},
+        "gpu_launches": args.steps,
+        "clocks": clk.summary(),
+    }
+    if extra:
+        line["extra"] = extra
+    print(json.dumps(line))
+    return 0
+
+
+def _time_loop(fn, n, stream, warm=5):
+    import torch
+    for i in range(warm):
+        fn(i)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(n):
+        fn(i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / n / 1e3  # seconds per call
+
+
+def run_extra(hbr, W, dev, stream, peaks):
+    import torch
+    out = {}
+    hbm = peaks["hbm_gbs"]
+    # rotate + quantise on the other workloads
+    for name, variant in (("down_proj", None), ("harp11008", "init_identity"), ("harp11008", "random")):
+        wl = W.make_workload(name)
+        if variant is None:
+            plan = hbr.Plan.rht(wl.K, wl.signs)
+        else:
+            plan = hbr.harp_plan(W.harp_draws(2, wl.extra["radices"]), wl.signs, variant)
+        nsets = 3 if wl.M * wl.K * 2 > 60e6 else 6
+        As = [torch.from_numpy(wl.A).to(torch.bfloat16).to(dev) for _ in range(nsets)]
+        for bits, G in wl.quant:
+            outs = [(torch.empty((wl.M, wl.K * bits // 8), dtype=torch.uint8, device=dev),
+                     torch.empty((wl.M, wl.K // G), dtype=torch.float16, device=dev)) for _ in range(nsets)]
+            n = 200 if variant != "random" else 20
+
+            def f(i):
+                c, s = outs[i % nsets]
+                hbr.rot_quant(As[i % nsets], plan, bits, G, codes=c, scales=s, stream=stream)
+            t = _time_loop(f, n, stream)
+            b = algorithmic_bytes(wl.M, wl.K, bits, G)
+            key = f"{name}{'_' + variant if variant else ''}_int{bits}_G{G}"
+            out[key] = {"us": round(t * 1e6, 2), "GB/s": round(b / t / 1e9, 1), "frac_hbm": round(b / t / 1e9 / hbm, 4)}
+        del As
+    # W4A4 linear: prefill TOPS and decode GB/s
+    int8_peak = measure_int8_peak(dev)
+    for name in ("q_proj_prefill", "up_proj_prefill", "q_proj_decode", "up_proj_decode"):
+        wl = W.make_workload(name)
+        bits, G = wl.quant[0]
+        plan = hbr.Plan.rht(wl.K, wl.signs)
+        Aq, As_ = hbr.rot_quant(torch.from_numpy(wl.A).to(torch.bfloat16).to(dev), plan, bits, G)
+        Wq, Ws = hbr.rot_quant(torch.from_numpy(np.ascontiguousarray(wl.W.T)).to(dev), plan, bits, G)
+        N = Wq.shape[0]
+        C = torch.empty((wl.M, N), dtype=torch.bfloat16, device=dev)
+        n = 50 if wl.M > 16 else 200
+        t = _time_loop(lambda i: hbr.w4a4_linear(Aq, As_, Wq, Ws, G, out=C, stream=stream), n, stream)
+        ops = 2.0 * wl.M * N * wl.K
+        wbytes = Wq.numel() + Ws.numel() * 2 + Aq.numel() + As_.numel() * 2 + C.numel() * 2
+        out[f"w4a4_{name}"] = {"us": round(t * 1e6, 2), "TOPS": round(ops / t / 1e12, 1),
+                               "frac_int8_spec": round(ops / t / 1e12 / INT8_DENSE_SPEC_TOPS, 4),
+                               "frac_int8_measured": round(ops / t / 1e12 / int8_peak, 4) if int8_peak else None,
+                               "GB/s": round(wbytes / t / 1e9, 1)}
+    out["int8_peak_measured_TOPS"] = round(int8_peak, 1) if int8_peak else None
+    return out
+
+
+def measure_int8_peak(dev):
+    """Same-run int8 tensor ceiling: torch._int_mm 8192^3 (library GEMM, reference only)."""
+    import torch
+    try:
+        a = torch.randint(-8, 8, (8192, 8192), dtype=torch.int8, device=dev)
+        b = torch.randint(-8, 8, (8192, 8192), dtype=torch.int8, device=dev).t()
+        t = _time_loop(lambda i: torch._int_mm(a, b), 10, torch.cuda.current_stream(dev), warm=2)
+        return 2 * 8192 ** 3 / t / 1e12
+    except Exception:
+        return None
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,281 @@
+"""Python binding of the B200 rotation / group-quantisation / W4A4 library (``include/rot_b200.h``).
+
+Argument marshalling only: every step runs in the CUDA library ``_lib/librot_b200.so``
+(build it with ``python -m hadamard_butterfly_rotation_b200.build``). PyTorch supplies
+device memory and the current CUDA stream. Importing this package without the built
+library raises ImportError; there is no CPU fallback.
+
+Names follow the C ABI: ``Plan`` (rot_plan_create / rot_plan_destroy), ``rot_apply``,
+``rot_quant``, ``rot_dequant``, ``w4a4_linear``, ``w4a4_group_partials``,
+``harp_givens_blocks``, ``harp_qr_block``, ``check_device``.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "_lib", "librot_b200.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is missing: build the CUDA library first "
+        "(python -m hadamard_butterfly_rotation_b200.build)")
+
+_lib = C.CDLL(LIB_PATH)
+
+ROT_OK, ROT_EINVAL, ROT_EUNSUPPORTED, ROT_ECUDA, ROT_ETIMEOUT, ROT_ENOMEM = range(6)
+ROT_F32, ROT_BF16 = 0, 1
+_STATUS = {0: "ROT_OK", 1: "ROT_EINVAL", 2: "ROT_EUNSUPPORTED", 3: "ROT_ECUDA", 4: "ROT_ETIMEOUT", 5: "ROT_ENOMEM"}
+
+_vp, _i64, _i32, _int = C.c_void_p, C.c_int64, C.c_int32, C.c_int
+_lib.rot_plan_create.argtypes = [C.POINTER(_vp), _int, _int, C.POINTER(_int), C.POINTER(C.POINTER(C.c_float)),
+                                 C.POINTER(_i64), C.POINTER(C.POINTER(_i32)), C.POINTER(C.c_int8)]
+_lib.rot_plan_destroy.argtypes = [_vp]
+_lib.rot_plan_info.argtypes = [_vp, C.POINTER(_int), C.POINTER(_int)]
+_lib.rot_apply.argtypes = [_vp, _int, _i64, _i64, _vp, _int, _vp, _i64, _vp]
+_lib.rot_quant.argtypes = [_vp, _int, _i64, _i64, _vp, _int, _int, _vp, _vp, _vp]
+_lib.rot_dequant.argtypes = [_vp, _vp, _i64, _vp, _int, _int, _int, _vp, _vp]
+_lib.w4a4_linear.argtypes = [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _int, _vp, _int, _vp]
+_lib.w4a4_group_partials.argtypes = [_vp, _vp, _i64, _i64, _i64, _int, _vp, _vp]
+_lib.rot_harp_givens_blocks.argtypes = [C.POINTER(C.c_double), _i64, C.POINTER(C.c_float)]
+_lib.rot_harp_qr_block.argtypes = [C.POINTER(C.c_double), _int, C.POINTER(C.c_float)]
+_lib.rot_check_device.argtypes = []
+_lib.rot_last_error.restype = C.c_char_p
+_lib.rot_version.restype = C.c_char_p
+for _f in ("rot_plan_create", "rot_plan_destroy", "rot_plan_info", "rot_apply", "rot_quant", "rot_dequant",
+           "w4a4_linear", "w4a4_group_partials", "rot_harp_givens_blocks", "rot_harp_qr_block",
+           "rot_check_device"):
+    getattr(_lib, _f).restype = _int
+
+
+class RotError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"{_STATUS.get(status, status)}: {msg}")
+        self.status = status
+
+
+def _check(st: int):
+    if st != ROT_OK:
+        raise RotError(st, _lib.rot_last_error().decode())
+
+
+def version() -> str:
+    return _lib.rot_version().decode()
+
+
+def last_error() -> str:
+    return _lib.rot_last_error().decode()
+
+
+def _stream(stream):
+    import torch
+    if stream is None:
+        return C.c_void_p(torch.cuda.current_stream().cuda_stream)
+    if isinstance(stream, int):
+        return C.c_void_p(stream)
+    return C.c_void_p(stream.cuda_stream)
+
+
+def _dtype_code(t) -> int:
+    import torch
+    if t.dtype == torch.bfloat16:
+        return ROT_BF16
+    if t.dtype == torch.float32:
+        return ROT_F32
+    raise TypeError(f"activations must be bf16 or fp32, got {t.dtype}")
+
+
+def _ptr(t) -> C.c_void_p:
+    return C.c_void_p(t.data_ptr()) if t is not None else C.c_void_p(0)
+
+
+class Plan:
+    """A rotation plan T = (P_{m-1} S_{m-1}) ... (P_0 S_0) D on the current CUDA device.
+
+    radices: schedule (prod == K); stage_params[t]: None (base mixer) or float32 array of
+    shape [n_blocks, b, b] (n_blocks 1 or K/b); perms[t]: None or int32 permutation
+    applied after stage t as a gather; signs: None or int8 +-1 of length K.
+    """
+
+    def __init__(self, K: int, radices, stage_params=None, perms=None, signs=None):
+        import torch  # noqa: F401  (ensures the CUDA runtime is initialised by torch)
+        m = len(radices)
+        self.K = int(K)
+        self.radices = [int(b) for b in radices]
+        rad = (_int * m)(*self.radices)
+        keep = []
+        sp = None
+        nb = None
+        if stage_params is not None and any(p is not None for p in stage_params):
+            sp = (C.POINTER(C.c_float) * m)()
+            nb = (_i64 * m)()
+            for t, prm in enumerate(stage_params):
+                if prm is None:
+                    sp[t] = C.POINTER(C.c_float)()
+                    nb[t] = 0
+                else:
+                    a = np.ascontiguousarray(prm, dtype=np.float32)
+                    b = self.radices[t]
+                    if a.size % (b * b):
+                        raise ValueError("stage params must hold whole b x b blocks")
+                    keep.append(a)
+                    sp[t] = a.ctypes.data_as(C.POINTER(C.c_float))
+                    nb[t] = a.size // (b * b)
+        pp = None
+        if perms is not None and any(p is not None for p in perms):
+            pp = (C.POINTER(_i32) * m)()
+            for t, P in enumerate(perms):
+                if P is None:
+                    pp[t] = C.POINTER(_i32)()
+                else:
+                    a = np.ascontiguousarray(P, dtype=np.int32)
+                    keep.append(a)
+                    pp[t] = a.ctypes.data_as(C.POINTER(_i32))
+        sg = None
+        if signs is not None:
+            s = np.ascontiguousarray(signs, dtype=np.int8)
+            keep.append(s)
+            sg = s.ctypes.data_as(C.POINTER(C.c_int8))
+        h = _vp()
+        _check(_lib.rot_plan_create(C.byref(h), self.K, m, rad, sp, nb, pp, sg))
+        self._h = h
+
+    @classmethod
+    def rht(cls, K: int, signs=None) -> "Plan":
+        """Randomized Hadamard transform of size K (power of two): radix-2 base mixers."""
+        n = int(K).bit_length() - 1
+        if (1 << n) != K:
+            raise ValueError("the randomized Hadamard transform needs a power-of-two K")
+        return cls(K, [2] * n, signs=signs)
+
+    @property
+    def handle(self):
+        return self._h
+
+    def info(self):
+        k, ch = _int(), _int()
+        _check(_lib.rot_plan_info(self._h, C.byref(k), C.byref(ch)))
+        return {"K": k.value, "chunk": ch.value}
+
+    def close(self):
+        if getattr(self, "_h", None) is not None and self._h.value:
+            _lib.rot_plan_destroy(self._h)
+            self._h = _vp()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def rot_apply(A, plan: Plan, *, inverse: bool = False, out=None, stream=None):
+    """y = T a (or T^T a) for every row of A (cuda bf16/fp32 [M, >=K]); fp32 [M, K] out."""
+    import torch
+    M = A.shape[0]
+    if out is None:
+        Kp = (plan.K + 3) // 4 * 4   # 16-byte aligned rows
+        out = torch.empty((M, Kp), dtype=torch.float32, device=A.device)[:, :plan.K]
+    _check(_lib.rot_apply(_ptr(A), _dtype_code(A), M, A.stride(0), plan.handle, int(inverse), _ptr(out),
+                          out.stride(0), _stream(stream)))
+    return out
+
+
+def rot_quant(A, plan: Plan, bits: int, G: int, *, codes=None, scales=None, stream=None):
+    """Fused rotate + group quantise + pack. Returns (codes uint8 [M, K*bits/8], scales fp16 [M, K/G])."""
+    import torch
+    M = A.shape[0]
+    K = plan.K
+    if codes is None:
+        codes = torch.empty((M, K * bits // 8), dtype=torch.uint8, device=A.device)
+    if scales is None:
+        scales = torch.empty((M, K // G), dtype=torch.float16, device=A.device)
+    _check(_lib.rot_quant(_ptr(A), _dtype_code(A), M, A.stride(0), plan.handle, bits, G, _ptr(codes),
+                          _ptr(scales), _stream(stream)))
+    return codes, scales
+
+
+def rot_dequant(codes, scales, plan: Plan, bits: int, G: int, *, inverse: bool = False, out=None, stream=None):
+    """x_hat = q * s (rotated basis) or T^T (q * s) (original basis); fp32 [M, K]."""
+    import torch
+    M = codes.shape[0]
+    if out is None:
+        out = torch.empty((M, plan.K), dtype=torch.float32, device=codes.device)
+    _check(_lib.rot_dequant(_ptr(codes), _ptr(scales), M, plan.handle, bits, G, int(inverse), _ptr(out),
+                            _stream(stream)))
+    return out
+
+
+def w4a4_linear(Aq, As, Wq, Ws, G: int, *, out_dtype=None, out=None, stream=None):
+    """C = sum_g sA sW (qA qW^T)_g for int4 codes Aq [M, K/2], Wq [N, K/2]; fp32 or bf16 [M, N]."""
+    import torch
+    M, N, K = Aq.shape[0], Wq.shape[0], Wq.shape[1] * 2
+    if out is None:
+        out = torch.empty((M, N), dtype=out_dtype or torch.float32, device=Wq.device)
+    cd = ROT_BF16 if out.dtype == torch.bfloat16 else ROT_F32
+    _check(_lib.w4a4_linear(_ptr(Aq), _ptr(As), _ptr(Wq), _ptr(Ws), M, N, K, G, _ptr(out), cd, _stream(stream)))
+    return out
+
+
+def w4a4_group_partials(Aq, Wq, G: int, *, out=None, stream=None):
+    """Exact int32 group sums P[m, n, g] of the W4A4 contraction."""
+    import torch
+    M, N, K = Aq.shape[0], Wq.shape[0], Wq.shape[1] * 2
+    if out is None:
+        out = torch.empty((M, N, K // G), dtype=torch.int32, device=Wq.device)
+    _check(_lib.w4a4_group_partials(_ptr(Aq), _ptr(Wq), M, N, K, G, _ptr(out), _stream(stream)))
+    return out
+
+
+def harp_givens_blocks(theta) -> np.ndarray:
+    """Host: R(theta) H_2 / sqrt(2) blocks, float32 [n, 2, 2]."""
+    th = np.ascontiguousarray(theta, dtype=np.float64)
+    out = np.empty((th.size, 2, 2), dtype=np.float32)
+    _check(_lib.rot_harp_givens_blocks(th.ctypes.data_as(C.POINTER(C.c_double)), th.size,
+                                       out.ctypes.data_as(C.POINTER(C.c_float))))
+    return out
+
+
+def harp_qr_block(g) -> np.ndarray:
+    """Host: Q factor (diag(R) > 0) of a square matrix, float32 [b, b]."""
+    a = np.ascontiguousarray(g, dtype=np.float64)
+    b = a.shape[0]
+    out = np.empty((b, b), dtype=np.float32)
+    _check(_lib.rot_harp_qr_block(a.ctypes.data_as(C.POINTER(C.c_double)), b,
+                                  out.ctypes.data_as(C.POINTER(C.c_float))))
+    return out
+
+
+def harp_plan(draws, signs, variant: str) -> Plan:
+    """Plan for a HARP processor built from seeded draws (``workloads.harp_draws``).
+
+    variant: ``random`` (Givens blocks per block from the angles, QR blocks from the
+    Gaussians, the drawn permutations), ``init_identity`` (theta = 0, identity for
+    non-power-of-two radices, no permutations) or ``init_qr`` (theta = 0, QR fallback
+    mixer for non-power-of-two radices).
+    """
+    radices = list(draws.radices)
+    K = int(np.prod(radices))
+    params = []
+    for t, b in enumerate(radices):
+        if variant == "random":
+            if b == 2:
+                params.append(harp_givens_blocks(draws.angles[t]))
+            else:
+                params.append(np.stack([harp_qr_block(gm) for gm in draws.gaussians[t]]))
+        elif variant == "init_identity":
+            params.append(None)
+        elif variant == "init_qr":
+            params.append(None if (b & (b - 1)) == 0 else harp_qr_block(draws.gaussians[t][0])[None])
+        else:
+            raise ValueError(variant)
+    perms = list(draws.perms) if variant == "random" else None
+    return Plan(K, radices, params, perms, signs)
+
+
+def check_device():
+    """Synchronise and raise if a bounded device wait gave up since the last check."""
+    _check(_lib.rot_check_device())

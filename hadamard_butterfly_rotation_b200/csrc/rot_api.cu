@@ -1,0 +1,115 @@
+// C-ABI entry points: argument validation and dispatch to the kernels.
+#include <cstdint>
+
+#include "rot_internal.cuh"
+
+using namespace rotb;
+
+namespace {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+rot_status check_plan(rot_plan_t plan, const char* fn) {
+  if (!plan) return set_error(ROT_EINVAL, std::string(fn) + ": plan is NULL");
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev != plan->device) return set_error(ROT_EINVAL, std::string(fn) + ": plan belongs to another device");
+  return ROT_OK;
+}
+
+rot_status check_rows(const void* A, int a_dtype, int64_t M, int64_t lda, int K, const char* fn) {
+  if (a_dtype != ROT_F32 && a_dtype != ROT_BF16) return set_error(ROT_EINVAL, std::string(fn) + ": a_dtype must be ROT_F32 or ROT_BF16");
+  if (M < 0) return set_error(ROT_EINVAL, std::string(fn) + ": M < 0");
+  if (M == 0) return ROT_OK;
+  if (!A) return set_error(ROT_EINVAL, std::string(fn) + ": A is NULL");
+  const int es = a_dtype == ROT_BF16 ? 2 : 4;
+  if (lda < K) return set_error(ROT_EINVAL, std::string(fn) + ": lda < K");
+  if (!aligned16(A) || (lda * es) % 16 != 0)
+    return set_error(ROT_EINVAL, std::string(fn) + ": A must be 16-byte aligned and lda*sizeof a multiple of 16");
+  return ROT_OK;
+}
+
+rot_status check_quant(int K, int bits, int G, const char* fn) {
+  if (bits != 4 && bits != 2) return set_error(ROT_EINVAL, std::string(fn) + ": bits must be 4 or 2");
+  const int cpw = 32 / bits;
+  if (G <= 0 || K % G != 0 || G % (bits == 4 ? 8 : 16) != 0)
+    return set_error(ROT_EINVAL, std::string(fn) + ": G must divide K and be a multiple of 8 (int4) / 16 (int2)");
+  if (K % cpw != 0) return set_error(ROT_EINVAL, std::string(fn) + ": K must be a multiple of the codes per word");
+  return ROT_OK;
+}
+
+}  // namespace
+
+extern "C" rot_status rot_apply(const void* A, int a_dtype, int64_t M, int64_t lda, rot_plan_t plan,
+                                int inverse, float* Y, int64_t ldy, void* stream) {
+  rot_status st = check_plan(plan, "rot_apply");
+  if (st) return st;
+  if ((st = check_rows(A, a_dtype, M, lda, plan->K, "rot_apply"))) return st;
+  if (M == 0) return ROT_OK;
+  if (!Y || !aligned16(Y) || ldy < plan->K || (ldy * 4) % 16 != 0)
+    return set_error(ROT_EINVAL, "rot_apply: Y must be 16-byte aligned with ldy >= K, ldy*4 % 16 == 0");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (plan->chunk_log2 >= 5) return fwht_apply(plan, A, a_dtype, M, lda, inverse, Y, ldy, s);
+  return stages_apply(plan, A, a_dtype, M, lda, inverse, Y, ldy, s);
+}
+
+extern "C" rot_status rot_quant(const void* A, int a_dtype, int64_t M, int64_t lda, rot_plan_t plan,
+                                int bits, int G, uint8_t* codes, uint16_t* scales, void* stream) {
+  rot_status st = check_plan(plan, "rot_quant");
+  if (st) return st;
+  if ((st = check_rows(A, a_dtype, M, lda, plan->K, "rot_quant"))) return st;
+  if ((st = check_quant(plan->K, bits, G, "rot_quant"))) return st;
+  if (M == 0) return ROT_OK;
+  if (!codes || !scales || !aligned16(codes) || !aligned16(scales))
+    return set_error(ROT_EINVAL, "rot_quant: codes and scales must be non-NULL and 16-byte aligned");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (fwht_quant_supported(plan, bits, G)) return fwht_quant(plan, A, a_dtype, M, lda, bits, G, codes, scales, s);
+  return stages_quant(plan, A, a_dtype, M, lda, bits, G, codes, scales, s);
+}
+
+extern "C" rot_status rot_dequant(const uint8_t* codes, const uint16_t* scales, int64_t M, rot_plan_t plan,
+                                  int bits, int G, int inverse, float* out, void* stream) {
+  rot_status st = check_plan(plan, "rot_dequant");
+  if (st) return st;
+  if ((st = check_quant(plan->K, bits, G, "rot_dequant"))) return st;
+  if (M < 0) return set_error(ROT_EINVAL, "rot_dequant: M < 0");
+  if (M == 0) return ROT_OK;
+  if (!codes || !scales || !out || !aligned16(codes) || !aligned16(out))
+    return set_error(ROT_EINVAL, "rot_dequant: pointers must be non-NULL, codes/out 16-byte aligned");
+  if ((plan->K * 4) % 16 != 0) return set_error(ROT_EINVAL, "rot_dequant: K*4 must be a multiple of 16");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if ((st = dequant_launch(codes, scales, M, plan->K, bits, G, out, s))) return st;
+  if (!inverse) return ROT_OK;
+  if (plan->chunk_log2 >= 5) return fwht_apply(plan, out, ROT_F32, M, plan->K, 1, out, plan->K, s);
+  return stages_apply(plan, out, ROT_F32, M, plan->K, 1, out, plan->K, s);
+}
+
+static rot_status check_w4a4(const uint8_t* Aq, const uint8_t* Wq, int64_t M, int64_t N, int64_t K, int G,
+                             const char* fn) {
+  if (M < 0 || N <= 0 || K <= 0) return set_error(ROT_EINVAL, std::string(fn) + ": need M >= 0, N > 0, K > 0");
+  if (G <= 0 || K % G != 0 || G % 32 != 0 || K % 64 != 0 || N % 16 != 0)
+    return set_error(ROT_EINVAL, std::string(fn) + ": need K % G == 0, G % 32 == 0, K % 64 == 0, N % 16 == 0");
+  if ((M > 0 && (!Aq || !aligned16(Aq))) || !Wq || !aligned16(Wq))
+    return set_error(ROT_EINVAL, std::string(fn) + ": Aq / Wq must be non-NULL and 16-byte aligned");
+  return ROT_OK;
+}
+
+extern "C" rot_status w4a4_linear(const uint8_t* Aq, const uint16_t* As, const uint8_t* Wq,
+                                  const uint16_t* Ws, int64_t M, int64_t N, int64_t K, int G, void* C,
+                                  int c_dtype, void* stream) {
+  rot_status st = check_w4a4(Aq, Wq, M, N, K, G, "w4a4_linear");
+  if (st) return st;
+  if (c_dtype != ROT_F32 && c_dtype != ROT_BF16) return set_error(ROT_EINVAL, "w4a4_linear: c_dtype must be ROT_F32 or ROT_BF16");
+  if (M == 0) return ROT_OK;
+  if (!As || !Ws || !C || !aligned16(C)) return set_error(ROT_EINVAL, "w4a4_linear: As, Ws, C must be non-NULL, C 16-byte aligned");
+  return w4a4_launch(Aq, As, Wq, Ws, M, N, K, G, C, c_dtype, nullptr, static_cast<cudaStream_t>(stream));
+}
+
+extern "C" rot_status w4a4_group_partials(const uint8_t* Aq, const uint8_t* Wq, int64_t M, int64_t N,
+                                          int64_t K, int G, int32_t* P, void* stream) {
+  rot_status st = check_w4a4(Aq, Wq, M, N, K, G, "w4a4_group_partials");
+  if (st) return st;
+  if (M == 0) return ROT_OK;
+  if (!P || !aligned16(P)) return set_error(ROT_EINVAL, "w4a4_group_partials: P must be non-NULL and 16-byte aligned");
+  return w4a4_launch(Aq, nullptr, Wq, nullptr, M, N, K, G, nullptr, ROT_F32, P, static_cast<cudaStream_t>(stream));
+}

@@ -1,0 +1,460 @@
+// Fused signed Walsh-Hadamard rotation (+ group quantisation + packing), one HBM pass.
+//
+// Computes, for every contiguous chunk of N = 2^n coordinates of every row,
+//     y = H_N D x / sqrt(N)
+// (the randomized Hadamard transform: random signs, fast Walsh-Hadamard transform,
+// times 1/sqrt(N) [Hadamard-Int4-Accuracy wiki, Method: fwht_norm; HARP abstract]),
+// then optionally the per-group symmetric absmax quantisation of y with fp16 scales and
+// two's-complement packing [same wiki, Method: q_dequant_vec].
+//
+// Work decomposition (sm_100a): a chunk is owned by TPC = 2^(n-e) consecutive threads
+// of one warp (or two warps for n = 13), each holding E = 2^e values in registers.
+//   phase A  thread t holds coordinates lo + (t << VA) + (hi << e), lo < 2^VA, hi < 2^(n-e)
+//            (VA = 2e - n): contiguous runs of 2^VA elements, read straight from HBM with
+//            vector loads that are coalesced across the chunk's threads; the e butterfly
+//            stages over these register bits run in registers.
+//   transpose through shared memory (fp32, XOR-swizzled 16-byte chunks: conflict-free
+//            stores and loads).
+//   phase B  thread t holds the contiguous coordinates (t << e) + j, j < E; the remaining
+//            n - e stages (register bits VA..e-1) run in registers, with packed
+//            add/sub.f32x2. Quantisation then sees whole groups (or group fragments
+//            reduced with warp shuffles) in contiguous registers and writes packed codes
+//            and scales with vector stores.
+// Scaling by 1/sqrt(N) is folded into the output (apply) or into the group factor (quant).
+#include <cmath>
+
+#include "rot_internal.cuh"
+
+namespace rotb {
+namespace {
+
+template <int LOGN>
+struct Cfg {
+  static constexpr int N = 1 << LOGN;
+  static constexpr int ELOG = LOGN <= 7 ? LOGN : (LOGN == 8 ? 5 : (LOGN == 9 ? 6 : 7));
+  static constexpr int E = 1 << ELOG;
+  static constexpr int HB = LOGN - ELOG;   // thread bits (= high register bits of phase A)
+  static constexpr int VA = ELOG - HB;     // contiguous run bits of phase A
+  static constexpr int TPC = 1 << HB;      // threads per chunk
+  static constexpr int NV = 1 << VA;       // run length
+  static constexpr int NH = 1 << HB;       // runs per thread
+  static constexpr int THREADS = LOGN <= 7 ? 256 : (LOGN == 8 ? 768 : (LOGN == 9 ? 512 : 384));
+  static constexpr int SLOTS = THREADS / TPC;
+  static constexpr int SSTRIDE = N + 4;    // floats per slot buffer (16-byte pad)
+  static_assert(VA >= 1, "phase A needs element pairs");
+};
+
+// Physical float index of chunk-local coordinate i in a slot buffer.
+template <int LOGN>
+__device__ __forceinline__ int swz(int i) {
+  constexpr int ELOG = Cfg<LOGN>::ELOG;
+  int x = ((i >> ELOG) & 7) << 2;
+  if (LOGN == 9 || LOGN == 10 || LOGN == 11) x ^= ((i >> 5) & 1) << 2;
+  if (LOGN == 10) x ^= ((i >> 6) & 1) << 3;
+  return i ^ x;
+}
+
+struct Args {
+  const void* A;
+  int64_t lda;
+  int64_t M;
+  int chunks;       // chunks per row (K / N)
+  int K;
+  const uint32_t* signmask;  // K/2 words or nullptr
+  float* Y;
+  int64_t ldy;
+  uint8_t* codes;
+  uint16_t* scales;
+  int G;
+  float norm;
+};
+
+enum { MODE_APPLY = 0, MODE_APPLY_INV = 1, MODE_QUANT = 2 };
+
+
+// NW consecutive sign-mask words starting at word w0 (w0 a multiple of NW), vector loads.
+template <int NW>
+__device__ __forceinline__ void load_masks(uint32_t (&m)[NW], const uint32_t* smask, int w0, bool on) {
+  if (!on) {
+#pragma unroll
+    for (int w = 0; w < NW; ++w) m[w] = 0u;
+    return;
+  }
+  if constexpr (NW >= 4) {
+#pragma unroll
+    for (int v = 0; v < NW / 4; ++v) {
+      const uint4 q = reinterpret_cast<const uint4*>(smask + w0)[v];
+      m[4 * v] = q.x; m[4 * v + 1] = q.y; m[4 * v + 2] = q.z; m[4 * v + 3] = q.w;
+    }
+  } else if constexpr (NW == 2) {
+    const uint2 q = *reinterpret_cast<const uint2*>(smask + w0);
+    m[0] = q.x; m[1] = q.y;
+  } else {
+    m[0] = smask[w0];
+  }
+}
+
+// Lanes of this thread's slot within its warp.
+template <int TPC>
+__device__ __forceinline__ unsigned slot_lanes() {
+  if constexpr (TPC >= 32) {
+    return 0xffffffffu;
+  } else {
+    const unsigned lane = threadIdx.x & 31;
+    return ((1u << TPC) - 1u) << (lane & ~(TPC - 1));
+  }
+}
+
+template <int TPC>
+__device__ __forceinline__ void slot_sync(int slot) {
+  if constexpr (TPC > 32) {
+    asm volatile("bar.sync %0, %1;" ::"r"(1 + slot), "r"(TPC) : "memory");
+  } else if constexpr (TPC > 1) {
+    __syncwarp(slot_lanes<TPC>());
+  }
+}
+
+__device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+// Pack 8 offset codes (low bytes of t[0..7], each 8 + q) into one int4 word.
+__device__ __forceinline__ uint32_t pack8_int4(const uint32_t (&t)[8]) {
+  uint32_t ev = prmt(prmt(t[0], t[2], 0x0040u), prmt(t[4], t[6], 0x4000u), 0x7610u);
+  uint32_t od = prmt(prmt(t[1], t[3], 0x0040u), prmt(t[5], t[7], 0x4000u), 0x7610u);
+  return ((od << 4) + ev) ^ 0x88888888u;
+}
+// Pack 16 offset codes (each 2 + q) into one int2 word.
+__device__ __forceinline__ uint32_t pack16_int2(const uint32_t (&t)[16]) {
+  uint32_t b[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    b[i] = prmt(prmt(t[i], t[4 + i], 0x0040u), prmt(t[8 + i], t[12 + i], 0x4000u), 0x7610u);
+  return (b[0] + (b[1] << 2) + (b[2] << 4) + (b[3] << 6)) ^ 0xAAAAAAAAu;
+}
+
+template <int LOGN, bool BF16, int MODE, int BITS>
+__global__ void __launch_bounds__(Cfg<LOGN>::THREADS, 1) fwht_kernel(const Args a) {
+  using C = Cfg<LOGN>;
+  constexpr int N = C::N, ELOG = C::ELOG, E = C::E, HB = C::HB, VA = C::VA, TPC = C::TPC;
+  constexpr int NV = C::NV, NH = C::NH, SLOTS = C::SLOTS, SSTRIDE = C::SSTRIDE;
+  extern __shared__ __align__(16) float smem[];
+  float* sbuf = smem;
+  uint32_t* smask = reinterpret_cast<uint32_t*>(smem + (HB > 0 ? SLOTS * SSTRIDE : 0));
+
+  const bool has_signs = a.signmask != nullptr;
+  if (has_signs) {
+    for (int i = threadIdx.x; i < a.K / 2; i += C::THREADS) smask[i] = a.signmask[i];
+  }
+  __syncthreads();
+
+  const int slot = threadIdx.x / TPC;
+  const int t = threadIdx.x % TPC;
+  float* buf = sbuf + slot * SSTRIDE;
+  const int64_t units = a.M * a.chunks;
+
+  for (int64_t u = (int64_t)blockIdx.x * SLOTS + slot; u < units; u += (int64_t)gridDim.x * SLOTS) {
+    const int64_t row = u / a.chunks;
+    const int cbase = (int)(u - row * a.chunks) * N;
+    float x[E];
+
+    // ---------------- phase A: load runs, apply signs, convert to fp32
+    {
+      const int run0 = cbase + (t << VA);
+      if constexpr (BF16) {
+        const __nv_bfloat16* src = static_cast<const __nv_bfloat16*>(a.A) + row * a.lda + run0;
+        constexpr int NW = NV / 2;  // 32-bit words per run
+        uint32_t raw[NH][NW];
+#pragma unroll
+        for (int h = 0; h < NH; ++h) {
+          const uint32_t* p = reinterpret_cast<const uint32_t*>(src + (h << ELOG));
+          if constexpr (NW >= 4) {
+#pragma unroll
+            for (int v = 0; v < NW / 4; ++v) {
+              uint4 q = __ldcs(reinterpret_cast<const uint4*>(p) + v);
+              raw[h][4 * v] = q.x; raw[h][4 * v + 1] = q.y; raw[h][4 * v + 2] = q.z; raw[h][4 * v + 3] = q.w;
+            }
+          } else if constexpr (NW == 2) {
+            uint2 q = __ldcs(reinterpret_cast<const uint2*>(p));
+            raw[h][0] = q.x; raw[h][1] = q.y;
+          } else {
+            raw[h][0] = __ldcs(p);
+          }
+        }
+#pragma unroll
+        for (int h = 0; h < NH; ++h) {
+          uint32_t m[NW];
+          load_masks<NW>(m, smask, (run0 + (h << ELOG)) >> 1, MODE != MODE_APPLY_INV && has_signs);
+#pragma unroll
+          for (int w = 0; w < NW; ++w) {
+            const uint32_t v = raw[h][w] ^ m[w];
+            x[h * NV + 2 * w] = bf16lo(v);
+            x[h * NV + 2 * w + 1] = bf16hi(v);
+          }
+        }
+      } else {
+        const float* src = static_cast<const float*>(a.A) + row * a.lda + run0;
+#pragma unroll
+        for (int h = 0; h < NH; ++h) {
+          const float* p = src + (h << ELOG);
+          if constexpr (NV >= 4) {
+#pragma unroll
+            for (int v = 0; v < NV / 4; ++v) {
+              float4 q = __ldcs(reinterpret_cast<const float4*>(p) + v);
+              x[h * NV + 4 * v] = q.x; x[h * NV + 4 * v + 1] = q.y;
+              x[h * NV + 4 * v + 2] = q.z; x[h * NV + 4 * v + 3] = q.w;
+            }
+          } else {
+            float2 q = __ldcs(reinterpret_cast<const float2*>(p));
+            x[h * NV] = q.x; x[h * NV + 1] = q.y;
+          }
+        }
+        if (MODE != MODE_APPLY_INV && has_signs) {
+#pragma unroll
+          for (int h = 0; h < NH; ++h) {
+            uint32_t m[NV / 2];
+            load_masks<NV / 2>(m, smask, (run0 + (h << ELOG)) >> 1, true);
+#pragma unroll
+            for (int w = 0; w < NV / 2; ++w) {
+              x[h * NV + 2 * w] = __uint_as_float(__float_as_uint(x[h * NV + 2 * w]) ^ (m[w] << 16));
+              x[h * NV + 2 * w + 1] = __uint_as_float(__float_as_uint(x[h * NV + 2 * w + 1]) ^ (m[w] & 0x80000000u));
+            }
+          }
+        }
+      }
+    }
+
+    // ---------------- phase A butterflies over all E register bits
+#pragma unroll
+    for (int r = 0; r < E; r += 2) {
+      const float p = x[r], q = x[r + 1];
+      x[r] = p + q;
+      x[r + 1] = p - q;
+    }
+#pragma unroll
+    for (int h = 2; h < E; h <<= 1) {
+#pragma unroll
+      for (int r = 0; r < E; r += 2)
+        if (!(r & h)) bfly_x2(x[r], x[r + 1], x[r + h], x[r + h + 1]);
+    }
+
+    // ---------------- transpose to phase B and remaining stages
+    if constexpr (HB > 0) {
+      slot_sync<TPC>(slot);  // previous unit's phase-B reads are done
+#pragma unroll
+      for (int h = 0; h < NH; ++h) {
+        const int i0 = (t << VA) + (h << ELOG);
+        if constexpr (NV >= 4) {
+#pragma unroll
+          for (int v = 0; v < NV / 4; ++v)
+            *reinterpret_cast<float4*>(buf + swz<LOGN>(i0 + 4 * v)) =
+                make_float4(x[h * NV + 4 * v], x[h * NV + 4 * v + 1], x[h * NV + 4 * v + 2], x[h * NV + 4 * v + 3]);
+        } else {
+          *reinterpret_cast<float2*>(buf + swz<LOGN>(i0)) = make_float2(x[h * NV], x[h * NV + 1]);
+        }
+      }
+      slot_sync<TPC>(slot);
+#pragma unroll
+      for (int jc = 0; jc < E / 4; ++jc) {
+        const float4 q = *reinterpret_cast<const float4*>(buf + swz<LOGN>((t << ELOG) + 4 * jc));
+        x[4 * jc] = q.x; x[4 * jc + 1] = q.y; x[4 * jc + 2] = q.z; x[4 * jc + 3] = q.w;
+      }
+#pragma unroll
+      for (int h = NV; h < E; h <<= 1) {
+#pragma unroll
+        for (int r = 0; r < E; r += 2)
+          if (!(r & h)) bfly_x2(x[r], x[r + 1], x[r + h], x[r + h + 1]);
+      }
+    }
+
+    // x[j] = z for chunk coordinate (t << ELOG) + j; y = z * norm
+    const int c0 = cbase + (t << ELOG);  // row coordinate of x[0]
+    if constexpr (MODE == MODE_APPLY || MODE == MODE_APPLY_INV) {
+      float* dst = a.Y + row * a.ldy + c0;
+#pragma unroll
+      for (int jc = 0; jc < E / 4; ++jc) {
+        float4 q = make_float4(x[4 * jc] * a.norm, x[4 * jc + 1] * a.norm, x[4 * jc + 2] * a.norm,
+                               x[4 * jc + 3] * a.norm);
+        if (MODE == MODE_APPLY_INV && has_signs) {
+          const uint32_t m0 = smask[(c0 >> 1) + 2 * jc], m1 = smask[(c0 >> 1) + 2 * jc + 1];
+          q.x = __uint_as_float(__float_as_uint(q.x) ^ ((m0 << 16) & 0x80000000u));
+          q.y = __uint_as_float(__float_as_uint(q.y) ^ (m0 & 0x80000000u));
+          q.z = __uint_as_float(__float_as_uint(q.z) ^ ((m1 << 16) & 0x80000000u));
+          q.w = __uint_as_float(__float_as_uint(q.w) ^ (m1 & 0x80000000u));
+        }
+        *reinterpret_cast<float4*>(dst + 4 * jc) = q;
+      }
+    } else {
+      // ---------------- quantisation: groups of G contiguous coordinates.
+      // Absmax per granule of 8 registers, then a predicated tree over granules for the
+      // runtime group size (G/8 granules), then warp shuffles when a group spans threads.
+      constexpr float QMAX = BITS == 4 ? 7.0f : 1.0f;
+      constexpr float MAGIC = BITS == 4 ? 8388616.0f : 8388610.0f;  // 2^23 + qmax + 1
+      constexpr int NG = E / 8;
+      const int G = a.G;
+      const int gg = G >> 3;  // granules per group (power of two)
+      float gm[NG];
+#pragma unroll
+      for (int i = 0; i < NG; ++i) {
+        float m = fmaxf(fabsf(x[8 * i]), fabsf(x[8 * i + 1]));
+        m = max3(m, fabsf(x[8 * i + 2]), fabsf(x[8 * i + 3]));
+        m = max3(m, fabsf(x[8 * i + 4]), fabsf(x[8 * i + 5]));
+        gm[i] = max3(m, fabsf(x[8 * i + 6]), fabsf(x[8 * i + 7]));
+      }
+#pragma unroll
+      for (int st = 1; st < NG; st <<= 1) {
+        if (st < gg) {
+#pragma unroll
+          for (int i = 0; i + st < NG; i += 2 * st) gm[i] = fmaxf(gm[i], gm[i + st]);
+        }
+      }
+      if (G > E) {
+        const unsigned lanes = slot_lanes<TPC>();
+        for (int o = 1; o < G / E; o <<= 1) gm[0] = fmaxf(gm[0], __shfl_xor_sync(lanes, gm[0], o));
+      }
+      float fw[NG];
+      bool slow[NG];
+      uint16_t sc[NG];
+#pragma unroll
+      for (int i = 0; i < NG; ++i) {
+        if ((i & (gg - 1)) == 0) {
+          sc[i] = group_scale(gm[i], a.norm, QMAX, &fw[i], &slow[i]);
+        } else {
+          fw[i] = fw[i - 1];
+          slow[i] = slow[i - 1];
+          sc[i] = sc[i - 1];
+        }
+      }
+      // scales: one binary16 per group
+      {
+        const int64_t ngr = a.K / G;
+        uint16_t* srow = a.scales + row * ngr;
+        if (G > E) {
+          if ((t & (G / E - 1)) == 0) srow[c0 / G] = sc[0];
+        } else {
+#pragma unroll
+          for (int i = 0; i < NG; ++i)
+            if ((i & (gg - 1)) == 0) srow[(c0 + 8 * i) / G] = sc[i];
+        }
+      }
+      // codes
+      constexpr int CPW = 32 / BITS;   // codes per 32-bit word
+      constexpr int NWD = E / CPW;     // words per thread
+      uint32_t words[NWD];
+#pragma unroll
+      for (int w = 0; w < NWD; ++w) {
+        const int gi = w * (CPW / 8);    // granule of the word's first code
+        uint32_t tt[CPW];
+        if (!slow[gi]) {
+#pragma unroll
+          for (int j = 0; j < CPW; ++j) tt[j] = code_magic(x[CPW * w + j], fw[gi], MAGIC);
+        } else {
+#pragma unroll
+          for (int j = 0; j < CPW; ++j) tt[j] = code_magic_clamped(x[CPW * w + j], fw[gi], QMAX, MAGIC);
+        }
+        if constexpr (BITS == 4) {
+          words[w] = pack8_int4(*reinterpret_cast<const uint32_t(*)[8]>(tt));
+        } else {
+          words[w] = pack16_int2(*reinterpret_cast<const uint32_t(*)[16]>(tt));
+        }
+      }
+      uint32_t* dst = reinterpret_cast<uint32_t*>(a.codes + row * (int64_t)(a.K / CPW) * 4) + c0 / CPW;
+      if constexpr (NWD >= 4) {
+#pragma unroll
+        for (int v = 0; v < NWD / 4; ++v)
+          reinterpret_cast<uint4*>(dst)[v] = make_uint4(words[4 * v], words[4 * v + 1], words[4 * v + 2], words[4 * v + 3]);
+      } else if constexpr (NWD == 2) {
+        *reinterpret_cast<uint2*>(dst) = make_uint2(words[0], words[1]);
+      } else {
+        dst[0] = words[0];
+      }
+    }
+  }
+}
+
+template <int LOGN, bool BF16, int MODE, int BITS>
+rot_status launch_one(const Args& a, cudaStream_t s) {
+  using C = Cfg<LOGN>;
+  const size_t smem = (C::HB > 0 ? (size_t)C::SLOTS * C::SSTRIDE * 4 : 0) + (size_t)(a.K / 2) * 4;
+  if (smem > 227 * 1024) return set_error(ROT_EUNSUPPORTED, "fused rotation: sign table too large for shared memory");
+  auto kern = fwht_kernel<LOGN, BF16, MODE, BITS>;
+  static int configured[64] = {0};  // per device: the opt-in limit is set once
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !configured[dev]) {
+    ROT_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024));
+    configured[dev] = 1;
+  }
+  const int64_t units = a.M * a.chunks;
+  int64_t grid = (units + C::SLOTS - 1) / C::SLOTS;
+  const int64_t cap = (int64_t)sm_count();
+  if (grid > cap) grid = cap;
+  if (grid < 1) return ROT_OK;
+  kern<<<(unsigned)grid, C::THREADS, smem, s>>>(a);
+  ROT_CUDA_TRY(cudaGetLastError());
+  return ROT_OK;
+}
+
+template <bool BF16, int MODE, int BITS>
+rot_status dispatch_logn(int logn, const Args& a, cudaStream_t s) {
+  switch (logn) {
+    case 5: return launch_one<5, BF16, MODE, BITS>(a, s);
+    case 6: return launch_one<6, BF16, MODE, BITS>(a, s);
+    case 7: return launch_one<7, BF16, MODE, BITS>(a, s);
+    case 8: return launch_one<8, BF16, MODE, BITS>(a, s);
+    case 9: return launch_one<9, BF16, MODE, BITS>(a, s);
+    case 10: return launch_one<10, BF16, MODE, BITS>(a, s);
+    case 11: return launch_one<11, BF16, MODE, BITS>(a, s);
+    case 12: return launch_one<12, BF16, MODE, BITS>(a, s);
+    case 13: return launch_one<13, BF16, MODE, BITS>(a, s);
+    default: return set_error(ROT_EUNSUPPORTED, "fused rotation: chunk size out of range");
+  }
+}
+
+Args make_args(const rot_plan_s* p, const void* A, int64_t M, int64_t lda) {
+  Args a{};
+  a.A = A;
+  a.lda = lda;
+  a.M = M;
+  a.K = p->K;
+  a.chunks = p->K >> p->chunk_log2;
+  a.signmask = p->has_signs ? p->d_signmask : nullptr;
+  a.norm = (float)(1.0 / std::sqrt((double)(1 << p->chunk_log2)));
+  return a;
+}
+
+}  // namespace
+
+bool fwht_quant_supported(const rot_plan_s* p, int bits, int G) {
+  if (p->chunk_log2 < 5) return false;
+  const int N = 1 << p->chunk_log2;
+  if (G < 8 || (G & (G - 1)) != 0 || G > N) return false;
+  if (bits == 2 && G < 16) return false;
+  int e = p->chunk_log2 <= 7 ? p->chunk_log2 : (p->chunk_log2 == 8 ? 5 : (p->chunk_log2 == 9 ? 6 : 7));
+  if (G > (1 << e) && G / (1 << e) > 32) return false;
+  return true;
+}
+
+rot_status fwht_apply(const rot_plan_s* p, const void* A, int a_dtype, int64_t M, int64_t lda,
+                      int inverse, float* Y, int64_t ldy, cudaStream_t s) {
+  Args a = make_args(p, A, M, lda);
+  a.Y = Y;
+  a.ldy = ldy;
+  const int n = p->chunk_log2;
+  if (a_dtype == ROT_BF16)
+    return inverse ? dispatch_logn<true, MODE_APPLY_INV, 4>(n, a, s) : dispatch_logn<true, MODE_APPLY, 4>(n, a, s);
+  return inverse ? dispatch_logn<false, MODE_APPLY_INV, 4>(n, a, s) : dispatch_logn<false, MODE_APPLY, 4>(n, a, s);
+}
+
+rot_status fwht_quant(const rot_plan_s* p, const void* A, int a_dtype, int64_t M, int64_t lda, int bits,
+                      int G, uint8_t* codes, uint16_t* scales, cudaStream_t s) {
+  Args a = make_args(p, A, M, lda);
+  a.codes = codes;
+  a.scales = scales;
+  a.G = G;
+  const int n = p->chunk_log2;
+  if (a_dtype == ROT_BF16)
+    return bits == 4 ? dispatch_logn<true, MODE_QUANT, 4>(n, a, s) : dispatch_logn<true, MODE_QUANT, 2>(n, a, s);
+  return bits == 4 ? dispatch_logn<false, MODE_QUANT, 4>(n, a, s) : dispatch_logn<false, MODE_QUANT, 2>(n, a, s);
+}
+
+}  // namespace rotb

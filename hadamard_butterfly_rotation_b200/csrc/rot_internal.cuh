@@ -1,0 +1,129 @@
+// Internal declarations shared by the library's translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include <cstdint>
+#include <string>
+#include <vector>
+
+#include "rot_b200.h"
+
+namespace rotb {
+
+// ---------------------------------------------------------------- errors (host)
+rot_status set_error(rot_status st, const std::string& msg);
+rot_status cuda_error(cudaError_t e, const char* what);
+#define ROT_CUDA_TRY(expr)                                   \
+  do {                                                       \
+    cudaError_t _e = (expr);                                 \
+    if (_e != cudaSuccess) return ::rotb::cuda_error(_e, #expr); \
+  } while (0)
+
+int sm_count();  // SMs of the current device (cached per device)
+
+// ---------------------------------------------------------------- plan
+struct Stage {
+  int b = 0;            // radix
+  int stride = 1;       // s_t = prod_{u<t} b_u
+  int64_t n_blocks = 0; // 1 or K/b (0 when the stage is the identity and skipped)
+  bool identity = false;
+  bool hadamard = false;  // blocks equal H_b / sqrt(b) (power-of-two b)
+  float* d_blocks = nullptr;   // [n_blocks, b, b] fp32 row-major (base mixer materialised)
+  int32_t* d_perm = nullptr;   // gather after the stage, or nullptr
+  int32_t* d_iperm = nullptr;  // inverse permutation (for T^T)
+};
+
+}  // namespace rotb
+
+struct rot_plan_s {
+  int K = 0;
+  int device = 0;
+  bool has_signs = false;
+  // fused butterfly path: T = blockdiag over K/chunk chunks of H_chunk D_c / sqrt(chunk)
+  int chunk_log2 = -1;          // >= 0 when the fused path applies, else -1
+  uint32_t* d_signmask = nullptr;  // K/2 words: bit 15 = sign of coord 2p, bit 31 = of 2p+1
+  float* d_signf = nullptr;        // K entries +-1.0f (generic stage kernel)
+  std::vector<rotb::Stage> stages;  // generic path (always built)
+  int max_radix = 0;
+};
+
+namespace rotb {
+
+// ---------------------------------------------------------------- launchers
+// fused butterfly path (rot_fwht.cu)
+rot_status fwht_apply(const rot_plan_s* p, const void* A, int a_dtype, int64_t M, int64_t lda,
+                      int inverse, float* Y, int64_t ldy, cudaStream_t s);
+rot_status fwht_quant(const rot_plan_s* p, const void* A, int a_dtype, int64_t M, int64_t lda,
+                      int bits, int G, uint8_t* codes, uint16_t* scales, cudaStream_t s);
+bool fwht_quant_supported(const rot_plan_s* p, int bits, int G);
+// generic stage path (rot_stages.cu)
+rot_status stages_apply(const rot_plan_s* p, const void* A, int a_dtype, int64_t M, int64_t lda,
+                        int inverse, float* Y, int64_t ldy, cudaStream_t s);
+rot_status stages_quant(const rot_plan_s* p, const void* A, int a_dtype, int64_t M, int64_t lda,
+                        int bits, int G, uint8_t* codes, uint16_t* scales, cudaStream_t s);
+// dequantisation (rot_dequant.cu)
+rot_status dequant_launch(const uint8_t* codes, const uint16_t* scales, int64_t M, int K, int bits,
+                          int G, float* out, cudaStream_t s);
+// W4A4 linear (w4a4_linear.cu)
+rot_status w4a4_launch(const uint8_t* Aq, const uint16_t* As, const uint8_t* Wq,
+                       const uint16_t* Ws, int64_t M, int64_t N, int64_t K, int G, void* C,
+                       int c_dtype, int32_t* partials, cudaStream_t s);
+
+// ---------------------------------------------------------------- device helpers
+#ifdef __CUDACC__
+// (a, b) <- (a + b, a - b) on two register pairs with packed fp32x2 adds
+__device__ __forceinline__ void bfly_x2(float& a0, float& a1, float& b0, float& b1) {
+  unsigned long long A, B, S, D;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(A) : "f"(a0), "f"(a1));
+  asm("mov.b64 %0, {%1, %2};" : "=l"(B) : "f"(b0), "f"(b1));
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(S) : "l"(A), "l"(B));
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(D) : "l"(A), "l"(B));
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a0), "=f"(a1) : "l"(S));
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(b0), "=f"(b1) : "l"(D));
+}
+
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// byte permute
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+  return d;
+}
+
+// Scale / code-factor of one quantisation group.
+//   m_z   : max |z| over the group, z the un-normalised rotated values (y = z * norm)
+// Returns the binary16 scale bits; *f receives the factor with v = z * f ~= y / s, nudged
+// up by 2^-22 relative so that exact ties of z * f round away from zero; *slow is set
+// when the scale is zero, subnormal or not finite (codes need clamping then).
+__device__ __forceinline__ uint16_t group_scale(float m_z, float norm, float qmax, float* f,
+                                                bool* slow) {
+  float my = m_z * norm;
+  __half s16 = __float2half_rn(__fdiv_rn(my, qmax));
+  float s = __half2float(s16);
+  bool ok = (s >= 6.103515625e-05f) && (s <= 65504.0f);  // normal binary16
+  float fv = (s > 0.0f && s <= 65504.0f) ? __fdiv_rn(norm, s) : 0.0f;
+  *f = __fmul_rn(fv, 1.0f + 0x1p-22f);
+  *slow = !ok;
+  return __half_as_ushort(s16);
+}
+
+// Offset code u = qmax + 1 + rne(v) in the low bits of the result (magic-number rounding);
+// with clamping for the slow path. v = z * f.
+__device__ __forceinline__ uint32_t code_magic(float z, float f, float magic) {
+  return __float_as_uint(__fmaf_rn(z, f, magic));
+}
+__device__ __forceinline__ uint32_t code_magic_clamped(float z, float f, float qmax, float magic) {
+  float v = fminf(fmaxf(__fmul_rn(z, f), -qmax), qmax);
+  return __float_as_uint(__fadd_rn(v, magic));
+}
+#endif
+
+}  // namespace rotb

@@ -1,0 +1,153 @@
+/*
+ * rot_b200.h -- C ABI of the B200 (sm_100a) rotation / group-quantisation / W4A4 library.
+ *
+ * The library implements the online hot path of rotation-based low-bit quantisation:
+ * each activation row a = A[m,:] is mapped to y = T a by an orthonormal rotation T,
+ * quantised in groups of G contiguous rotated coordinates with symmetric absmax
+ * scales, packed, and fed to a W4A4 linear whose weights went through the same T
+ * offline, so that A.B = (A.T^T)(T.B).
+ *
+ *   T = randomized Hadamard transform (RHT): random +-1 signs D, a fast Walsh-Hadamard
+ *       transform of size K, scaled by 1/sqrt(K)            [Hadamard-Int4-Accuracy wiki,
+ *       Hypothesis and Method (fwht_norm); HARP abstract and gist.science summary,
+ *       section 1]; or
+ *   T = HARP processor (P_{m-1} S_{m-1}) ... (P_0 S_0) D: a product of block-diagonal
+ *       orthogonal stages over a mixed-radix schedule prod b_t = K, with optional
+ *       permutations between stages                         [HARP gist.science summary,
+ *       sections 2.1 and 2.2; HARP abstract].
+ *
+ * Conventions shared by every call:
+ *   - Device pointers are caller-owned CUDA device memory on the device that is current
+ *     when the call is made (for rot_plan_create: the device the plan lives on). The
+ *     library never frees or keeps caller pointers.
+ *   - Calls that take a stream are asynchronous on that stream (a cudaStream_t passed as
+ *     void*, NULL = legacy default stream) and never synchronise; argument errors are
+ *     detected on the host and returned before any launch.
+ *   - Device pointers must be 16-byte aligned; leading dimensions are in elements and
+ *     lda * sizeof(element) must be a multiple of 16 bytes.
+ *   - Layouts (row-major):
+ *       activations  A      [M, lda]  bf16 or fp32
+ *       codes        uint8  [M, K*bits/8]  int4: byte j = q[2j] | q[2j+1] << 4
+ *                                          int2: byte j holds q[4j+i] in bits 2i..2i+1
+ *                           (two's complement, symmetric levels -qmax..qmax,
+ *                            qmax = 2^(bits-1) - 1)
+ *       scales       uint16 [M, K/G]  IEEE binary16 bit patterns, one per (row, group)
+ *   - Quantisation [Hadamard-Int4-Accuracy wiki, Method: q_dequant_vec]: per group
+ *       s = fp16_rn(fp32(max|y| / qmax)),  q = clamp(round_half_away(y / s), +-qmax),
+ *       s == 0 (or not finite) gives q = 0.
+ *   - On failure a call returns a non-zero rot_status and rot_last_error() (per host
+ *     thread) holds a one-line message.
+ */
+#ifndef ROT_B200_H
+#define ROT_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct rot_plan_s* rot_plan_t;
+
+typedef enum {
+  ROT_OK = 0,
+  ROT_EINVAL = 1,        /* invalid argument (shape, alignment, null pointer, bad plan) */
+  ROT_EUNSUPPORTED = 2,  /* valid but outside what this build implements */
+  ROT_ECUDA = 3,         /* a CUDA runtime call failed */
+  ROT_ETIMEOUT = 4,      /* a bounded device-side wait gave up (reported by rot_check_device) */
+  ROT_ENOMEM = 5         /* device allocation failed (plan creation only) */
+} rot_status;
+
+enum { ROT_F32 = 0, ROT_BF16 = 1 };
+
+/* Build a rotation plan and copy its parameters to the current device.
+ *
+ * Defines T = (P_{m-1} S_{m-1}) ... (P_0 S_0) D [HARP gist.science summary, 2.1-2.2].
+ *   K            dimension, K = prod radices[t]
+ *   n_stages     m >= 1
+ *   radices      host int[m], every b_t >= 2
+ *   stage_params host array of m pointers; stage_params[t] is NULL (base mixer:
+ *                H_b / sqrt(b) for a power-of-two b, the identity otherwise) or a host fp32
+ *                array of n_blocks[t] * b * b row-major b x b orthogonal blocks
+ *   n_blocks     host int64[m] (may be NULL when every stage_params[t] is NULL):
+ *                1 (one block shared by the stage) or K / b_t (block c for coordinates
+ *                base + r * s_t, s_t = prod_{u<t} b_u, c = low + high * s_t where low/high
+ *                are the digits below/above t)
+ *   perms        NULL or host array of m pointers; perms[t] NULL or a host int32[K]
+ *                permutation applied after stage t as a gather x''[j] = x'[P_t[j]]
+ *   signs        NULL (all +1) or host int8[K] with entries +1 / -1 (the D of the RHT)
+ * The RHT of size K is radices = {2, ..., 2}, stage_params all NULL, signs = the random
+ * signs. Host arrays are copied; the caller may free them after the call.
+ * Errors: ROT_EINVAL (product != K, radix < 2, n_blocks not 1 or K/b, perms not a
+ * permutation, signs not +-1), ROT_ENOMEM, ROT_ECUDA. */
+rot_status rot_plan_create(rot_plan_t* out, int K, int n_stages, const int* radices,
+                           const float* const* stage_params, const int64_t* n_blocks,
+                           const int32_t* const* perms, const int8_t* signs);
+
+/* Release a plan's device memory (synchronises the device). NULL is accepted. */
+rot_status rot_plan_destroy(rot_plan_t plan);
+
+/* Which kernel a plan uses: *chunk = 2^n > 0 when T acts as independent signed
+ * Walsh-Hadamard transforms on contiguous chunks of 2^n coordinates (the fused
+ * butterfly kernel), 0 when the generic stage kernel runs. *K receives the plan's K. */
+rot_status rot_plan_info(rot_plan_t plan, int* K, int* chunk);
+
+/* y = T a (inverse = 0) or y = T^T a (inverse = 1) for every row: fp32 output.
+ * A: [M, lda] of a_dtype; Y: fp32 [M, ldy]. M may be 0. In-place (A == Y, fp32, lda == ldy)
+ * is allowed. */
+rot_status rot_apply(const void* A, int a_dtype, int64_t M, int64_t lda, rot_plan_t plan,
+                     int inverse, float* Y, int64_t ldy, void* stream);
+
+/* Fused rotate + quantise + pack, one HBM pass [HARP abstract; Hadamard-Int4-Accuracy
+ * wiki, Method]: codes [M, K*bits/8], scales [M, K/G] (binary16 bits).
+ * bits in {2, 4}; G must divide K and be a multiple of 8 (int4) or 16 (int2).
+ * Errors: ROT_EINVAL for a bad G / bits / pointer / leading dimension. */
+rot_status rot_quant(const void* A, int a_dtype, int64_t M, int64_t lda, rot_plan_t plan,
+                     int bits, int G, uint8_t* codes, uint16_t* scales, void* stream);
+
+/* Dequantise: x_hat = q * s (inverse = 0: in the rotated basis) or T^T (q * s)
+ * (inverse = 1: back in the original basis). out: fp32 [M, K] dense. */
+rot_status rot_dequant(const uint8_t* codes, const uint16_t* scales, int64_t M, rot_plan_t plan,
+                       int bits, int G, int inverse, float* out, void* stream);
+
+/* W4A4 linear [Hadamard-Int4-Accuracy wiki, Hypothesis: same-precision int4 MAC]:
+ *   C[m, n] = sum_g float(As[m, g]) * float(Ws[n, g]) * P[m, n, g],
+ *   P[m, n, g] = sum_{k in group g} qA[m, k] * qW[n, k]   (exact int32)
+ * Aq: uint8 [M, K/2], As: binary16 [M, K/G] (rot_quant output, int4);
+ * Wq: uint8 [N, K/2], Ws: binary16 [N, K/G] (rows of W^T through the same plan, int4);
+ * C:  [M, N] fp32 (c_dtype = ROT_F32) or bf16 (ROT_BF16), row-major, ldc = N.
+ * Requires K % G == 0, G % 32 == 0, K % 64 == 0, N % 16 == 0; M >= 0 arbitrary. */
+rot_status w4a4_linear(const uint8_t* Aq, const uint16_t* As, const uint8_t* Wq,
+                       const uint16_t* Ws, int64_t M, int64_t N, int64_t K, int G, void* C,
+                       int c_dtype, void* stream);
+
+/* The exact int32 group partial sums P[m, n, g] of the same contraction, written to
+ * P: int32 [M, N, K/G]. Same constraints as w4a4_linear. For checking only. */
+rot_status w4a4_group_partials(const uint8_t* Aq, const uint8_t* Wq, int64_t M, int64_t N,
+                               int64_t K, int G, int32_t* P, void* stream);
+
+/* Host helpers building HARP stage blocks from their parameters
+ * [HARP gist.science summary, 2.2: B = Q(theta) G_b]:
+ *   rot_harp_givens_blocks: out[i] = R(theta_i) . H_2 / sqrt(2) (fp32 2x2 row-major),
+ *     R(t) = [[cos t, -sin t], [sin t, cos t]]; out holds n * 4 floats.
+ *   rot_harp_qr_block: the Q factor (diag(R) > 0) of the b x b row-major matrix g
+ *     (Householder QR in double), out holds b * b floats. */
+rot_status rot_harp_givens_blocks(const double* theta, int64_t n, float* out);
+rot_status rot_harp_qr_block(const double* g, int b, float* out);
+
+/* Synchronise the current device and report device-side errors recorded by bounded
+ * waits (ROT_ETIMEOUT) since the last call; clears the record. */
+rot_status rot_check_device(void);
+
+/* Last error message of the calling host thread ("" if none). */
+const char* rot_last_error(void);
+
+/* Library version string. */
+const char* rot_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ROT_B200_H */

@@ -1,0 +1,84 @@
+"""CPU checks of the C-ABI library: it loads, exports every declared entry point, its host
+helpers match the oracle, and argument errors are reported before any device work."""
+import os
+import re
+
+import numpy as np
+import pytest
+
+import workloads as W
+from oracle import harp as Hp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "rot_b200.h")
+
+
+def _declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:rot_status|const char\*)\s+(\w+)\s*\(", src, flags=re.M)))
+
+
+def test_header_declares_the_entry_points():
+    names = _declared_functions()
+    for n in ("rot_plan_create", "rot_plan_destroy", "rot_quant", "rot_dequant", "rot_apply", "w4a4_linear"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in _declared_functions():
+        assert hasattr(lib._lib, name), name
+    assert "sm_100a" in lib.version()
+
+
+def test_givens_blocks_match_oracle(lib):
+    th = W.rng(3).uniform(-np.pi, np.pi, 1000)
+    got = lib.harp_givens_blocks(th).astype(np.float64)
+    ref = Hp.givens_blocks(th)
+    assert np.max(np.abs(got - ref)) < 1e-6
+
+
+@pytest.mark.parametrize("b", [3, 5, 43])
+def test_qr_block_matches_oracle(lib, b):
+    g = W.rng(b).standard_normal((b, b))
+    got = lib.harp_qr_block(g).astype(np.float64)
+    ref = Hp.qr_block(g)
+    assert np.max(np.abs(got - ref)) < 1e-5
+    assert np.max(np.abs(got @ got.T - np.eye(b))) < 1e-5
+
+
+def test_null_plan_is_rejected_without_a_device(lib):
+    import ctypes as C
+    st = lib._lib.rot_quant(C.c_void_p(0), lib.ROT_BF16, 1, 16, C.c_void_p(0), 4, 16, C.c_void_p(0),
+                            C.c_void_p(0), C.c_void_p(0))
+    assert st == lib.ROT_EINVAL
+    assert "plan" in lib.last_error()
+    st = lib._lib.rot_apply(C.c_void_p(0), lib.ROT_BF16, 1, 16, C.c_void_p(0), 0, C.c_void_p(0), 16, C.c_void_p(0))
+    assert st == lib.ROT_EINVAL
+
+
+def test_bad_w4a4_shapes_rejected_without_a_device(lib):
+    import ctypes as C
+    buf = (C.c_uint8 * 64)()
+    p = C.cast(buf, C.c_void_p)
+    # G not a multiple of 32
+    st = lib._lib.w4a4_linear(p, p, p, p, 1, 16, 128, 48, p, lib.ROT_F32, C.c_void_p(0))
+    assert st == lib.ROT_EINVAL
+    # N not a multiple of 16
+    st = lib._lib.w4a4_linear(p, p, p, p, 1, 24, 128, 32, p, lib.ROT_F32, C.c_void_p(0))
+    assert st == lib.ROT_EINVAL
+
+
+def test_plan_create_rejects_bad_schedules(lib):
+    import ctypes as C
+    h = C.c_void_p()
+    rad = (C.c_int * 2)(2, 3)
+    st = lib._lib.rot_plan_create(C.byref(h), 8, 2, rad, None, None, None, None)
+    assert st == lib.ROT_EINVAL and "product" in lib.last_error()
+    rad1 = (C.c_int * 1)(1)
+    st = lib._lib.rot_plan_create(C.byref(h), 1, 1, rad1, None, None, None, None)
+    assert st == lib.ROT_EINVAL
+    s = (C.c_int8 * 2)(1, 0)
+    rad2 = (C.c_int * 1)(2)
+    st = lib._lib.rot_plan_create(C.byref(h), 2, 1, rad2, None, None, None, s)
+    assert st == lib.ROT_EINVAL and "signs" in lib.last_error()

@@ -1,0 +1,104 @@
+"""GPU parity of the tcgen05 W4A4 linear against the oracle (exact int32 group sums,
+fp32 output within 1e-4 relative), plus the end-to-end rotated pipeline."""
+import numpy as np
+import pytest
+
+import workloads as W
+from oracle import hadamard as Hd
+from oracle import linear as L
+from oracle import quant as Q
+from parity import assert_linear_close, sample_rows, to_device
+
+pytestmark = pytest.mark.gpu
+
+
+def _codes(seed, rows, K, G):
+    """Oracle-quantised rows of a heavy-tailed matrix: (codes int8, packed uint8, scales fp16)."""
+    g = W.rng(seed)
+    X = g.standard_normal((rows, K)) * np.exp(g.uniform(-2, 2, (rows, 1)))
+    X[:, g.choice(K, max(1, K // 64), replace=False)] *= 20.0
+    q, s = Q.quantize(X, 4, G)
+    return q, Q.pack(q, 4), s
+
+
+def _dev(a):
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+
+@pytest.mark.parametrize("M,N,K,G", [(1, 16, 128, 32), (3, 48, 256, 64), (128, 256, 512, 128),
+                                     (129, 272, 384, 128), (64, 512, 4096, 128), (200, 176, 192, 32),
+                                     (16, 256, 1024, 256), (300, 784, 640, 64)])
+def test_group_partials_exact(lib, M, N, K, G):
+    qa, pa, sa = _codes(M + K, M, K, G)
+    qw, pw, sw = _codes(N + K + 1, N, K, G)
+    P = lib.w4a4_group_partials(_dev(pa), _dev(pw), G).cpu().numpy()
+    assert np.array_equal(P, L.group_partials(qa, qw, G))
+
+
+@pytest.mark.parametrize("M,N,K,G", [(1, 16, 128, 32), (3, 48, 256, 64), (129, 272, 384, 128),
+                                     (64, 512, 4096, 128), (200, 176, 192, 32), (16, 256, 1024, 256),
+                                     (300, 784, 640, 64)])
+@pytest.mark.parametrize("out", ["f32", "bf16"])
+def test_w4a4_linear_small(lib, M, N, K, G, out):
+    import torch
+    qa, pa, sa = _codes(M + K + 7, M, K, G)
+    qw, pw, sw = _codes(N + K + 9, N, K, G)
+    C = lib.w4a4_linear(_dev(pa), _dev(sa), _dev(pw), _dev(sw), G,
+                        out_dtype=torch.float32 if out == "f32" else torch.bfloat16)
+    C_ref = L.w4a4_reference(qa, sa, qw, sw, G)
+    if out == "f32":
+        assert_linear_close(C.cpu().numpy(), C_ref)
+    else:
+        # bf16 output: the fp32 result rounded once (8-bit mantissa)
+        assert_linear_close(C.float().cpu().numpy(), C_ref, tol=2 ** -8)
+
+
+def test_w4a4_empty_M(lib):
+    import torch
+    _, pw, sw = _codes(1, 32, 256, 128)
+    Aq = torch.empty((0, 128), dtype=torch.uint8, device="cuda")
+    As = torch.empty((0, 2), dtype=torch.float16, device="cuda")
+    C = lib.w4a4_linear(Aq, As, _dev(pw), _dev(sw), 128)
+    assert C.shape == (0, 32)
+
+
+@pytest.mark.parametrize("name", ["q_proj_prefill", "q_proj_decode", "up_proj_decode"])
+def test_w4a4_workload_oracle_codes(lib, name):
+    """Full-size linear on the oracle's own codes (so parity isolates the GEMM)."""
+    wl = W.make_workload(name)
+    bits, G = wl.quant[0]
+    rows = sample_rows(wl.M, 32)
+    qa, sa = Q.quantize(Hd.rht_apply(wl.A, wl.signs), bits, G) if wl.M <= 16 else (None, None)
+    if qa is None:
+        # quantise all rows in chunks (the oracle is exact and row-independent)
+        qa = np.empty((wl.M, wl.K), dtype=np.int8)
+        sa = np.empty((wl.M, wl.K // G), dtype=np.float16)
+        for r0 in range(0, wl.M, 256):
+            qa[r0:r0 + 256], sa[r0:r0 + 256] = Q.quantize(Hd.rht_apply(wl.A[r0:r0 + 256], wl.signs), bits, G)
+    qw, sw = Q.quantize(Hd.rht_apply(wl.W.T, wl.signs), bits, G)
+    C = lib.w4a4_linear(_dev(Q.pack(qa, 4)), _dev(sa), _dev(Q.pack(qw, 4)), _dev(sw), G).cpu().numpy()
+    C_ref = L.w4a4_reference(qa[rows], sa[rows], qw, sw, G)
+    assert_linear_close(C[rows], C_ref)
+
+
+def test_w4a4_end_to_end_rotated_pipeline(lib):
+    """GPU rotate+quantise of A and W^T, then the GPU linear: close to the oracle pipeline
+    (codes may differ only at boundary elements) and the page-2 accuracy trend holds."""
+    import torch
+    wl = W.make_workload("q_proj_prefill", M=256)
+    bits, G = wl.quant[0]
+    plan = lib.Plan.rht(wl.K, wl.signs)
+    Aq, As = lib.rot_quant(to_device(wl.A, True), plan, bits, G)
+    Wq, Ws = lib.rot_quant(to_device(wl.W.T.copy(), False), plan, bits, G)
+    C = lib.w4a4_linear(Aq, As, Wq, Ws, G, out_dtype=torch.bfloat16).float().cpu().numpy()
+    qa, sa = Q.quantize(Hd.rht_apply(wl.A, wl.signs), bits, G)
+    qw, sw = Q.quantize(Hd.rht_apply(wl.W.T, wl.signs), bits, G)
+    C_ref = L.w4a4_reference(qa, sa, qw, sw, G)
+    assert np.linalg.norm(C - C_ref) / np.linalg.norm(C_ref) < 5e-3
+    exact = wl.A.astype(np.float64) @ wl.W.astype(np.float64)
+    err_rot = np.linalg.norm(C - exact) / np.linalg.norm(exact)
+    qa0, sa0 = Q.quantize(wl.A, bits, G)
+    qw0, sw0 = Q.quantize(wl.W.T, bits, G)
+    err_plain = np.linalg.norm(L.w4a4_reference(qa0, sa0, qw0, sw0, G) - exact) / np.linalg.norm(exact)
+    assert err_rot < 0.8 * err_plain
