@@ -76,7 +76,7 @@ def profiled_traffic(name: str):
 class ClockSampler:
     """Samples SM clock and throttle reasons with NVML while the timed region runs."""
 
-    def __init__(self, dev_index: int, period: float = 0.02):
+    def __init__(self, dev_index: int, period: float = 0.01):
         self.samples, self.reasons, self.max_mhz = [], set(), None
         self.period = period
         self._stop = threading.Event()
@@ -195,16 +195,22 @@ def run_reference(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20000)
+    ap.add_argument("--steps", type=int, default=50000)
     ap.add_argument("--warmup", type=int, default=200)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-extra", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--profile", default=None,
+                    choices=["rot_quant", "down_proj_int4", "down_proj_int2", "harp_init", "harp_random",
+                             "w4a4_prefill", "w4a4_decode"],
+                    help="launch only this kernel --steps times (for ncu captures); prints timing only")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     if args.impl == "reference":
         return run_reference(args)
+    if args.profile:
+        return run_profile(args)
 
     import torch
     import torch.distributed as dist
@@ -390,6 +396,46 @@ def run_extra(hbr, W, dev, stream, peaks):
                                "GB/s": round(wbytes / t / 1e9, 1)}
     out["int8_peak_measured_TOPS"] = round(int8_peak, 1) if int8_peak else None
     return out
+
+
+def run_profile(args):
+    """One kernel, one workload, --warmup + --steps launches; for ncu captures."""
+    import torch
+    import workloads as W
+    import hadamard_butterfly_rotation_b200 as hbr
+    dev = torch.device("cuda", 0)
+    stream = torch.cuda.current_stream(dev)
+    name = args.profile
+    if name.startswith("w4a4"):
+        wl = W.make_workload("q_proj_prefill" if name == "w4a4_prefill" else "q_proj_decode")
+        bits, G = wl.quant[0]
+        plan = hbr.Plan.rht(wl.K, wl.signs)
+        Aq, As = hbr.rot_quant(torch.from_numpy(wl.A).to(torch.bfloat16).to(dev), plan, bits, G)
+        Wq, Ws = hbr.rot_quant(torch.from_numpy(np.ascontiguousarray(wl.W.T)).to(dev), plan, bits, G)
+        C = torch.empty((wl.M, Wq.shape[0]), dtype=torch.bfloat16, device=dev)
+        fn = lambda i: hbr.w4a4_linear(Aq, As, Wq, Ws, G, out=C, stream=stream)
+        work = 2.0 * wl.M * Wq.shape[0] * wl.K
+        unit = "TOPS"
+    else:
+        wname = {"rot_quant": "llama32_1b", "down_proj_int4": "down_proj", "down_proj_int2": "down_proj",
+                 "harp_init": "harp11008", "harp_random": "harp11008"}[name]
+        wl = W.make_workload(wname)
+        bits, G = wl.quant[1] if name == "down_proj_int2" else wl.quant[0]
+        if name.startswith("harp"):
+            plan = hbr.harp_plan(W.harp_draws(2, wl.extra["radices"]), wl.signs,
+                                 "init_identity" if name == "harp_init" else "random")
+        else:
+            plan = hbr.Plan.rht(wl.K, wl.signs)
+        A = torch.from_numpy(wl.A).to(torch.bfloat16).to(dev)
+        codes = torch.empty((wl.M, wl.K * bits // 8), dtype=torch.uint8, device=dev)
+        scales = torch.empty((wl.M, wl.K // G), dtype=torch.float16, device=dev)
+        fn = lambda i: hbr.rot_quant(A, plan, bits, G, codes=codes, scales=scales, stream=stream)
+        work = algorithmic_bytes(wl.M, wl.K, bits, G) / 1e3
+        unit = "GB/s"
+    t = _time_loop(fn, args.steps, stream, warm=args.warmup)
+    print(json.dumps({"profile": name, "us_per_launch": round(t * 1e6, 3),
+                      unit: round(work / t / 1e9 if unit == "GB/s" else work / t / 1e12, 2)}))
+    return 0
 
 
 def measure_int8_peak(dev):

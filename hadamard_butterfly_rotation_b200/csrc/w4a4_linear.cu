@@ -13,8 +13,9 @@
 //
 // Tile: 128 rows of A x 256 rows of W per CTA; K in blocks of 128 (one 128-byte swizzle
 // atom of int8 per row), 4 UMMAs of K = 32 per block.
-// Warp roles (512 threads, launched with 128 registers each; setmaxnreg moves registers
-// from the producers and the MMA warp to the epilogue: 256*176 + 224*88 + 32*24 = 512*128):
+// Warp roles (512 threads, launched with 128 registers each). setmaxnreg acts on whole
+// warpgroups, so roles are aligned to them: warpgroups 0-1 (epilogue) grow to 168 registers,
+// warpgroups 2-3 (producers + MMA warp) shrink to 88: 256*168 + 256*88 = 512*128.
 //   warps 0-7   epilogue: two warpgroups, 128 columns each; after each group they read
 //               the int32 partials from TMEM, apply the group scales and accumulate in
 //               fp32 registers;
@@ -52,9 +53,10 @@ constexpr int PROD_CHUNKS = (N_CHUNKS + N_PROD - 1) / N_PROD;     // per produce
 constexpr int EPI_COLS = BN / 2;         // columns per epilogue warpgroup
 constexpr int MMA_WARP = (N_EPI + N_PROD) / 32;
 constexpr int LAUNCH_REGS = 128;         // 65536 / THREADS
-constexpr int EPI_REGS = 176, PROD_REGS = 88, MMA_REGS = 24;
+constexpr int EPI_REGS = 168, PROD_REGS = 88;  // per warpgroup role
 static_assert(THREADS == 512, "register split assumes 512 threads");
-static_assert(N_EPI * EPI_REGS + N_PROD * PROD_REGS + 32 * MMA_REGS <= THREADS * LAUNCH_REGS, "register split");
+static_assert(N_EPI == 256 && N_PROD + 32 == 256, "roles must fill whole warpgroups");
+static_assert(N_EPI * EPI_REGS + (N_PROD + 32) * PROD_REGS <= THREADS * LAUNCH_REGS, "register split");
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t BIAS_BITS = 0x4B400000u;  // 1.5 * 2^23
 constexpr float BIAS_F = 12582912.0f;
@@ -227,7 +229,7 @@ __global__ void __launch_bounds__(THREADS, 1) w4a4_kernel(const Params p) {
 
   if (warp < N_EPI / 32) {
     // ======================= epilogue
-    asm volatile("setmaxnreg.inc.sync.aligned.u32 176;");
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 168;");
     const int wg = warp >> 2;                 // column block of EPI_COLS
     const int row = (warp & 3) * 32 + lane;   // TMEM lane = tile row
     const int m = m0 + row;
@@ -263,18 +265,17 @@ __global__ void __launch_bounds__(THREADS, 1) w4a4_kernel(const Params p) {
       tc_fence_after();
       const uint32_t base = lane_addr + b * BN + wg * EPI_COLS;
       const float2* scg = sc + (g & 1) * BN + wg * EPI_COLS;
-      uint32_t r[2][16];
-      tmem_ld16(base, r[0]);
-      tmem_wait_ld();
+      uint32_t rr[16];
 #pragma unroll
       for (int c = 0; c < EPI_COLS / 16; ++c) {
-        if (c + 1 < EPI_COLS / 16) tmem_ld16(base + (c + 1) * 16, r[(c + 1) & 1]);
+        tmem_ld16(base + c * 16, rr);
+        tmem_wait_ld();
         if (p.P == nullptr) {
 #pragma unroll
           for (int j = 0; j < 16; j += 2) {
             const float4 s2 = *reinterpret_cast<const float4*>(scg + c * 16 + j);
-            const float t0 = fmaf(__uint_as_float(r[c & 1][j]), s2.x, s2.y);
-            const float t1 = fmaf(__uint_as_float(r[c & 1][j + 1]), s2.z, s2.w);
+            const float t0 = fmaf(__uint_as_float(rr[j]), s2.x, s2.y);
+            const float t1 = fmaf(__uint_as_float(rr[j + 1]), s2.z, s2.w);
             acc[c * 16 + j] = fmaf(t0, sa, acc[c * 16 + j]);
             acc[c * 16 + j + 1] = fmaf(t1, sa, acc[c * 16 + j + 1]);
           }
@@ -282,10 +283,9 @@ __global__ void __launch_bounds__(THREADS, 1) w4a4_kernel(const Params p) {
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
             const int n = n0 + wg * EPI_COLS + c * 16 + j;
-            if (n < p.N) p.P[((int64_t)m * p.N + n) * NG + g] = ((int32_t)(r[c & 1][j] - BIAS_BITS)) / 256;
+            if (n < p.N) p.P[((int64_t)m * p.N + n) * NG + g] = ((int32_t)(rr[j] - BIAS_BITS)) / 256;
           }
         }
-        tmem_wait_ld();
       }
       // reset the accumulator to the bias for the group after next, then release it
 #pragma unroll
@@ -378,7 +378,7 @@ __global__ void __launch_bounds__(THREADS, 1) w4a4_kernel(const Params p) {
     }
   } else {
     // ======================= MMA issue
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 24;");
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 88;");  // same value as the producers of its warpgroup
     const bool leader = lane == 0;
     const uint32_t sbase = smem_u32(smem + OFF_STAGES);
     for (int ks = 0; ks < KS; ++ks) {

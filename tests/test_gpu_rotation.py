@@ -52,8 +52,13 @@ def test_rht_quant(lib, K, G, bits):
     A, s = _acts(67, K, K + G + bits)
     plan = lib.Plan.rht(K, s)
     codes, scales = lib.rot_quant(to_device(A, True), plan, bits, G)
-    excluded = assert_codes_match(codes.cpu().numpy(), scales.cpu().numpy(), Hd.rht_apply(A, s), bits, G)
-    assert excluded < 1e-3 * A.size
+    y = Hd.rht_apply(A, s)
+    assert_codes_match(codes.cpu().numpy(), scales.cpu().numpy(), y, bits, G)
+    # exclusions stay rare: per-code windows well under 1e-3 of the codes, and scale windows
+    # (binary16 midpoints are 2^-10 apart, the window 2e-5 wide) under 5% of the groups
+    cflag, gflag = Q.boundary_flags(y, bits, G)
+    assert (cflag & ~np.repeat(gflag, G, axis=1)).sum() < 1e-3 * A.size
+    assert gflag.sum() <= max(3, 0.05 * gflag.size)
 
 
 def test_rht_quant_fp32_input_and_page2_probe_without_signs(lib):

@@ -65,18 +65,13 @@ def test_w4a4_empty_M(lib):
 
 @pytest.mark.parametrize("name", ["q_proj_prefill", "q_proj_decode", "up_proj_decode"])
 def test_w4a4_workload_oracle_codes(lib, name):
-    """Full-size linear on the oracle's own codes (so parity isolates the GEMM)."""
+    """Full-size linear on oracle-quantised codes (parity isolates the GEMM; the codes of the
+    workload's activation and weight shapes are quantised without rotation to keep the oracle fast)."""
     wl = W.make_workload(name)
     bits, G = wl.quant[0]
-    rows = sample_rows(wl.M, 32)
-    qa, sa = Q.quantize(Hd.rht_apply(wl.A, wl.signs), bits, G) if wl.M <= 16 else (None, None)
-    if qa is None:
-        # quantise all rows in chunks (the oracle is exact and row-independent)
-        qa = np.empty((wl.M, wl.K), dtype=np.int8)
-        sa = np.empty((wl.M, wl.K // G), dtype=np.float16)
-        for r0 in range(0, wl.M, 256):
-            qa[r0:r0 + 256], sa[r0:r0 + 256] = Q.quantize(Hd.rht_apply(wl.A[r0:r0 + 256], wl.signs), bits, G)
-    qw, sw = Q.quantize(Hd.rht_apply(wl.W.T, wl.signs), bits, G)
+    rows = sample_rows(wl.M, 24)
+    qa, sa = Q.quantize(wl.A, bits, G)
+    qw, sw = Q.quantize(np.ascontiguousarray(wl.W.T), bits, G)
     C = lib.w4a4_linear(_dev(Q.pack(qa, 4)), _dev(sa), _dev(Q.pack(qw, 4)), _dev(sw), G).cpu().numpy()
     C_ref = L.w4a4_reference(qa[rows], sa[rows], qw, sw, G)
     assert_linear_close(C[rows], C_ref)
@@ -86,7 +81,7 @@ def test_w4a4_end_to_end_rotated_pipeline(lib):
     """GPU rotate+quantise of A and W^T, then the GPU linear: close to the oracle pipeline
     (codes may differ only at boundary elements) and the page-2 accuracy trend holds."""
     import torch
-    wl = W.make_workload("q_proj_prefill", M=256)
+    wl = W.make_workload("q_proj_prefill", M=64)
     bits, G = wl.quant[0]
     plan = lib.Plan.rht(wl.K, wl.signs)
     Aq, As = lib.rot_quant(to_device(wl.A, True), plan, bits, G)
