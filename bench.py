@@ -430,7 +430,7 @@ def run_profile(args):
         codes = torch.empty((wl.M, wl.K * bits // 8), dtype=torch.uint8, device=dev)
         scales = torch.empty((wl.M, wl.K // G), dtype=torch.float16, device=dev)
         fn = lambda i: hbr.rot_quant(A, plan, bits, G, codes=codes, scales=scales, stream=stream)
-        work = algorithmic_bytes(wl.M, wl.K, bits, G) / 1e3
+        work = algorithmic_bytes(wl.M, wl.K, bits, G)
         unit = "GB/s"
     t = _time_loop(fn, args.steps, stream, warm=args.warmup)
     print(json.dumps({"profile": name, "us_per_launch": round(t * 1e6, 3),

@@ -28,6 +28,10 @@
 namespace rotb {
 namespace {
 
+#ifndef ROT_FWHT_THREADS_E128
+#define ROT_FWHT_THREADS_E128 256   // threads per CTA for the 128-register-value layouts
+#endif
+
 template <int LOGN>
 struct Cfg {
   static constexpr int N = 1 << LOGN;
@@ -38,7 +42,7 @@ struct Cfg {
   static constexpr int TPC = 1 << HB;      // threads per chunk
   static constexpr int NV = 1 << VA;       // run length
   static constexpr int NH = 1 << HB;       // runs per thread
-  static constexpr int THREADS = LOGN <= 7 ? 256 : (LOGN == 8 ? 768 : (LOGN == 9 ? 512 : 384));
+  static constexpr int THREADS = LOGN <= 7 ? 256 : (LOGN == 8 ? 768 : (LOGN == 9 ? 512 : ROT_FWHT_THREADS_E128));
   static constexpr int SLOTS = THREADS / TPC;
   static constexpr int SSTRIDE = N + 4;    // floats per slot buffer (16-byte pad)
   static_assert(VA >= 1, "phase A needs element pairs");
@@ -66,6 +70,8 @@ struct Args {
   uint8_t* codes;
   uint16_t* scales;
   int G;
+  int log2G;
+  int64_t ngroups;   // K / G
   float norm;
 };
 
@@ -132,173 +138,249 @@ __device__ __forceinline__ uint32_t pack16_int2(const uint32_t (&t)[16]) {
   return (b[0] + (b[1] << 2) + (b[2] << 4) + (b[3] << 6)) ^ 0xAAAAAAAAu;
 }
 
+__device__ int g_fwht_error = 0;
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// Bounded wait on a slot's staging barrier (the bulk copy always completes; the bound only
+// protects against a programming error). Returns false after about 1 s.
+__device__ __forceinline__ bool stage_wait(uint64_t* bar, uint32_t parity) {
+  const uint32_t addr = smem_addr(bar);
+  unsigned long long t0 = 0;
+  for (uint32_t it = 0;; ++it) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(addr), "r"(parity)
+        : "memory");
+    if (done) return true;
+    if ((it & 255) == 255) {
+      unsigned long long now;
+      asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(now));
+      if (t0 == 0) t0 = now;
+      else if (now - t0 > 1000000000ull) {
+        atomicExch(&g_fwht_error, (int)ROT_ETIMEOUT);
+        return false;
+      }
+    }
+  }
+}
+
+// One elected thread: announce the bytes and start the bulk copy global -> slot buffer.
+__device__ __forceinline__ void stage_issue(uint64_t* bar, void* dst, const void* src, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)), "r"(bytes) : "memory");
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   smem_addr(dst)),
+               "l"(src), "r"(bytes), "r"(smem_addr(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ float min3(float a, float b, float c) {
+  float d;
+  asm("min.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// Radix-2 butterflies along pair-index bit b: (P, Q) <- (P + Q, P - Q) on fp32 pairs.
+template <int NP>
+__device__ __forceinline__ void stage_pairs(float2 (&xp)[NP], int b) {
+  const float2 m1 = make_float2(-1.0f, -1.0f);
+#pragma unroll
+  for (int i = 0; i < NP; ++i)
+    if (!(i & (1 << b))) {
+      const float2 P = xp[i], Q = xp[i + (1 << b)];
+      xp[i] = __fadd2_rn(P, Q);
+      xp[i + (1 << b)] = __ffma2_rn(Q, m1, P);
+    }
+}
+
 template <int LOGN, bool BF16, int MODE, int BITS>
 __global__ void __launch_bounds__(Cfg<LOGN>::THREADS, 1) fwht_kernel(const Args a) {
   using C = Cfg<LOGN>;
   constexpr int N = C::N, ELOG = C::ELOG, E = C::E, HB = C::HB, VA = C::VA, TPC = C::TPC;
   constexpr int NV = C::NV, NH = C::NH, SLOTS = C::SLOTS, SSTRIDE = C::SSTRIDE;
-  extern __shared__ __align__(16) float smem[];
+  constexpr int NP = E / 2;  // fp32 pairs per thread: xp[i] = coordinates (2i, 2i+1) of the layout
+  extern __shared__ __align__(128) float smem[];
   float* sbuf = smem;
-  uint32_t* smask = reinterpret_cast<uint32_t*>(smem + (HB > 0 ? SLOTS * SSTRIDE : 0));
-
-  const bool has_signs = a.signmask != nullptr;
-  if (has_signs) {
-    for (int i = threadIdx.x; i < a.K / 2; i += C::THREADS) smask[i] = a.signmask[i];
-  }
-  __syncthreads();
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SLOTS * SSTRIDE);
+  uint32_t* smask = reinterpret_cast<uint32_t*>(bars + ((SLOTS + 1) & ~1));  // 16-byte aligned
 
   const int slot = threadIdx.x / TPC;
   const int t = threadIdx.x % TPC;
   float* buf = sbuf + slot * SSTRIDE;
+  uint64_t* bar = bars + slot;
+  const bool has_signs = a.signmask != nullptr;
+  if (threadIdx.x < SLOTS) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_addr(bars + threadIdx.x)) : "memory");
+  }
+  if (has_signs) {
+    for (int i = threadIdx.x; i < a.K / 2; i += C::THREADS) smask[i] = a.signmask[i];
+  }
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  __syncthreads();
+
   const int64_t units = a.M * a.chunks;
+  const int64_t stride = (int64_t)gridDim.x * SLOTS;
+  int64_t u = (int64_t)blockIdx.x * SLOTS + slot;
+  const int64_t drow = stride / a.chunks;
+  const int dchunk = (int)(stride - drow * a.chunks);
+  int64_t row = u / a.chunks;
+  int chunk = (int)(u - row * a.chunks);
+  constexpr uint32_t ELEM = BF16 ? 2 : 4;
+  const uint32_t chunk_bytes = (uint32_t)N * ELEM;
+  auto src_of = [&](int64_t r, int c) -> const void* {
+    return static_cast<const uint8_t*>(a.A) + ((int64_t)r * a.lda + (int64_t)c * N) * ELEM;
+  };
+  if (t == 0 && u < units) stage_issue(bar, buf, src_of(row, chunk), chunk_bytes);
+  uint32_t parity = 0;
+  const int log2G = a.log2G;
 
-  for (int64_t u = (int64_t)blockIdx.x * SLOTS + slot; u < units; u += (int64_t)gridDim.x * SLOTS) {
-    const int64_t row = u / a.chunks;
-    const int cbase = (int)(u - row * a.chunks) * N;
-    float x[E];
+  for (; u < units; u += stride) {
+    const int cbase = chunk * N;
+    float2 xp[NP];
+    if (!stage_wait(bar, parity)) break;
+    parity ^= 1u;
 
-    // ---------------- phase A: load runs, apply signs, convert to fp32
+    // ---------------- phase A: runs of NV elements from the staged chunk, signs, fp32 pairs
     {
-      const int run0 = cbase + (t << VA);
+      const int run0 = t << VA;
       if constexpr (BF16) {
-        const __nv_bfloat16* src = static_cast<const __nv_bfloat16*>(a.A) + row * a.lda + run0;
-        constexpr int NW = NV / 2;  // 32-bit words per run
-        uint32_t raw[NH][NW];
+        constexpr int NW = NV / 2;
+        const uint32_t* sraw = reinterpret_cast<const uint32_t*>(buf);
 #pragma unroll
         for (int h = 0; h < NH; ++h) {
-          const uint32_t* p = reinterpret_cast<const uint32_t*>(src + (h << ELOG));
-          if constexpr (NW >= 4) {
-#pragma unroll
-            for (int v = 0; v < NW / 4; ++v) {
-              uint4 q = __ldcs(reinterpret_cast<const uint4*>(p) + v);
-              raw[h][4 * v] = q.x; raw[h][4 * v + 1] = q.y; raw[h][4 * v + 2] = q.z; raw[h][4 * v + 3] = q.w;
-            }
-          } else if constexpr (NW == 2) {
-            uint2 q = __ldcs(reinterpret_cast<const uint2*>(p));
-            raw[h][0] = q.x; raw[h][1] = q.y;
-          } else {
-            raw[h][0] = __ldcs(p);
-          }
-        }
-#pragma unroll
-        for (int h = 0; h < NH; ++h) {
-          uint32_t m[NW];
-          load_masks<NW>(m, smask, (run0 + (h << ELOG)) >> 1, MODE != MODE_APPLY_INV && has_signs);
+          const int w0 = (run0 + (h << ELOG)) >> 1;   // word index within the chunk
+          uint32_t raw[NW], m[NW];
+          load_masks<NW>(raw, sraw, w0, true);
+          load_masks<NW>(m, smask, (cbase >> 1) + w0, MODE != MODE_APPLY_INV && has_signs);
 #pragma unroll
           for (int w = 0; w < NW; ++w) {
-            const uint32_t v = raw[h][w] ^ m[w];
-            x[h * NV + 2 * w] = bf16lo(v);
-            x[h * NV + 2 * w + 1] = bf16hi(v);
+            const uint32_t v = raw[w] ^ m[w];
+            xp[h * NW + w] = make_float2(bf16lo(v), bf16hi(v));
           }
         }
       } else {
-        const float* src = static_cast<const float*>(a.A) + row * a.lda + run0;
 #pragma unroll
         for (int h = 0; h < NH; ++h) {
-          const float* p = src + (h << ELOG);
+          const int i0 = run0 + (h << ELOG);
+          constexpr int NW = NV / 2;
           if constexpr (NV >= 4) {
 #pragma unroll
             for (int v = 0; v < NV / 4; ++v) {
-              float4 q = __ldcs(reinterpret_cast<const float4*>(p) + v);
-              x[h * NV + 4 * v] = q.x; x[h * NV + 4 * v + 1] = q.y;
-              x[h * NV + 4 * v + 2] = q.z; x[h * NV + 4 * v + 3] = q.w;
+              const float4 q = *reinterpret_cast<const float4*>(buf + i0 + 4 * v);
+              xp[h * NW + 2 * v] = make_float2(q.x, q.y);
+              xp[h * NW + 2 * v + 1] = make_float2(q.z, q.w);
             }
           } else {
-            float2 q = __ldcs(reinterpret_cast<const float2*>(p));
-            x[h * NV] = q.x; x[h * NV + 1] = q.y;
+            xp[h * NW] = *reinterpret_cast<const float2*>(buf + i0);
           }
-        }
-        if (MODE != MODE_APPLY_INV && has_signs) {
+          if (MODE != MODE_APPLY_INV && has_signs) {
+            uint32_t m[NW];
+            load_masks<NW>(m, smask, (cbase + i0) >> 1, true);
 #pragma unroll
-          for (int h = 0; h < NH; ++h) {
-            uint32_t m[NV / 2];
-            load_masks<NV / 2>(m, smask, (run0 + (h << ELOG)) >> 1, true);
-#pragma unroll
-            for (int w = 0; w < NV / 2; ++w) {
-              x[h * NV + 2 * w] = __uint_as_float(__float_as_uint(x[h * NV + 2 * w]) ^ (m[w] << 16));
-              x[h * NV + 2 * w + 1] = __uint_as_float(__float_as_uint(x[h * NV + 2 * w + 1]) ^ (m[w] & 0x80000000u));
+            for (int w = 0; w < NW; ++w) {
+              xp[h * NW + w].x = __uint_as_float(__float_as_uint(xp[h * NW + w].x) ^ (m[w] << 16));
+              xp[h * NW + w].y = __uint_as_float(__float_as_uint(xp[h * NW + w].y) ^ (m[w] & 0x80000000u));
             }
           }
         }
       }
     }
 
-    // ---------------- phase A butterflies over all E register bits
+    // ---------------- phase A butterflies: register bit 0 (inside the pairs), then bits 1..e-1
 #pragma unroll
-    for (int r = 0; r < E; r += 2) {
-      const float p = x[r], q = x[r + 1];
-      x[r] = p + q;
-      x[r + 1] = p - q;
+    for (int i = 0; i < NP; ++i) {
+      const float p = xp[i].x, q = xp[i].y;
+      xp[i] = make_float2(p + q, p - q);
     }
 #pragma unroll
-    for (int h = 2; h < E; h <<= 1) {
-#pragma unroll
-      for (int r = 0; r < E; r += 2)
-        if (!(r & h)) bfly_x2(x[r], x[r + 1], x[r + h], x[r + h + 1]);
-    }
+    for (int b = 0; b < ELOG - 1; ++b) stage_pairs<NP>(xp, b);
 
-    // ---------------- transpose to phase B and remaining stages
+    // ---------------- transpose through the slot buffer
     if constexpr (HB > 0) {
-      slot_sync<TPC>(slot);  // previous unit's phase-B reads are done
+      slot_sync<TPC>(slot);  // every thread has read its staged runs
 #pragma unroll
       for (int h = 0; h < NH; ++h) {
         const int i0 = (t << VA) + (h << ELOG);
+        constexpr int NW = NV / 2;
         if constexpr (NV >= 4) {
 #pragma unroll
-          for (int v = 0; v < NV / 4; ++v)
-            *reinterpret_cast<float4*>(buf + swz<LOGN>(i0 + 4 * v)) =
-                make_float4(x[h * NV + 4 * v], x[h * NV + 4 * v + 1], x[h * NV + 4 * v + 2], x[h * NV + 4 * v + 3]);
+          for (int v = 0; v < NV / 4; ++v) {
+            const float2 p0 = xp[h * NW + 2 * v], p1 = xp[h * NW + 2 * v + 1];
+            *reinterpret_cast<float4*>(buf + swz<LOGN>(i0 + 4 * v)) = make_float4(p0.x, p0.y, p1.x, p1.y);
+          }
         } else {
-          *reinterpret_cast<float2*>(buf + swz<LOGN>(i0)) = make_float2(x[h * NV], x[h * NV + 1]);
+          *reinterpret_cast<float2*>(buf + swz<LOGN>(i0)) = xp[h * NW];
         }
       }
       slot_sync<TPC>(slot);
 #pragma unroll
       for (int jc = 0; jc < E / 4; ++jc) {
         const float4 q = *reinterpret_cast<const float4*>(buf + swz<LOGN>((t << ELOG) + 4 * jc));
-        x[4 * jc] = q.x; x[4 * jc + 1] = q.y; x[4 * jc + 2] = q.z; x[4 * jc + 3] = q.w;
-      }
-#pragma unroll
-      for (int h = NV; h < E; h <<= 1) {
-#pragma unroll
-        for (int r = 0; r < E; r += 2)
-          if (!(r & h)) bfly_x2(x[r], x[r + 1], x[r + h], x[r + h + 1]);
+        xp[2 * jc] = make_float2(q.x, q.y);
+        xp[2 * jc + 1] = make_float2(q.z, q.w);
       }
     }
+    // the slot buffer is free: stage the next unit while this one finishes
+    int64_t nrow = row + drow;
+    int nchunk = chunk + dchunk;
+    if (nchunk >= a.chunks) { nchunk -= a.chunks; ++nrow; }
+    if (u + stride < units) {
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      slot_sync<TPC>(slot);
+      if (t == 0) stage_issue(bar, buf, src_of(nrow, nchunk), chunk_bytes);
+    }
+    // ---------------- phase B butterflies: register bits VA..e-1 (pair-index bits VA-1..e-2)
+    if constexpr (HB > 0) {
+#pragma unroll
+      for (int b = VA - 1; b < ELOG - 1; ++b) stage_pairs<NP>(xp, b);
+    }
+    const int64_t cur_row = row;
+    row = nrow;
+    chunk = nchunk;
 
-    // x[j] = z for chunk coordinate (t << ELOG) + j; y = z * norm
-    const int c0 = cbase + (t << ELOG);  // row coordinate of x[0]
+    // xp[j/2] holds z for chunk coordinates (t << ELOG) + j; y = z * norm
+    const int c0 = cbase + (t << ELOG);  // row coordinate of the first element
     if constexpr (MODE == MODE_APPLY || MODE == MODE_APPLY_INV) {
-      float* dst = a.Y + row * a.ldy + c0;
+      float* dst = a.Y + cur_row * a.ldy + c0;
+      const float2 nn = make_float2(a.norm, a.norm);
 #pragma unroll
       for (int jc = 0; jc < E / 4; ++jc) {
-        float4 q = make_float4(x[4 * jc] * a.norm, x[4 * jc + 1] * a.norm, x[4 * jc + 2] * a.norm,
-                               x[4 * jc + 3] * a.norm);
+        const float2 p0 = __fmul2_rn(xp[2 * jc], nn), p1 = __fmul2_rn(xp[2 * jc + 1], nn);
+        float4 q = make_float4(p0.x, p0.y, p1.x, p1.y);
         if (MODE == MODE_APPLY_INV && has_signs) {
           const uint32_t m0 = smask[(c0 >> 1) + 2 * jc], m1 = smask[(c0 >> 1) + 2 * jc + 1];
-          q.x = __uint_as_float(__float_as_uint(q.x) ^ ((m0 << 16) & 0x80000000u));
+          q.x = __uint_as_float(__float_as_uint(q.x) ^ (m0 << 16));
           q.y = __uint_as_float(__float_as_uint(q.y) ^ (m0 & 0x80000000u));
-          q.z = __uint_as_float(__float_as_uint(q.z) ^ ((m1 << 16) & 0x80000000u));
+          q.z = __uint_as_float(__float_as_uint(q.z) ^ (m1 << 16));
           q.w = __uint_as_float(__float_as_uint(q.w) ^ (m1 & 0x80000000u));
         }
         *reinterpret_cast<float4*>(dst + 4 * jc) = q;
       }
     } else {
       // ---------------- quantisation: groups of G contiguous coordinates.
-      // Absmax per granule of 8 registers, then a predicated tree over granules for the
-      // runtime group size (G/8 granules), then warp shuffles when a group spans threads.
       constexpr float QMAX = BITS == 4 ? 7.0f : 1.0f;
       constexpr float MAGIC = BITS == 4 ? 8388616.0f : 8388610.0f;  // 2^23 + qmax + 1
       constexpr int NG = E / 8;
-      const int G = a.G;
-      const int gg = G >> 3;  // granules per group (power of two)
+      const int gg = a.G >> 3;  // granules per group (power of two)
       float gm[NG];
 #pragma unroll
       for (int i = 0; i < NG; ++i) {
-        float m = fmaxf(fabsf(x[8 * i]), fabsf(x[8 * i + 1]));
-        m = max3(m, fabsf(x[8 * i + 2]), fabsf(x[8 * i + 3]));
-        m = max3(m, fabsf(x[8 * i + 4]), fabsf(x[8 * i + 5]));
-        gm[i] = max3(m, fabsf(x[8 * i + 6]), fabsf(x[8 * i + 7]));
+        const float2 p0 = xp[4 * i], p1 = xp[4 * i + 1], p2 = xp[4 * i + 2], p3 = xp[4 * i + 3];
+        float mx = max3(p0.x, p0.y, p1.x);
+        float mn = min3(p0.x, p0.y, p1.x);
+        mx = max3(mx, p1.y, p2.x);
+        mn = min3(mn, p1.y, p2.x);
+        mx = max3(mx, p2.y, p3.x);
+        mn = min3(mn, p2.y, p3.x);
+        mx = fmaxf(mx, p3.y);
+        mn = fminf(mn, p3.y);
+        gm[i] = fmaxf(mx, -mn);
       }
 #pragma unroll
       for (int st = 1; st < NG; st <<= 1) {
@@ -307,9 +389,9 @@ __global__ void __launch_bounds__(Cfg<LOGN>::THREADS, 1) fwht_kernel(const Args 
           for (int i = 0; i + st < NG; i += 2 * st) gm[i] = fmaxf(gm[i], gm[i + st]);
         }
       }
-      if (G > E) {
+      if (a.G > E) {
         const unsigned lanes = slot_lanes<TPC>();
-        for (int o = 1; o < G / E; o <<= 1) gm[0] = fmaxf(gm[0], __shfl_xor_sync(lanes, gm[0], o));
+        for (int o = 1; o < a.G / E; o <<= 1) gm[0] = fmaxf(gm[0], __shfl_xor_sync(lanes, gm[0], o));
       }
       float fw[NG];
       bool slow[NG];
@@ -324,32 +406,38 @@ __global__ void __launch_bounds__(Cfg<LOGN>::THREADS, 1) fwht_kernel(const Args 
           sc[i] = sc[i - 1];
         }
       }
-      // scales: one binary16 per group
       {
-        const int64_t ngr = a.K / G;
-        uint16_t* srow = a.scales + row * ngr;
-        if (G > E) {
-          if ((t & (G / E - 1)) == 0) srow[c0 / G] = sc[0];
+        uint16_t* srow = a.scales + cur_row * a.ngroups;
+        if (a.G > E) {
+          if ((t & (a.G / E - 1)) == 0) srow[c0 >> log2G] = sc[0];
         } else {
 #pragma unroll
           for (int i = 0; i < NG; ++i)
-            if ((i & (gg - 1)) == 0) srow[(c0 + 8 * i) / G] = sc[i];
+            if ((i & (gg - 1)) == 0) srow[(c0 + 8 * i) >> log2G] = sc[i];
         }
       }
-      // codes
       constexpr int CPW = 32 / BITS;   // codes per 32-bit word
       constexpr int NWD = E / CPW;     // words per thread
+      const float2 mg = make_float2(MAGIC, MAGIC);
       uint32_t words[NWD];
 #pragma unroll
       for (int w = 0; w < NWD; ++w) {
         const int gi = w * (CPW / 8);    // granule of the word's first code
         uint32_t tt[CPW];
         if (!slow[gi]) {
+          const float2 ff = make_float2(fw[gi], fw[gi]);
 #pragma unroll
-          for (int j = 0; j < CPW; ++j) tt[j] = code_magic(x[CPW * w + j], fw[gi], MAGIC);
+          for (int j = 0; j < CPW; j += 2) {
+            const float2 r = __ffma2_rn(xp[(CPW * w + j) / 2], ff, mg);
+            tt[j] = __float_as_uint(r.x);
+            tt[j + 1] = __float_as_uint(r.y);
+          }
         } else {
 #pragma unroll
-          for (int j = 0; j < CPW; ++j) tt[j] = code_magic_clamped(x[CPW * w + j], fw[gi], QMAX, MAGIC);
+          for (int j = 0; j < CPW; j += 2) {
+            tt[j] = code_magic_clamped(xp[(CPW * w + j) / 2].x, fw[gi], QMAX, MAGIC);
+            tt[j + 1] = code_magic_clamped(xp[(CPW * w + j) / 2].y, fw[gi], QMAX, MAGIC);
+          }
         }
         if constexpr (BITS == 4) {
           words[w] = pack8_int4(*reinterpret_cast<const uint32_t(*)[8]>(tt));
@@ -357,7 +445,7 @@ __global__ void __launch_bounds__(Cfg<LOGN>::THREADS, 1) fwht_kernel(const Args 
           words[w] = pack16_int2(*reinterpret_cast<const uint32_t(*)[16]>(tt));
         }
       }
-      uint32_t* dst = reinterpret_cast<uint32_t*>(a.codes + row * (int64_t)(a.K / CPW) * 4) + c0 / CPW;
+      uint32_t* dst = reinterpret_cast<uint32_t*>(a.codes + cur_row * (int64_t)(a.K / CPW) * 4) + c0 / CPW;
       if constexpr (NWD >= 4) {
 #pragma unroll
         for (int v = 0; v < NWD / 4; ++v)
@@ -374,7 +462,7 @@ __global__ void __launch_bounds__(Cfg<LOGN>::THREADS, 1) fwht_kernel(const Args 
 template <int LOGN, bool BF16, int MODE, int BITS>
 rot_status launch_one(const Args& a, cudaStream_t s) {
   using C = Cfg<LOGN>;
-  const size_t smem = (C::HB > 0 ? (size_t)C::SLOTS * C::SSTRIDE * 4 : 0) + (size_t)(a.K / 2) * 4;
+  const size_t smem = (size_t)C::SLOTS * C::SSTRIDE * 4 + (size_t)((C::SLOTS + 1) & ~1) * 8 + (size_t)(a.K / 2) * 4;
   if (smem > 227 * 1024) return set_error(ROT_EUNSUPPORTED, "fused rotation: sign table too large for shared memory");
   auto kern = fwht_kernel<LOGN, BF16, MODE, BITS>;
   static int configured[64] = {0};  // per device: the opt-in limit is set once
@@ -424,6 +512,17 @@ Args make_args(const rot_plan_s* p, const void* A, int64_t M, int64_t lda) {
 
 }  // namespace
 
+rot_status fwht_fetch_device_error() {
+  int v = 0;
+  ROT_CUDA_TRY(cudaMemcpyFromSymbol(&v, g_fwht_error, sizeof(int)));
+  if (v) {
+    int z = 0;
+    ROT_CUDA_TRY(cudaMemcpyToSymbol(g_fwht_error, &z, sizeof(int)));
+    return set_error((rot_status)v, "a bounded wait in the fused rotation kernel gave up");
+  }
+  return ROT_OK;
+}
+
 bool fwht_quant_supported(const rot_plan_s* p, int bits, int G) {
   if (p->chunk_log2 < 5) return false;
   const int N = 1 << p->chunk_log2;
@@ -451,6 +550,9 @@ rot_status fwht_quant(const rot_plan_s* p, const void* A, int a_dtype, int64_t M
   a.codes = codes;
   a.scales = scales;
   a.G = G;
+  a.log2G = 0;
+  while ((1 << a.log2G) < G) ++a.log2G;
+  a.ngroups = p->K / G;
   const int n = p->chunk_log2;
   if (a_dtype == ROT_BF16)
     return bits == 4 ? dispatch_logn<true, MODE_QUANT, 4>(n, a, s) : dispatch_logn<true, MODE_QUANT, 2>(n, a, s);

@@ -59,6 +59,7 @@ rot_status fwht_apply(const rot_plan_s* p, const void* A, int a_dtype, int64_t M
 rot_status fwht_quant(const rot_plan_s* p, const void* A, int a_dtype, int64_t M, int64_t lda,
                       int bits, int G, uint8_t* codes, uint16_t* scales, cudaStream_t s);
 bool fwht_quant_supported(const rot_plan_s* p, int bits, int G);
+rot_status fwht_fetch_device_error();
 // generic stage path (rot_stages.cu)
 rot_status stages_apply(const rot_plan_s* p, const void* A, int a_dtype, int64_t M, int64_t lda,
                         int inverse, float* Y, int64_t ldy, cudaStream_t s);

@@ -477,5 +477,7 @@ rot_status w4a4_fetch_device_error() {
 extern "C" rot_status rot_check_device(void) {
   cudaError_t e = cudaDeviceSynchronize();
   if (e != cudaSuccess) return rotb::cuda_error(e, "rot_check_device");
-  return rotb::w4a4_fetch_device_error();
+  rot_status st = rotb::fwht_fetch_device_error();
+  rot_status st2 = rotb::w4a4_fetch_device_error();
+  return st != ROT_OK ? st : st2;
 }
