@@ -29,7 +29,7 @@ namespace rotb {
 namespace {
 
 #ifndef ROT_FWHT_THREADS_E128
-#define ROT_FWHT_THREADS_E128 256   // threads per CTA for the 128-register-value layouts
+#define ROT_FWHT_THREADS_E128 384   // threads per CTA for the 128-register-value layouts
 #endif
 
 template <int LOGN>
@@ -48,13 +48,15 @@ struct Cfg {
   static_assert(VA >= 1, "phase A needs element pairs");
 };
 
-// Physical float index of chunk-local coordinate i in a slot buffer.
+// Physical float index of chunk-local coordinate i in a slot buffer: 16-byte chunks are
+// XOR-swizzled by the three coordinate bits above the phase-B thread's run (and, for
+// n = 9 and 11, also by coordinate bit 5), which makes phase-A stores and phase-B loads
+// conflict-free (n = 10 keeps 4-way conflicts on the stores).
 template <int LOGN>
 __device__ __forceinline__ int swz(int i) {
   constexpr int ELOG = Cfg<LOGN>::ELOG;
   int x = ((i >> ELOG) & 7) << 2;
-  if (LOGN == 9 || LOGN == 10 || LOGN == 11) x ^= ((i >> 5) & 1) << 2;
-  if (LOGN == 10) x ^= ((i >> 6) & 1) << 3;
+  if constexpr (LOGN == 9 || LOGN == 11) x ^= ((i >> 5) & 1) << 2;
   return i ^ x;
 }
 
@@ -199,12 +201,160 @@ __device__ __forceinline__ void stage_pairs(float2 (&xp)[NP], int b) {
     }
 }
 
-template <int LOGN, bool BF16, int MODE, int BITS>
+// Quantise the E values a thread holds (coordinates c0 .. c0+E-1 of one row) and store
+// packed codes and scales. GT > 0: compile-time group size; GT == 0: runtime a.G.
+template <int LOGN, int BITS, int GT, int E, int TPC>
+__device__ __forceinline__ void quantise_store(const Args& a, const float2 (&xp)[E / 2], int64_t row, int c0, int t) {
+  constexpr float QMAX = BITS == 4 ? 7.0f : 1.0f;
+  constexpr float MAGIC = BITS == 4 ? 8388616.0f : 8388610.0f;  // 2^23 + qmax + 1
+  constexpr int CPW = 32 / BITS;   // codes per 32-bit word
+  constexpr int NWD = E / CPW;     // words per thread
+  uint16_t* srow = a.scales + row * a.ngroups;
+  uint32_t words[NWD];
+  if constexpr (GT > 0) {
+    constexpr int GE = GT <= E ? GT : E;     // elements of one group held by this thread
+    constexpr int NGT = E / GE;              // groups (or group fragments) per thread
+    float f[NGT];
+    bool any_slow = false;
+#pragma unroll
+    for (int g = 0; g < NGT; ++g) {
+      float m = 0.0f;
+#pragma unroll
+      for (int j = 0; j < GE / 2; ++j) {
+        const float2 p = xp[g * (GE / 2) + j];
+        m = fmaxf(m, fmaxf(fabsf(p.x), fabsf(p.y)));
+      }
+      if constexpr (GT > E) {
+        const unsigned lanes = slot_lanes<TPC>();
+#pragma unroll
+        for (int o = 1; o < GT / E; o <<= 1) m = fmaxf(m, __shfl_xor_sync(lanes, m, o));
+      }
+      bool slow;
+      const uint16_t s16 = group_scale(m, a.norm, QMAX, &f[g], &slow);
+      any_slow |= slow;
+      if constexpr (GT > E) {
+        if ((t & (GT / E - 1)) == 0) srow[c0 / GT] = s16;
+      } else {
+        srow[c0 / GT + g] = s16;
+      }
+    }
+    const float2 mg = make_float2(MAGIC, MAGIC);
+    if (!any_slow) {
+#pragma unroll
+      for (int w = 0; w < NWD; ++w) {
+        const float fg = f[(w * CPW) / GE];
+        const float2 ff = make_float2(fg, fg);
+        uint32_t tt[CPW];
+#pragma unroll
+        for (int j = 0; j < CPW; j += 2) {
+          const float2 r = __ffma2_rn(xp[(CPW * w + j) / 2], ff, mg);
+          tt[j] = __float_as_uint(r.x);
+          tt[j + 1] = __float_as_uint(r.y);
+        }
+        if constexpr (BITS == 4) words[w] = pack8_int4(*reinterpret_cast<const uint32_t(*)[8]>(tt));
+        else words[w] = pack16_int2(*reinterpret_cast<const uint32_t(*)[16]>(tt));
+      }
+    } else {
+#pragma unroll
+      for (int w = 0; w < NWD; ++w) {
+        const float fg = f[(w * CPW) / GE];
+        uint32_t tt[CPW];
+#pragma unroll
+        for (int j = 0; j < CPW; j += 2) {
+          tt[j] = code_magic_clamped(xp[(CPW * w + j) / 2].x, fg, QMAX, MAGIC);
+          tt[j + 1] = code_magic_clamped(xp[(CPW * w + j) / 2].y, fg, QMAX, MAGIC);
+        }
+        if constexpr (BITS == 4) words[w] = pack8_int4(*reinterpret_cast<const uint32_t(*)[8]>(tt));
+        else words[w] = pack16_int2(*reinterpret_cast<const uint32_t(*)[16]>(tt));
+      }
+    }
+  } else {
+    // runtime group size: max per granule of 8, predicated tree, shuffles across threads
+    constexpr int NG = E / 8;
+    const int G = a.G;
+    const int gg = G >> 3;
+    float gm[NG];
+#pragma unroll
+    for (int i = 0; i < NG; ++i) {
+      float m = 0.0f;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) m = fmaxf(m, fmaxf(fabsf(xp[4 * i + j].x), fabsf(xp[4 * i + j].y)));
+      gm[i] = m;
+    }
+#pragma unroll
+    for (int st = 1; st < NG; st <<= 1) {
+      if (st < gg) {
+#pragma unroll
+        for (int i = 0; i + st < NG; i += 2 * st) gm[i] = fmaxf(gm[i], gm[i + st]);
+      }
+    }
+    if (G > E) {
+      const unsigned lanes = slot_lanes<TPC>();
+      for (int o = 1; o < G / E; o <<= 1) gm[0] = fmaxf(gm[0], __shfl_xor_sync(lanes, gm[0], o));
+    }
+    float fw[NG];
+    bool slow[NG];
+    uint16_t sc[NG];
+#pragma unroll
+    for (int i = 0; i < NG; ++i) {
+      if ((i & (gg - 1)) == 0) {
+        sc[i] = group_scale(gm[i], a.norm, QMAX, &fw[i], &slow[i]);
+      } else {
+        fw[i] = fw[i - 1];
+        slow[i] = slow[i - 1];
+        sc[i] = sc[i - 1];
+      }
+    }
+    if (G > E) {
+      if ((t & (G / E - 1)) == 0) srow[c0 >> a.log2G] = sc[0];
+    } else {
+#pragma unroll
+      for (int i = 0; i < NG; ++i)
+        if ((i & (gg - 1)) == 0) srow[(c0 + 8 * i) >> a.log2G] = sc[i];
+    }
+    const float2 mg = make_float2(MAGIC, MAGIC);
+#pragma unroll
+    for (int w = 0; w < NWD; ++w) {
+      const int gi = w * (CPW / 8);
+      uint32_t tt[CPW];
+      if (!slow[gi]) {
+        const float2 ff = make_float2(fw[gi], fw[gi]);
+#pragma unroll
+        for (int j = 0; j < CPW; j += 2) {
+          const float2 r = __ffma2_rn(xp[(CPW * w + j) / 2], ff, mg);
+          tt[j] = __float_as_uint(r.x);
+          tt[j + 1] = __float_as_uint(r.y);
+        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < CPW; j += 2) {
+          tt[j] = code_magic_clamped(xp[(CPW * w + j) / 2].x, fw[gi], QMAX, MAGIC);
+          tt[j + 1] = code_magic_clamped(xp[(CPW * w + j) / 2].y, fw[gi], QMAX, MAGIC);
+        }
+      }
+      if constexpr (BITS == 4) words[w] = pack8_int4(*reinterpret_cast<const uint32_t(*)[8]>(tt));
+      else words[w] = pack16_int2(*reinterpret_cast<const uint32_t(*)[16]>(tt));
+    }
+  }
+  uint32_t* dst = reinterpret_cast<uint32_t*>(a.codes + row * (int64_t)(a.K / CPW) * 4) + c0 / CPW;
+  if constexpr (NWD >= 4) {
+#pragma unroll
+    for (int v = 0; v < NWD / 4; ++v)
+      reinterpret_cast<uint4*>(dst)[v] = make_uint4(words[4 * v], words[4 * v + 1], words[4 * v + 2], words[4 * v + 3]);
+  } else if constexpr (NWD == 2) {
+    *reinterpret_cast<uint2*>(dst) = make_uint2(words[0], words[1]);
+  } else {
+    dst[0] = words[0];
+  }
+}
+
+template <int LOGN, bool BF16, int MODE, int BITS, int GT>
 __global__ void __launch_bounds__(Cfg<LOGN>::THREADS, 1) fwht_kernel(const Args a) {
   using C = Cfg<LOGN>;
   constexpr int N = C::N, ELOG = C::ELOG, E = C::E, HB = C::HB, VA = C::VA, TPC = C::TPC;
   constexpr int NV = C::NV, NH = C::NH, SLOTS = C::SLOTS, SSTRIDE = C::SSTRIDE;
-  constexpr int NP = E / 2;  // fp32 pairs per thread: xp[i] = coordinates (2i, 2i+1) of the layout
+  constexpr int NP = E / 2;   // fp32 pairs per thread: xp[i] = layout coordinates (2i, 2i+1)
+  constexpr int NW = NV / 2;  // pairs per phase-A run
   extern __shared__ __align__(128) float smem[];
   float* sbuf = smem;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SLOTS * SSTRIDE);
@@ -224,6 +374,20 @@ __global__ void __launch_bounds__(Cfg<LOGN>::THREADS, 1) fwht_kernel(const Args 
   asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   __syncthreads();
 
+  // per-thread shared-memory bases (loop invariant); compile-time offsets are added per access
+  const int T = t << VA;                       // first coordinate of this thread's phase-A runs
+  constexpr int NPA = VA >= 5 ? 1 : (1 << (5 - (VA < 2 ? 2 : VA)));
+  constexpr bool B5 = (LOGN == 9 || LOGN == 11);  // extra swizzle term from coordinate bit 5
+  // phase-A store bases: pa[k] = T ^ (k << max(VA, 2)); with the bit-5 term (VA = 3, bit 5 =
+  // thread bit 2) the XOR on coordinate bit 2 also depends on the thread: fold it in.
+  const int tb = B5 ? ((T >> 5) & 1) << 2 : 0;
+  int pa[NPA];
+#pragma unroll
+  for (int k = 0; k < NPA; ++k) pa[k] = (T ^ (k << (VA < 2 ? 2 : VA))) ^ tb;
+  int qb[8];                                    // phase-B load bases
+#pragma unroll
+  for (int r = 0; r < 8; ++r) qb[r] = (t << ELOG) + ((4 * r) ^ ((t & 7) << 2));
+
   const int64_t units = a.M * a.chunks;
   const int64_t stride = (int64_t)gridDim.x * SLOTS;
   int64_t u = (int64_t)blockIdx.x * SLOTS + slot;
@@ -238,7 +402,6 @@ __global__ void __launch_bounds__(Cfg<LOGN>::THREADS, 1) fwht_kernel(const Args 
   };
   if (t == 0 && u < units) stage_issue(bar, buf, src_of(row, chunk), chunk_bytes);
   uint32_t parity = 0;
-  const int log2G = a.log2G;
 
   for (; u < units; u += stride) {
     const int cbase = chunk * N;
@@ -247,46 +410,42 @@ __global__ void __launch_bounds__(Cfg<LOGN>::THREADS, 1) fwht_kernel(const Args 
     parity ^= 1u;
 
     // ---------------- phase A: runs of NV elements from the staged chunk, signs, fp32 pairs
-    {
-      const int run0 = t << VA;
-      if constexpr (BF16) {
-        constexpr int NW = NV / 2;
-        const uint32_t* sraw = reinterpret_cast<const uint32_t*>(buf);
+    if constexpr (BF16) {
+      const uint32_t* sraw = reinterpret_cast<const uint32_t*>(buf) + (T >> 1);
+      const uint32_t* smk = smask + ((cbase + T) >> 1);
+      const bool sg = MODE != MODE_APPLY_INV && has_signs;
 #pragma unroll
-        for (int h = 0; h < NH; ++h) {
-          const int w0 = (run0 + (h << ELOG)) >> 1;   // word index within the chunk
-          uint32_t raw[NW], m[NW];
-          load_masks<NW>(raw, sraw, w0, true);
-          load_masks<NW>(m, smask, (cbase >> 1) + w0, MODE != MODE_APPLY_INV && has_signs);
+      for (int h = 0; h < NH; ++h) {
+        uint32_t raw[NW], m[NW];
+        load_masks<NW>(raw, sraw + h * (E / 2), 0, true);
+        load_masks<NW>(m, smk + h * (E / 2), 0, sg);
+#pragma unroll
+        for (int w = 0; w < NW; ++w) {
+          const uint32_t v = raw[w] ^ m[w];
+          xp[h * NW + w] = make_float2(bf16lo(v), bf16hi(v));
+        }
+      }
+    } else {
+#pragma unroll
+      for (int h = 0; h < NH; ++h) {
+        const float* src = buf + T + (h << ELOG);
+        if constexpr (NV >= 4) {
+#pragma unroll
+          for (int v = 0; v < NV / 4; ++v) {
+            const float4 q = reinterpret_cast<const float4*>(src)[v];
+            xp[h * NW + 2 * v] = make_float2(q.x, q.y);
+            xp[h * NW + 2 * v + 1] = make_float2(q.z, q.w);
+          }
+        } else {
+          xp[h * NW] = *reinterpret_cast<const float2*>(src);
+        }
+        if (MODE != MODE_APPLY_INV && has_signs) {
+          uint32_t m[NW];
+          load_masks<NW>(m, smask + ((cbase + T) >> 1) + h * (E / 2), 0, true);
 #pragma unroll
           for (int w = 0; w < NW; ++w) {
-            const uint32_t v = raw[w] ^ m[w];
-            xp[h * NW + w] = make_float2(bf16lo(v), bf16hi(v));
-          }
-        }
-      } else {
-#pragma unroll
-        for (int h = 0; h < NH; ++h) {
-          const int i0 = run0 + (h << ELOG);
-          constexpr int NW = NV / 2;
-          if constexpr (NV >= 4) {
-#pragma unroll
-            for (int v = 0; v < NV / 4; ++v) {
-              const float4 q = *reinterpret_cast<const float4*>(buf + i0 + 4 * v);
-              xp[h * NW + 2 * v] = make_float2(q.x, q.y);
-              xp[h * NW + 2 * v + 1] = make_float2(q.z, q.w);
-            }
-          } else {
-            xp[h * NW] = *reinterpret_cast<const float2*>(buf + i0);
-          }
-          if (MODE != MODE_APPLY_INV && has_signs) {
-            uint32_t m[NW];
-            load_masks<NW>(m, smask, (cbase + i0) >> 1, true);
-#pragma unroll
-            for (int w = 0; w < NW; ++w) {
-              xp[h * NW + w].x = __uint_as_float(__float_as_uint(xp[h * NW + w].x) ^ (m[w] << 16));
-              xp[h * NW + w].y = __uint_as_float(__float_as_uint(xp[h * NW + w].y) ^ (m[w] & 0x80000000u));
-            }
+            xp[h * NW + w].x = __uint_as_float(__float_as_uint(xp[h * NW + w].x) ^ (m[w] << 16));
+            xp[h * NW + w].y = __uint_as_float(__float_as_uint(xp[h * NW + w].y) ^ (m[w] & 0x80000000u));
           }
         }
       }
@@ -306,22 +465,28 @@ __global__ void __launch_bounds__(Cfg<LOGN>::THREADS, 1) fwht_kernel(const Args 
       slot_sync<TPC>(slot);  // every thread has read its staged runs
 #pragma unroll
       for (int h = 0; h < NH; ++h) {
-        const int i0 = (t << VA) + (h << ELOG);
-        constexpr int NW = NV / 2;
+        constexpr int SH = VA < 2 ? 2 : VA;        // lowest XOR bit not inside a run
+        const int X = (h & 7) << 2;                // phys = i ^ X, i = T + (h << ELOG) + 4v
+        const int base = pa[(X >> SH) & (NPA - 1)] + (h << ELOG);
         if constexpr (NV >= 4) {
 #pragma unroll
           for (int v = 0; v < NV / 4; ++v) {
             const float2 p0 = xp[h * NW + 2 * v], p1 = xp[h * NW + 2 * v + 1];
-            *reinterpret_cast<float4*>(buf + swz<LOGN>(i0 + 4 * v)) = make_float4(p0.x, p0.y, p1.x, p1.y);
+            // bit 2 of the physical index: (4v ^ X) bit 2, flipped by tb (folded into base)
+            const int off = (4 * v) ^ (X & ((1 << SH) - 1));
+            const int adr = B5 ? (base ^ (off & 4)) + (off & ~4) : base + off;
+            *reinterpret_cast<float4*>(buf + adr) = make_float4(p0.x, p0.y, p1.x, p1.y);
           }
         } else {
-          *reinterpret_cast<float2*>(buf + swz<LOGN>(i0)) = xp[h * NW];
+          *reinterpret_cast<float2*>(buf + base) = xp[h * NW];
         }
       }
       slot_sync<TPC>(slot);
 #pragma unroll
       for (int jc = 0; jc < E / 4; ++jc) {
-        const float4 q = *reinterpret_cast<const float4*>(buf + swz<LOGN>((t << ELOG) + 4 * jc));
+        // coordinate (t << ELOG) + 4jc; bit 5 of it is bit 3 of jc (compile-time)
+        const int r = B5 ? ((jc & 7) ^ ((jc >> 3) & 1)) : (jc & 7);
+        const float4 q = *reinterpret_cast<const float4*>(buf + qb[r] + 32 * (jc >> 3));
         xp[2 * jc] = make_float2(q.x, q.y);
         xp[2 * jc + 1] = make_float2(q.z, q.w);
       }
@@ -344,7 +509,6 @@ __global__ void __launch_bounds__(Cfg<LOGN>::THREADS, 1) fwht_kernel(const Args 
     row = nrow;
     chunk = nchunk;
 
-    // xp[j/2] holds z for chunk coordinates (t << ELOG) + j; y = z * norm
     const int c0 = cbase + (t << ELOG);  // row coordinate of the first element
     if constexpr (MODE == MODE_APPLY || MODE == MODE_APPLY_INV) {
       float* dst = a.Y + cur_row * a.ldy + c0;
@@ -363,108 +527,17 @@ __global__ void __launch_bounds__(Cfg<LOGN>::THREADS, 1) fwht_kernel(const Args 
         *reinterpret_cast<float4*>(dst + 4 * jc) = q;
       }
     } else {
-      // ---------------- quantisation: groups of G contiguous coordinates.
-      constexpr float QMAX = BITS == 4 ? 7.0f : 1.0f;
-      constexpr float MAGIC = BITS == 4 ? 8388616.0f : 8388610.0f;  // 2^23 + qmax + 1
-      constexpr int NG = E / 8;
-      const int gg = a.G >> 3;  // granules per group (power of two)
-      float gm[NG];
-#pragma unroll
-      for (int i = 0; i < NG; ++i) {
-        const float2 p0 = xp[4 * i], p1 = xp[4 * i + 1], p2 = xp[4 * i + 2], p3 = xp[4 * i + 3];
-        float mx = max3(p0.x, p0.y, p1.x);
-        float mn = min3(p0.x, p0.y, p1.x);
-        mx = max3(mx, p1.y, p2.x);
-        mn = min3(mn, p1.y, p2.x);
-        mx = max3(mx, p2.y, p3.x);
-        mn = min3(mn, p2.y, p3.x);
-        mx = fmaxf(mx, p3.y);
-        mn = fminf(mn, p3.y);
-        gm[i] = fmaxf(mx, -mn);
-      }
-#pragma unroll
-      for (int st = 1; st < NG; st <<= 1) {
-        if (st < gg) {
-#pragma unroll
-          for (int i = 0; i + st < NG; i += 2 * st) gm[i] = fmaxf(gm[i], gm[i + st]);
-        }
-      }
-      if (a.G > E) {
-        const unsigned lanes = slot_lanes<TPC>();
-        for (int o = 1; o < a.G / E; o <<= 1) gm[0] = fmaxf(gm[0], __shfl_xor_sync(lanes, gm[0], o));
-      }
-      float fw[NG];
-      bool slow[NG];
-      uint16_t sc[NG];
-#pragma unroll
-      for (int i = 0; i < NG; ++i) {
-        if ((i & (gg - 1)) == 0) {
-          sc[i] = group_scale(gm[i], a.norm, QMAX, &fw[i], &slow[i]);
-        } else {
-          fw[i] = fw[i - 1];
-          slow[i] = slow[i - 1];
-          sc[i] = sc[i - 1];
-        }
-      }
-      {
-        uint16_t* srow = a.scales + cur_row * a.ngroups;
-        if (a.G > E) {
-          if ((t & (a.G / E - 1)) == 0) srow[c0 >> log2G] = sc[0];
-        } else {
-#pragma unroll
-          for (int i = 0; i < NG; ++i)
-            if ((i & (gg - 1)) == 0) srow[(c0 + 8 * i) >> log2G] = sc[i];
-        }
-      }
-      constexpr int CPW = 32 / BITS;   // codes per 32-bit word
-      constexpr int NWD = E / CPW;     // words per thread
-      const float2 mg = make_float2(MAGIC, MAGIC);
-      uint32_t words[NWD];
-#pragma unroll
-      for (int w = 0; w < NWD; ++w) {
-        const int gi = w * (CPW / 8);    // granule of the word's first code
-        uint32_t tt[CPW];
-        if (!slow[gi]) {
-          const float2 ff = make_float2(fw[gi], fw[gi]);
-#pragma unroll
-          for (int j = 0; j < CPW; j += 2) {
-            const float2 r = __ffma2_rn(xp[(CPW * w + j) / 2], ff, mg);
-            tt[j] = __float_as_uint(r.x);
-            tt[j + 1] = __float_as_uint(r.y);
-          }
-        } else {
-#pragma unroll
-          for (int j = 0; j < CPW; j += 2) {
-            tt[j] = code_magic_clamped(xp[(CPW * w + j) / 2].x, fw[gi], QMAX, MAGIC);
-            tt[j + 1] = code_magic_clamped(xp[(CPW * w + j) / 2].y, fw[gi], QMAX, MAGIC);
-          }
-        }
-        if constexpr (BITS == 4) {
-          words[w] = pack8_int4(*reinterpret_cast<const uint32_t(*)[8]>(tt));
-        } else {
-          words[w] = pack16_int2(*reinterpret_cast<const uint32_t(*)[16]>(tt));
-        }
-      }
-      uint32_t* dst = reinterpret_cast<uint32_t*>(a.codes + cur_row * (int64_t)(a.K / CPW) * 4) + c0 / CPW;
-      if constexpr (NWD >= 4) {
-#pragma unroll
-        for (int v = 0; v < NWD / 4; ++v)
-          reinterpret_cast<uint4*>(dst)[v] = make_uint4(words[4 * v], words[4 * v + 1], words[4 * v + 2], words[4 * v + 3]);
-      } else if constexpr (NWD == 2) {
-        *reinterpret_cast<uint2*>(dst) = make_uint2(words[0], words[1]);
-      } else {
-        dst[0] = words[0];
-      }
+      quantise_store<LOGN, BITS, GT, E, TPC>(a, xp, cur_row, c0, t);
     }
   }
 }
 
-template <int LOGN, bool BF16, int MODE, int BITS>
+template <int LOGN, bool BF16, int MODE, int BITS, int GT>
 rot_status launch_one(const Args& a, cudaStream_t s) {
   using C = Cfg<LOGN>;
   const size_t smem = (size_t)C::SLOTS * C::SSTRIDE * 4 + (size_t)((C::SLOTS + 1) & ~1) * 8 + (size_t)(a.K / 2) * 4;
   if (smem > 227 * 1024) return set_error(ROT_EUNSUPPORTED, "fused rotation: sign table too large for shared memory");
-  auto kern = fwht_kernel<LOGN, BF16, MODE, BITS>;
+  auto kern = fwht_kernel<LOGN, BF16, MODE, BITS, GT>;
   static int configured[64] = {0};  // per device: the opt-in limit is set once
   int dev = 0;
   cudaGetDevice(&dev);
@@ -482,18 +555,29 @@ rot_status launch_one(const Args& a, cudaStream_t s) {
   return ROT_OK;
 }
 
+template <int LOGN, bool BF16, int MODE, int BITS>
+rot_status launch_g(const Args& a, cudaStream_t s) {
+  // compile-time group sizes for the common shapes (bf16 quantisation on large chunks)
+  if constexpr (MODE == MODE_QUANT && BF16 && (LOGN == 8 || LOGN >= 11)) {
+    if (a.G == 32) return launch_one<LOGN, BF16, MODE, BITS, 32>(a, s);
+    if (a.G == 64) return launch_one<LOGN, BF16, MODE, BITS, 64>(a, s);
+    if (a.G == 128) return launch_one<LOGN, BF16, MODE, BITS, 128>(a, s);
+  }
+  return launch_one<LOGN, BF16, MODE, BITS, 0>(a, s);
+}
+
 template <bool BF16, int MODE, int BITS>
 rot_status dispatch_logn(int logn, const Args& a, cudaStream_t s) {
   switch (logn) {
-    case 5: return launch_one<5, BF16, MODE, BITS>(a, s);
-    case 6: return launch_one<6, BF16, MODE, BITS>(a, s);
-    case 7: return launch_one<7, BF16, MODE, BITS>(a, s);
-    case 8: return launch_one<8, BF16, MODE, BITS>(a, s);
-    case 9: return launch_one<9, BF16, MODE, BITS>(a, s);
-    case 10: return launch_one<10, BF16, MODE, BITS>(a, s);
-    case 11: return launch_one<11, BF16, MODE, BITS>(a, s);
-    case 12: return launch_one<12, BF16, MODE, BITS>(a, s);
-    case 13: return launch_one<13, BF16, MODE, BITS>(a, s);
+    case 5: return launch_g<5, BF16, MODE, BITS>(a, s);
+    case 6: return launch_g<6, BF16, MODE, BITS>(a, s);
+    case 7: return launch_g<7, BF16, MODE, BITS>(a, s);
+    case 8: return launch_g<8, BF16, MODE, BITS>(a, s);
+    case 9: return launch_g<9, BF16, MODE, BITS>(a, s);
+    case 10: return launch_g<10, BF16, MODE, BITS>(a, s);
+    case 11: return launch_g<11, BF16, MODE, BITS>(a, s);
+    case 12: return launch_g<12, BF16, MODE, BITS>(a, s);
+    case 13: return launch_g<13, BF16, MODE, BITS>(a, s);
     default: return set_error(ROT_EUNSUPPORTED, "fused rotation: chunk size out of range");
   }
 }

@@ -101,16 +101,17 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
 
 // Scale / code-factor of one quantisation group.
 //   m_z   : max |z| over the group, z the un-normalised rotated values (y = z * norm)
-// Returns the binary16 scale bits; *f receives the factor with v = z * f ~= y / s, nudged
-// up by 2^-22 relative so that exact ties of z * f round away from zero; *slow is set
-// when the scale is zero, subnormal or not finite (codes need clamping then).
+// Returns the binary16 scale bits (fp32 IEEE quotient absmax / qmax, rounded to binary16);
+// *f receives the factor with v = z * f ~= y / s (within an ulp or two), nudged up by
+// 2^-22 relative so that exact ties of z * f round away from zero; *slow is set when the
+// scale is zero, subnormal or not finite (codes need clamping then).
 __device__ __forceinline__ uint16_t group_scale(float m_z, float norm, float qmax, float* f,
                                                 bool* slow) {
   float my = m_z * norm;
   __half s16 = __float2half_rn(__fdiv_rn(my, qmax));
   float s = __half2float(s16);
   bool ok = (s >= 6.103515625e-05f) && (s <= 65504.0f);  // normal binary16
-  float fv = (s > 0.0f && s <= 65504.0f) ? __fdiv_rn(norm, s) : 0.0f;
+  float fv = (s > 0.0f && s <= 65504.0f) ? __fmul_rn(norm, __frcp_rn(s)) : 0.0f;
   *f = __fmul_rn(fv, 1.0f + 0x1p-22f);
   *slow = !ok;
   return __half_as_ushort(s16);
