@@ -12,13 +12,14 @@
 // same K permutation is applied to both operands, so every group sum is unchanged.
 //
 // Tile: 128 rows of A x 256 rows of W per CTA; K in blocks of 128 (one 128-byte swizzle
-// atom of int8 per row), 4 UMMAs of K = 32 per block.
+// atom of int8 per row), 4 UMMAs of K = 32 per block, 3-stage smem ring. (A 128 x 128 tile
+// avoids the epilogue's register spills but re-reads A twice as often and measured slower.)
 // Warp roles (512 threads, launched with 128 registers each). setmaxnreg acts on whole
 // warpgroups, so roles are aligned to them: warpgroups 0-1 (epilogue) grow to 168 registers,
 // warpgroups 2-3 (producers + MMA warp) shrink to 88: 256*168 + 256*88 = 512*128.
 //   warps 0-7   epilogue: two warpgroups, 128 columns each; after each group they read
 //               the int32 partials from TMEM, apply the group scales and accumulate in
-//               fp32 registers;
+//               fp32 registers (packed f32x2 FMAs);
 //   warps 8-14  producers: load packed codes from global memory (register prefetch two
 //               K-blocks ahead), unpack, store into the swizzled K-major smem layout, then
 //               fence.proxy.async + mbarrier arrive;
@@ -57,14 +58,14 @@ constexpr int EPI_REGS = 168, PROD_REGS = 88;  // per warpgroup role
 static_assert(THREADS == 512, "register split assumes 512 threads");
 static_assert(N_EPI == 256 && N_PROD + 32 == 256, "roles must fill whole warpgroups");
 static_assert(N_EPI * EPI_REGS + (N_PROD + 32) * PROD_REGS <= THREADS * LAUNCH_REGS, "register split");
-constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t TMEM_COLS = 2 * BN;   // two group accumulators (all 512 columns)
 constexpr uint32_t BIAS_BITS = 0x4B400000u;  // 1.5 * 2^23
 constexpr float BIAS_F = 12582912.0f;
 constexpr unsigned long long WAIT_NS = 2000000000ull;
 
 // smem layout (offsets from a 1024-byte aligned base)
 constexpr int OFF_STAGES = 0;
-constexpr int OFF_SCALES = STAGES * STAGE_BYTES;          // [2][BN] float2 (sW/256, -bias*sW/256)
+constexpr int OFF_SCALES = STAGES * STAGE_BYTES;          // [2][2][BN] fp32: sW/256 and -1.5*2^23*sW/256
 constexpr int OFF_BARS = OFF_SCALES + 2 * BN * 8;
 constexpr int OFF_TMEM = OFF_BARS + 16 * 8;
 constexpr int SMEM_BYTES = OFF_TMEM + 16 + 1024;          // + alignment slack
@@ -163,13 +164,11 @@ __device__ __forceinline__ void umma_commit(uint64_t* bar) {
                : "memory");
 }
 
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-      : "r"(taddr)
-      : "memory");
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t (&r)[8]) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+               : "r"(taddr)
+               : "memory");
 }
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_st16_const(uint32_t taddr, uint32_t v) {
@@ -180,10 +179,21 @@ __device__ __forceinline__ void tmem_st16_const(uint32_t taddr, uint32_t v) {
 }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
+// Ordered shared-memory vector load: kept next to the TMEM load it serves, so the scale loads
+// of all column chunks are not hoisted ahead (which would need a register per loaded value).
+__device__ __forceinline__ float4 lds128(const float* p) {
+  float4 v;
+  asm volatile("ld.shared.v4.f32 {%0,%1,%2,%3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(smem_u32(p)));
+  return v;
+}
+
 __device__ __forceinline__ void named_bar(int id, int n) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
 }
 
+template <bool PARTIALS>
 __global__ void __launch_bounds__(THREADS, 1) w4a4_kernel(const Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -194,7 +204,7 @@ __global__ void __launch_bounds__(THREADS, 1) w4a4_kernel(const Params p) {
   uint64_t* tempty = bars + 2 * STAGES + 2;  // [2] epilogue -> MMA
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_TMEM);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + OFF_TMEM + 8);
-  float2* sc = reinterpret_cast<float2*>(smem + OFF_SCALES);
+  float* sc = reinterpret_cast<float*>(smem + OFF_SCALES);  // [buf][0: sW/256, 1: c][BN]
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -245,45 +255,65 @@ __global__ void __launch_bounds__(THREADS, 1) w4a4_kernel(const Params p) {
     mbar_arrive(&tempty[0]);
     mbar_arrive(&tempty[1]);
 
-    float acc[EPI_COLS];
+    // fp32 accumulators as pairs of adjacent columns
+    float2 acc[EPI_COLS / 2];
 #pragma unroll
-    for (int j = 0; j < EPI_COLS; ++j) acc[j] = 0.0f;
+    for (int j = 0; j < EPI_COLS / 2; ++j) acc[j] = make_float2(0.0f, 0.0f);
     const bool row_ok = m < p.M;
     const int n_col = n0 + ep_tid;            // the column whose scale this thread stages
+    // scales of the next group are fetched one group ahead
+    float sw_next = 0.0f, sa_next = 0.0f;
+    if (!PARTIALS) {
+      if (ep_tid < BN && n_col < p.N) sw_next = __half2float(__ushort_as_half(p.Ws[(int64_t)n_col * NG]));
+      if (row_ok) sa_next = __half2float(__ushort_as_half(p.As[(int64_t)m * NG]));
+    }
     bool ok = true;
     for (int g = 0; g < NG; ++g) {
-      // stage the column scales of group g: (sW/256, -1.5*2^23 * sW/256)
-      if (p.Ws && ep_tid < BN) {
-        float sw = 0.0f;
-        if (n_col < p.N) sw = __half2float(__ushort_as_half(p.Ws[(int64_t)n_col * NG + g])) * (1.0f / 256.0f);
-        sc[(g & 1) * BN + ep_tid] = make_float2(sw, -BIAS_F * sw);
+      const float sa = sa_next;
+      if (!PARTIALS) {
+        if (ep_tid < BN) {
+          const float sw = sw_next * (1.0f / 256.0f);
+          sc[((g & 1) * 2 + 0) * BN + ep_tid] = sw;
+          sc[((g & 1) * 2 + 1) * BN + ep_tid] = -BIAS_F * sw;
+        }
+        if (g + 1 < NG) {
+          if (ep_tid < BN && n_col < p.N) sw_next = __half2float(__ushort_as_half(p.Ws[(int64_t)n_col * NG + g + 1]));
+          if (row_ok) sa_next = __half2float(__ushort_as_half(p.As[(int64_t)m * NG + g + 1]));
+        }
       }
-      const float sa = (p.As && row_ok) ? __half2float(__ushort_as_half(p.As[(int64_t)m * NG + g])) : 0.0f;
       named_bar(1, N_EPI);
       const int b = g & 1;
       if (!ok || !mbar_wait(&tfull[b], (g >> 1) & 1, abort_flag)) { ok = false; continue; }
       tc_fence_after();
       const uint32_t base = lane_addr + b * BN + wg * EPI_COLS;
-      const float2* scg = sc + (g & 1) * BN + wg * EPI_COLS;
-      uint32_t rr[16];
+      const float* scw = sc + ((g & 1) * 2 + 0) * BN + wg * EPI_COLS;
+      const float* scc = sc + ((g & 1) * 2 + 1) * BN + wg * EPI_COLS;
+      const float2 sa2 = make_float2(sa, sa);
 #pragma unroll
-      for (int c = 0; c < EPI_COLS / 16; ++c) {
-        tmem_ld16(base + c * 16, rr);
+      for (int c = 0; c < EPI_COLS / 8; ++c) {
+        uint32_t rr[8];
+        tmem_ld8(base + c * 8, rr);
         tmem_wait_ld();
-        if (p.P == nullptr) {
+        if constexpr (!PARTIALS) {
 #pragma unroll
-          for (int j = 0; j < 16; j += 2) {
-            const float4 s2 = *reinterpret_cast<const float4*>(scg + c * 16 + j);
-            const float t0 = fmaf(__uint_as_float(rr[j]), s2.x, s2.y);
-            const float t1 = fmaf(__uint_as_float(rr[j + 1]), s2.z, s2.w);
-            acc[c * 16 + j] = fmaf(t0, sa, acc[c * 16 + j]);
-            acc[c * 16 + j + 1] = fmaf(t1, sa, acc[c * 16 + j + 1]);
+          for (int j = 0; j < 8; j += 4) {
+            const float4 w4 = lds128(scw + c * 8 + j);
+            const float4 c4 = lds128(scc + c * 8 + j);
+            const float2 u0 = make_float2(__uint_as_float(rr[j]), __uint_as_float(rr[j + 1]));
+            const float2 u1 = make_float2(__uint_as_float(rr[j + 2]), __uint_as_float(rr[j + 3]));
+            // exact P*sW (the bias cancels inside one rounding), then acc += (P*sW)*sA
+            const float2 t0 = __ffma2_rn(u0, make_float2(w4.x, w4.y), make_float2(c4.x, c4.y));
+            const float2 t1 = __ffma2_rn(u1, make_float2(w4.z, w4.w), make_float2(c4.z, c4.w));
+            acc[(c * 8 + j) / 2] = __ffma2_rn(t0, sa2, acc[(c * 8 + j) / 2]);
+            acc[(c * 8 + j) / 2 + 1] = __ffma2_rn(t1, sa2, acc[(c * 8 + j) / 2 + 1]);
           }
-        } else if (row_ok) {
+        } else {
+          if (row_ok) {
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const int n = n0 + wg * EPI_COLS + c * 16 + j;
-            if (n < p.N) p.P[((int64_t)m * p.N + n) * NG + g] = ((int32_t)(rr[j] - BIAS_BITS)) / 256;
+            for (int j = 0; j < 8; ++j) {
+              const int n = n0 + wg * EPI_COLS + c * 8 + j;
+              if (n < p.N) p.P[((int64_t)m * p.N + n) * NG + g] = ((int32_t)(rr[j] - BIAS_BITS)) / 256;
+            }
           }
         }
       }
@@ -294,23 +324,25 @@ __global__ void __launch_bounds__(THREADS, 1) w4a4_kernel(const Params p) {
       tc_fence_before();
       mbar_arrive(&tempty[b]);
     }
-    if (ok && p.P == nullptr && row_ok) {
+    if (!PARTIALS && ok && row_ok) {
       const int nb = n0 + wg * EPI_COLS;
       if (!p.c_bf16) {
         float* crow = static_cast<float*>(p.C) + (int64_t)m * p.N + nb;
 #pragma unroll
         for (int j = 0; j < EPI_COLS; j += 4)
-          if (nb + j < p.N) *reinterpret_cast<float4*>(crow + j) = make_float4(acc[j], acc[j + 1], acc[j + 2], acc[j + 3]);
+          if (nb + j < p.N)
+            *reinterpret_cast<float4*>(crow + j) =
+                make_float4(acc[j / 2].x, acc[j / 2].y, acc[j / 2 + 1].x, acc[j / 2 + 1].y);
       } else {
         __nv_bfloat16* crow = static_cast<__nv_bfloat16*>(p.C) + (int64_t)m * p.N + nb;
 #pragma unroll
         for (int j = 0; j < EPI_COLS; j += 8) {
           if (nb + j < p.N) {
             uint4 v;
-            __nv_bfloat162 h0 = __floats2bfloat162_rn(acc[j], acc[j + 1]);
-            __nv_bfloat162 h1 = __floats2bfloat162_rn(acc[j + 2], acc[j + 3]);
-            __nv_bfloat162 h2 = __floats2bfloat162_rn(acc[j + 4], acc[j + 5]);
-            __nv_bfloat162 h3 = __floats2bfloat162_rn(acc[j + 6], acc[j + 7]);
+            __nv_bfloat162 h0 = __floats2bfloat162_rn(acc[j / 2].x, acc[j / 2].y);
+            __nv_bfloat162 h1 = __floats2bfloat162_rn(acc[j / 2 + 1].x, acc[j / 2 + 1].y);
+            __nv_bfloat162 h2 = __floats2bfloat162_rn(acc[j / 2 + 2].x, acc[j / 2 + 2].y);
+            __nv_bfloat162 h3 = __floats2bfloat162_rn(acc[j / 2 + 3].x, acc[j / 2 + 3].y);
             v.x = *reinterpret_cast<uint32_t*>(&h0);
             v.y = *reinterpret_cast<uint32_t*>(&h1);
             v.z = *reinterpret_cast<uint32_t*>(&h2);
@@ -325,22 +357,30 @@ __global__ void __launch_bounds__(THREADS, 1) w4a4_kernel(const Params p) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 88;");
     const int pt = threadIdx.x - N_EPI;    // 0..N_PROD-1
     const int64_t ldp = p.K / 2;           // packed bytes per row
-    // chunk q = pt + N_PROD*i: rows 0..BM-1 of A then 0..BN-1 of W, 4 chunks (16 B = 32 codes) per row
+    // chunk q = pt + N_PROD*i: rows 0..BM-1 of A then 0..BN-1 of W, 4 chunks (16 B = 32 codes)
+    // per row. The global row pointers are fixed for the CTA; nullptr marks rows beyond M / N.
+    const uint8_t* gsrc[PROD_CHUNKS];
+#pragma unroll
+    for (int i = 0; i < PROD_CHUNKS; ++i) {
+      const int q = pt + N_PROD * i;
+      const int r = q >> 2, c = q & 3;
+      const uint8_t* src = nullptr;
+      if (q < N_CHUNKS) {
+        if (r < BM) {
+          if (m0 + r < p.M) src = p.Aq + (int64_t)(m0 + r) * ldp + c * 16;
+        } else {
+          if (n0 + r - BM < p.N) src = p.Wq + (int64_t)(n0 + r - BM) * ldp + c * 16;
+        }
+      }
+      gsrc[i] = src;
+    }
     auto load = [&](int kb, uint4 (&dst)[PROD_CHUNKS]) {
+      const int64_t koff = (int64_t)kb * (KB / 2);
 #pragma unroll
       for (int i = 0; i < PROD_CHUNKS; ++i) {
-        const int q = pt + N_PROD * i;
-        const int r = q >> 2, c = q & 3;
-        const int64_t kbyte = (int64_t)kb * (KB / 2) + c * 16;
+        const int c = (pt + N_PROD * i) & 3;
         uint4 v = make_uint4(0u, 0u, 0u, 0u);
-        if (q >= N_CHUNKS) {
-        } else if (r < BM) {
-          const int mm = m0 + r;
-          if (mm < p.M && kbyte < ldp) v = __ldg(reinterpret_cast<const uint4*>(p.Aq + (int64_t)mm * ldp + kbyte));
-        } else {
-          const int nn = n0 + r - BM;
-          if (nn < p.N && kbyte < ldp) v = __ldg(reinterpret_cast<const uint4*>(p.Wq + (int64_t)nn * ldp + kbyte));
-        }
+        if (gsrc[i] != nullptr && koff + c * 16 < ldp) v = __ldg(reinterpret_cast<const uint4*>(gsrc[i] + koff));
         dst[i] = v;
       }
     };
@@ -436,11 +476,14 @@ rot_status w4a4_launch(const uint8_t* Aq, const uint16_t* As, const uint8_t* Wq,
   if (dev < 64 && !configured[dev]) {
     // The setmaxnreg split is only valid for the register count it was sized for: refuse
     // to launch otherwise (an over-subscribed split would wait for registers forever).
-    cudaFuncAttributes fa;
-    ROT_CUDA_TRY(cudaFuncGetAttributes(&fa, w4a4_kernel));
-    if (fa.numRegs != LAUNCH_REGS)
-      return set_error(ROT_EUNSUPPORTED, "w4a4_linear: kernel built with an unexpected register count");
-    ROT_CUDA_TRY(cudaFuncSetAttribute(w4a4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES));
+    for (int v = 0; v < 2; ++v) {
+      const void* k = v ? (const void*)w4a4_kernel<true> : (const void*)w4a4_kernel<false>;
+      cudaFuncAttributes fa;
+      ROT_CUDA_TRY(cudaFuncGetAttributes(&fa, k));
+      if (fa.numRegs != LAUNCH_REGS)
+        return set_error(ROT_EUNSUPPORTED, "w4a4_linear: kernel built with an unexpected register count");
+      ROT_CUDA_TRY(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES));
+    }
     configured[dev] = 1;
   }
   Params p{};
@@ -456,7 +499,8 @@ rot_status w4a4_launch(const uint8_t* Aq, const uint16_t* As, const uint8_t* Wq,
   p.G = G;
   p.c_bf16 = c_dtype == ROT_BF16;
   dim3 grid((unsigned)((N + BN - 1) / BN), (unsigned)((M + BM - 1) / BM));
-  w4a4_kernel<<<grid, THREADS, SMEM_BYTES, s>>>(p);
+  if (partials) w4a4_kernel<true><<<grid, THREADS, SMEM_BYTES, s>>>(p);
+  else w4a4_kernel<false><<<grid, THREADS, SMEM_BYTES, s>>>(p);
   ROT_CUDA_TRY(cudaGetLastError());
   return ROT_OK;
 }
