@@ -75,6 +75,8 @@ struct Args {
   int log2G;
   int64_t ngroups;   // K / G
   float norm;
+  float cdiv;        // fp32(norm / qmax)
+  float cf;          // fp32(norm * (1 + 2^-22))
 };
 
 enum { MODE_APPLY = 0, MODE_APPLY_INV = 1, MODE_QUANT = 2 };
@@ -125,19 +127,19 @@ __device__ __forceinline__ void slot_sync(int slot) {
 __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
 
-// Pack 8 offset codes (low bytes of t[0..7], each 8 + q) into one int4 word.
+// Pack 8 offset codes (low bytes of t[0..7], each 8 + q) into one int4 word: byte j holds
+// codes 2j (low nibble) and 2j+1 (high nibble), two's complement.
 __device__ __forceinline__ uint32_t pack8_int4(const uint32_t (&t)[8]) {
-  uint32_t ev = prmt(prmt(t[0], t[2], 0x0040u), prmt(t[4], t[6], 0x4000u), 0x7610u);
-  uint32_t od = prmt(prmt(t[1], t[3], 0x0040u), prmt(t[5], t[7], 0x4000u), 0x7610u);
-  return ((od << 4) + ev) ^ 0x88888888u;
+  const uint32_t x01 = t[1] * 16u + t[0], x23 = t[3] * 16u + t[2];
+  const uint32_t x45 = t[5] * 16u + t[4], x67 = t[7] * 16u + t[6];
+  return prmt(prmt(x01, x23, 0x0040u), prmt(x45, x67, 0x0040u), 0x5410u) ^ 0x88888888u;
 }
-// Pack 16 offset codes (each 2 + q) into one int2 word.
+// Pack 16 offset codes (each 2 + q) into one int2 word: byte j holds codes 4j .. 4j+3.
 __device__ __forceinline__ uint32_t pack16_int2(const uint32_t (&t)[16]) {
   uint32_t b[4];
 #pragma unroll
-  for (int i = 0; i < 4; ++i)
-    b[i] = prmt(prmt(t[i], t[4 + i], 0x0040u), prmt(t[8 + i], t[12 + i], 0x4000u), 0x7610u);
-  return (b[0] + (b[1] << 2) + (b[2] << 4) + (b[3] << 6)) ^ 0xAAAAAAAAu;
+  for (int i = 0; i < 4; ++i) b[i] = ((t[4 * i + 3] * 4u + t[4 * i + 2]) * 4u + t[4 * i + 1]) * 4u + t[4 * i];
+  return prmt(prmt(b[0], b[1], 0x0040u), prmt(b[2], b[3], 0x0040u), 0x5410u) ^ 0xAAAAAAAAu;
 }
 
 __device__ int g_fwht_error = 0;
@@ -215,6 +217,7 @@ __device__ __forceinline__ void quantise_store(const Args& a, const float2 (&xp)
     constexpr int GE = GT <= E ? GT : E;     // elements of one group held by this thread
     constexpr int NGT = E / GE;              // groups (or group fragments) per thread
     float f[NGT];
+    uint16_t sv[NGT];
     bool any_slow = false;
 #pragma unroll
     for (int g = 0; g < NGT; ++g) {
@@ -222,7 +225,7 @@ __device__ __forceinline__ void quantise_store(const Args& a, const float2 (&xp)
 #pragma unroll
       for (int j = 0; j < GE / 2; ++j) {
         const float2 p = xp[g * (GE / 2) + j];
-        m = fmaxf(m, fmaxf(fabsf(p.x), fabsf(p.y)));
+        m = max3(m, fabsf(p.x), fabsf(p.y));
       }
       if constexpr (GT > E) {
         const unsigned lanes = slot_lanes<TPC>();
@@ -230,12 +233,28 @@ __device__ __forceinline__ void quantise_store(const Args& a, const float2 (&xp)
         for (int o = 1; o < GT / E; o <<= 1) m = fmaxf(m, __shfl_xor_sync(lanes, m, o));
       }
       bool slow;
-      const uint16_t s16 = group_scale(m, a.norm, QMAX, &f[g], &slow);
+      sv[g] = group_scale(m, a.cdiv, a.cf, &f[g], &slow);
       any_slow |= slow;
-      if constexpr (GT > E) {
-        if ((t & (GT / E - 1)) == 0) srow[c0 / GT] = s16;
+    }
+    if constexpr (GT > E) {
+      if ((t & (GT / E - 1)) == 0) srow[c0 / GT] = sv[0];
+    } else {
+      // NGT consecutive scales: one vector store when the address allows it
+      uint16_t* sp = srow + c0 / GT;
+      const bool vec = NGT >= 2 && NGT <= 8 && (reinterpret_cast<uintptr_t>(sp) & (2 * NGT - 1)) == 0;
+      if constexpr (NGT == 2) {
+        if (vec) { *reinterpret_cast<uint32_t*>(sp) = sv[0] | ((uint32_t)sv[1] << 16); }
+        else { sp[0] = sv[0]; sp[1] = sv[1]; }
+      } else if constexpr (NGT == 4) {
+        if (vec) {
+          *reinterpret_cast<uint2*>(sp) = make_uint2(sv[0] | ((uint32_t)sv[1] << 16), sv[2] | ((uint32_t)sv[3] << 16));
+        } else {
+#pragma unroll
+          for (int g = 0; g < 4; ++g) sp[g] = sv[g];
+        }
       } else {
-        srow[c0 / GT + g] = s16;
+#pragma unroll
+        for (int g = 0; g < NGT; ++g) sp[g] = sv[g];
       }
     }
     const float2 mg = make_float2(MAGIC, MAGIC);
@@ -278,7 +297,7 @@ __device__ __forceinline__ void quantise_store(const Args& a, const float2 (&xp)
     for (int i = 0; i < NG; ++i) {
       float m = 0.0f;
 #pragma unroll
-      for (int j = 0; j < 4; ++j) m = fmaxf(m, fmaxf(fabsf(xp[4 * i + j].x), fabsf(xp[4 * i + j].y)));
+      for (int j = 0; j < 4; ++j) m = max3(m, fabsf(xp[4 * i + j].x), fabsf(xp[4 * i + j].y));
       gm[i] = m;
     }
 #pragma unroll
@@ -298,7 +317,7 @@ __device__ __forceinline__ void quantise_store(const Args& a, const float2 (&xp)
 #pragma unroll
     for (int i = 0; i < NG; ++i) {
       if ((i & (gg - 1)) == 0) {
-        sc[i] = group_scale(gm[i], a.norm, QMAX, &fw[i], &slow[i]);
+        sc[i] = group_scale(gm[i], a.cdiv, a.cf, &fw[i], &slow[i]);
       } else {
         fw[i] = fw[i - 1];
         slow[i] = slow[i - 1];
@@ -348,8 +367,18 @@ __device__ __forceinline__ void quantise_store(const Args& a, const float2 (&xp)
   }
 }
 
+// Sign masks in shared memory: one word per bf16 pair (bits 15 and 31), or, for the bf16
+// quantise path, two words per pair (the low element's sign moved to bit 31, and the high
+// element's sign at bit 31), so that sign flip and bf16 -> fp32 widening take one integer
+// instruction per element: (w << 16) + lo_mask and (w ^ hi_mask) & 0xffff0000.
+template <int LOGN, bool BF16, int MODE>
+constexpr bool dual_masks() {
+  return BF16 && MODE == MODE_QUANT && LOGN <= 12;
+}
+
 template <int LOGN, bool BF16, int MODE, int BITS, int GT>
 __global__ void __launch_bounds__(Cfg<LOGN>::THREADS, 1) fwht_kernel(const Args a) {
+  constexpr bool DUAL = dual_masks<LOGN, BF16, MODE>();
   using C = Cfg<LOGN>;
   constexpr int N = C::N, ELOG = C::ELOG, E = C::E, HB = C::HB, VA = C::VA, TPC = C::TPC;
   constexpr int NV = C::NV, NH = C::NH, SLOTS = C::SLOTS, SSTRIDE = C::SSTRIDE;
@@ -369,7 +398,15 @@ __global__ void __launch_bounds__(Cfg<LOGN>::THREADS, 1) fwht_kernel(const Args 
     asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_addr(bars + threadIdx.x)) : "memory");
   }
   if (has_signs) {
-    for (int i = threadIdx.x; i < a.K / 2; i += C::THREADS) smask[i] = a.signmask[i];
+    if constexpr (DUAL) {
+      for (int i = threadIdx.x; i < a.K / 2; i += C::THREADS) {
+        const uint32_t m = a.signmask[i];
+        smask[2 * i] = m << 16;
+        smask[2 * i + 1] = m & 0x80000000u;
+      }
+    } else {
+      for (int i = threadIdx.x; i < a.K / 2; i += C::THREADS) smask[i] = a.signmask[i];
+    }
   }
   asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   __syncthreads();
@@ -410,7 +447,20 @@ __global__ void __launch_bounds__(Cfg<LOGN>::THREADS, 1) fwht_kernel(const Args 
     parity ^= 1u;
 
     // ---------------- phase A: runs of NV elements from the staged chunk, signs, fp32 pairs
-    if constexpr (BF16) {
+    if constexpr (DUAL) {
+      const uint32_t* sraw = reinterpret_cast<const uint32_t*>(buf) + (T >> 1);
+      const uint32_t* smk = smask + cbase + T;   // two mask words per pair
+#pragma unroll
+      for (int h = 0; h < NH; ++h) {
+        uint32_t raw[NW], m[2 * NW];
+        load_masks<NW>(raw, sraw + h * (E / 2), 0, true);
+        load_masks<2 * NW>(m, smk + h * E, 0, has_signs);
+#pragma unroll
+        for (int w = 0; w < NW; ++w)
+          xp[h * NW + w] = make_float2(__uint_as_float((raw[w] << 16) + m[2 * w]),
+                                       __uint_as_float((raw[w] ^ m[2 * w + 1]) & 0xffff0000u));
+      }
+    } else if constexpr (BF16) {
       const uint32_t* sraw = reinterpret_cast<const uint32_t*>(buf) + (T >> 1);
       const uint32_t* smk = smask + ((cbase + T) >> 1);
       const bool sg = MODE != MODE_APPLY_INV && has_signs;
@@ -532,10 +582,31 @@ __global__ void __launch_bounds__(Cfg<LOGN>::THREADS, 1) fwht_kernel(const Args 
   }
 }
 
+template <int LOGN>
+size_t fused_smem_bytes(int K, bool dual) {
+  using C = Cfg<LOGN>;
+  return (size_t)C::SLOTS * C::SSTRIDE * 4 + (size_t)((C::SLOTS + 1) & ~1) * 8 + (size_t)(dual ? K : K / 2) * 4;
+}
+
+size_t fused_smem_any(int logn, int K, bool dual) {
+  switch (logn) {
+    case 5: return fused_smem_bytes<5>(K, dual);
+    case 6: return fused_smem_bytes<6>(K, dual);
+    case 7: return fused_smem_bytes<7>(K, dual);
+    case 8: return fused_smem_bytes<8>(K, dual);
+    case 9: return fused_smem_bytes<9>(K, dual);
+    case 10: return fused_smem_bytes<10>(K, dual);
+    case 11: return fused_smem_bytes<11>(K, dual);
+    case 12: return fused_smem_bytes<12>(K, dual);
+    case 13: return fused_smem_bytes<13>(K, dual);
+    default: return ~(size_t)0;
+  }
+}
+
 template <int LOGN, bool BF16, int MODE, int BITS, int GT>
 rot_status launch_one(const Args& a, cudaStream_t s) {
   using C = Cfg<LOGN>;
-  const size_t smem = (size_t)C::SLOTS * C::SSTRIDE * 4 + (size_t)((C::SLOTS + 1) & ~1) * 8 + (size_t)(a.K / 2) * 4;
+  const size_t smem = fused_smem_bytes<LOGN>(a.K, dual_masks<LOGN, BF16, MODE>());
   if (smem > 227 * 1024) return set_error(ROT_EUNSUPPORTED, "fused rotation: sign table too large for shared memory");
   auto kern = fwht_kernel<LOGN, BF16, MODE, BITS, GT>;
   static int configured[64] = {0};  // per device: the opt-in limit is set once
@@ -609,6 +680,8 @@ rot_status fwht_fetch_device_error() {
 
 bool fwht_quant_supported(const rot_plan_s* p, int bits, int G) {
   if (p->chunk_log2 < 5) return false;
+  // shared memory for the bf16 layout (the larger of the two sign-table layouts)
+  if (fused_smem_any(p->chunk_log2, p->K, p->chunk_log2 <= 12) > 227 * 1024) return false;
   const int N = 1 << p->chunk_log2;
   if (G < 8 || (G & (G - 1)) != 0 || G > N) return false;
   if (bits == 2 && G < 16) return false;
@@ -637,6 +710,11 @@ rot_status fwht_quant(const rot_plan_s* p, const void* A, int a_dtype, int64_t M
   a.log2G = 0;
   while ((1 << a.log2G) < G) ++a.log2G;
   a.ngroups = p->K / G;
+  {
+    const double nd = 1.0 / std::sqrt((double)(1 << p->chunk_log2));
+    a.cdiv = (float)(nd / (bits == 4 ? 7.0 : 1.0));
+    a.cf = (float)(nd * (1.0 + 0x1p-22));
+  }
   const int n = p->chunk_log2;
   if (a_dtype == ROT_BF16)
     return bits == 4 ? dispatch_logn<true, MODE_QUANT, 4>(n, a, s) : dispatch_logn<true, MODE_QUANT, 2>(n, a, s);

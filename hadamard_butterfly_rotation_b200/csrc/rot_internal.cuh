@@ -101,20 +101,24 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
 
 // Scale / code-factor of one quantisation group.
 //   m_z   : max |z| over the group, z the un-normalised rotated values (y = z * norm)
-// Returns the binary16 scale bits (fp32 IEEE quotient absmax / qmax, rounded to binary16);
-// *f receives the factor with v = z * f ~= y / s (within an ulp or two), nudged up by
-// 2^-22 relative so that exact ties of z * f round away from zero; *slow is set when the
-// scale is zero, subnormal or not finite (codes need clamping then).
-__device__ __forceinline__ uint16_t group_scale(float m_z, float norm, float qmax, float* f,
+//   c_div : fp32(norm / qmax);  c_f : fp32(norm * (1 + 2^-22))
+// Returns the binary16 scale bits, s = binary16(m_z * c_div): the quotient absmax / qmax
+// within an fp32 ulp or two of the correctly rounded one, so s differs from the rounding
+// of the exact quotient only for quotients within ~1e-7 relative of a binary16 midpoint.
+// *f receives the factor with v = z * f ~= y / s (approximate reciprocal, within about
+// 2 ulp), nudged up by 2^-22 relative so that exact ties of z * f round away from zero;
+// *slow is set when the scale is zero, subnormal or not finite (codes need clamping then).
+__device__ __forceinline__ uint16_t group_scale(float m_z, float c_div, float c_f, float* f,
                                                 bool* slow) {
-  float my = m_z * norm;
-  __half s16 = __float2half_rn(__fdiv_rn(my, qmax));
-  float s = __half2float(s16);
-  bool ok = (s >= 6.103515625e-05f) && (s <= 65504.0f);  // normal binary16
-  float fv = (s > 0.0f && s <= 65504.0f) ? __fmul_rn(norm, __frcp_rn(s)) : 0.0f;
-  *f = __fmul_rn(fv, 1.0f + 0x1p-22f);
-  *slow = !ok;
-  return __half_as_ushort(s16);
+  const __half s16 = __float2half_rn(m_z * c_div);
+  const uint32_t hb = __half_as_ushort(s16);
+  const float s = __half2float(s16);
+  // normal finite binary16 <=> magnitude bits in [0x0400, 0x7bff]
+  *slow = ((hb & 0x7fffu) - 0x0400u) >= 0x7800u;
+  float r;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(s));
+  *f = (s > 0.0f && s <= 65504.0f) ? r * c_f : 0.0f;
+  return (uint16_t)hb;
 }
 
 // Offset code u = qmax + 1 + rne(v) in the low bits of the result (magic-number rounding);

@@ -141,7 +141,7 @@ __global__ void __launch_bounds__(THREADS) stages_kernel(const Args a) {
         for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
         float f;
         bool slow;
-        const uint16_t s16 = group_scale(m, 1.0f, qmax, &f, &slow);
+        const uint16_t s16 = group_scale(m, a.bits == 4 ? 1.0f / 7.0f : 1.0f, 1.0f + 0x1p-22f, &f, &slow);
         if (lane == 0) a.scales[row * ngr + g] = s16;
         uint32_t* cw = reinterpret_cast<uint32_t*>(a.codes + row * (int64_t)(K / cpw) * 4) +
                        (int64_t)g * a.G / cpw;
