@@ -22,6 +22,7 @@
 //            and scales with vector stores.
 // Scaling by 1/sqrt(N) is folded into the output (apply) or into the group factor (quant).
 #include <cmath>
+#include <cstdlib>
 
 #include "rot_internal.cuh"
 
@@ -31,18 +32,28 @@ namespace {
 #ifndef ROT_FWHT_THREADS_E128
 #define ROT_FWHT_THREADS_E128 384   // threads per CTA for the 128-register-value layouts
 #endif
+#ifndef ROT_FWHT_THREADS_N11
+#define ROT_FWHT_THREADS_N11 640    // one warp per 2048-coordinate chunk, 20 chunks per CTA
+#endif
+
+// log2 of the values each thread holds for a chunk of 2^n coordinates
+constexpr int elog_of(int n) { return n <= 7 ? n : (n == 8 ? 5 : (n == 9 || n == 11) ? 6 : 7); }
+// threads per CTA
+constexpr int threads_of(int n) {
+  return n <= 7 ? 256 : (n == 8 ? 768 : (n == 9 ? 512 : (n == 11 ? ROT_FWHT_THREADS_N11 : ROT_FWHT_THREADS_E128)));
+}
 
 template <int LOGN>
 struct Cfg {
   static constexpr int N = 1 << LOGN;
-  static constexpr int ELOG = LOGN <= 7 ? LOGN : (LOGN == 8 ? 5 : (LOGN == 9 ? 6 : 7));
+  static constexpr int ELOG = elog_of(LOGN);
   static constexpr int E = 1 << ELOG;
   static constexpr int HB = LOGN - ELOG;   // thread bits (= high register bits of phase A)
   static constexpr int VA = ELOG - HB;     // contiguous run bits of phase A
   static constexpr int TPC = 1 << HB;      // threads per chunk
   static constexpr int NV = 1 << VA;       // run length
   static constexpr int NH = 1 << HB;       // runs per thread
-  static constexpr int THREADS = LOGN <= 7 ? 256 : (LOGN == 8 ? 768 : (LOGN == 9 ? 512 : ROT_FWHT_THREADS_E128));
+  static constexpr int THREADS = threads_of(LOGN);
   static constexpr int SLOTS = THREADS / TPC;
   static constexpr int SSTRIDE = N + 4;    // floats per slot buffer (16-byte pad)
   static_assert(VA >= 1, "phase A needs element pairs");
@@ -394,36 +405,6 @@ __global__ void __launch_bounds__(Cfg<LOGN>::THREADS, 1) fwht_kernel(const Args 
   float* buf = sbuf + slot * SSTRIDE;
   uint64_t* bar = bars + slot;
   const bool has_signs = a.signmask != nullptr;
-  if (threadIdx.x < SLOTS) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_addr(bars + threadIdx.x)) : "memory");
-  }
-  if (has_signs) {
-    if constexpr (DUAL) {
-      for (int i = threadIdx.x; i < a.K / 2; i += C::THREADS) {
-        const uint32_t m = a.signmask[i];
-        smask[2 * i] = m << 16;
-        smask[2 * i + 1] = m & 0x80000000u;
-      }
-    } else {
-      for (int i = threadIdx.x; i < a.K / 2; i += C::THREADS) smask[i] = a.signmask[i];
-    }
-  }
-  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-  __syncthreads();
-
-  // per-thread shared-memory bases (loop invariant); compile-time offsets are added per access
-  const int T = t << VA;                       // first coordinate of this thread's phase-A runs
-  constexpr int NPA = VA >= 5 ? 1 : (1 << (5 - (VA < 2 ? 2 : VA)));
-  constexpr bool B5 = (LOGN == 9 || LOGN == 11);  // extra swizzle term from coordinate bit 5
-  // phase-A store bases: pa[k] = T ^ (k << max(VA, 2)); with the bit-5 term (VA = 3, bit 5 =
-  // thread bit 2) the XOR on coordinate bit 2 also depends on the thread: fold it in.
-  const int tb = B5 ? ((T >> 5) & 1) << 2 : 0;
-  int pa[NPA];
-#pragma unroll
-  for (int k = 0; k < NPA; ++k) pa[k] = (T ^ (k << (VA < 2 ? 2 : VA))) ^ tb;
-  int qb[8];                                    // phase-B load bases
-#pragma unroll
-  for (int r = 0; r < 8; ++r) qb[r] = (t << ELOG) + ((4 * r) ^ ((t & 7) << 2));
 
   const int64_t units = a.M * a.chunks;
   const int64_t stride = (int64_t)gridDim.x * SLOTS;
@@ -437,7 +418,46 @@ __global__ void __launch_bounds__(Cfg<LOGN>::THREADS, 1) fwht_kernel(const Args 
   auto src_of = [&](int64_t r, int c) -> const void* {
     return static_cast<const uint8_t*>(a.A) + ((int64_t)r * a.lda + (int64_t)c * N) * ELEM;
   };
+
+  // Prologue that touches no memory written by earlier kernels: the slot barriers and the
+  // sign table (plan memory). Under programmatic dependent launch it overlaps the tail of
+  // the previous kernel in the stream; griddepcontrol.wait then orders every access to A
+  // and to the outputs after that kernel's completion (a no-op for an ordinary launch).
+  if (t == 0) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_addr(bar)) : "memory");
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (has_signs) {
+    if constexpr (DUAL) {
+      for (int i = threadIdx.x; i < a.K / 2; i += C::THREADS) {
+        const uint32_t m = a.signmask[i];
+        smask[2 * i] = m << 16;
+        smask[2 * i + 1] = m & 0x80000000u;
+      }
+    } else {
+      for (int i = threadIdx.x; i < a.K / 2; i += C::THREADS) smask[i] = a.signmask[i];
+    }
+  }
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  // the slot leader initialised its own barrier: it can start the first copy at once
   if (t == 0 && u < units) stage_issue(bar, buf, src_of(row, chunk), chunk_bytes);
+  __syncthreads();
+
+  // per-thread shared-memory bases (loop invariant); compile-time offsets are added per access
+  const int T = t << VA;                       // first coordinate of this thread's phase-A runs
+  constexpr int NPA = VA >= 5 ? 1 : (1 << (5 - (VA < 2 ? 2 : VA)));
+  constexpr bool B5 = (LOGN == 9 || LOGN == 11);  // extra swizzle term from coordinate bit 5
+  // phase-A store bases: pa[k] = T ^ (k << max(VA, 2)); with the bit-5 term (bit 5 of the
+  // coordinate is a thread bit) the XOR on coordinate bit 2 also depends on the thread.
+  const int tb = B5 ? ((T >> 5) & 1) << 2 : 0;
+  int pa[NPA];
+#pragma unroll
+  for (int k = 0; k < NPA; ++k) pa[k] = (T ^ (k << (VA < 2 ? 2 : VA))) ^ tb;
+  int qb[8];                                    // phase-B load bases
+#pragma unroll
+  for (int r = 0; r < 8; ++r) qb[r] = (t << ELOG) + ((4 * r) ^ ((t & 7) << 2));
+
   uint32_t parity = 0;
 
   for (; u < units; u += stride) {
@@ -582,6 +602,16 @@ __global__ void __launch_bounds__(Cfg<LOGN>::THREADS, 1) fwht_kernel(const Args 
   }
 }
 
+// Programmatic dependent launch (the kernel's prologue may overlap the previous kernel in
+// the stream); ROT_B200_PDL=0 in the environment turns it off.
+bool pdl_enabled() {
+  static const bool on = [] {
+    const char* e = std::getenv("ROT_B200_PDL");
+    return !(e && e[0] == '0');
+  }();
+  return on;
+}
+
 template <int LOGN>
 size_t fused_smem_bytes(int K, bool dual) {
   using C = Cfg<LOGN>;
@@ -621,7 +651,17 @@ rot_status launch_one(const Args& a, cudaStream_t s) {
   const int64_t cap = (int64_t)sm_count();
   if (grid > cap) grid = cap;
   if (grid < 1) return ROT_OK;
-  kern<<<(unsigned)grid, C::THREADS, smem, s>>>(a);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3(C::THREADS);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl_enabled() ? 1 : 0;
+  ROT_CUDA_TRY(cudaLaunchKernelEx(&cfg, kern, a));
   ROT_CUDA_TRY(cudaGetLastError());
   return ROT_OK;
 }
@@ -685,7 +725,7 @@ bool fwht_quant_supported(const rot_plan_s* p, int bits, int G) {
   const int N = 1 << p->chunk_log2;
   if (G < 8 || (G & (G - 1)) != 0 || G > N) return false;
   if (bits == 2 && G < 16) return false;
-  int e = p->chunk_log2 <= 7 ? p->chunk_log2 : (p->chunk_log2 == 8 ? 5 : (p->chunk_log2 == 9 ? 6 : 7));
+  const int e = elog_of(p->chunk_log2);
   if (G > (1 << e) && G / (1 << e) > 32) return false;
   return true;
 }
