@@ -195,11 +195,6 @@ __device__ __forceinline__ void stage_issue(uint64_t* bar, void* dst, const void
                : "memory");
 }
 
-__device__ __forceinline__ float min3(float a, float b, float c) {
-  float d;
-  asm("min.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
-  return d;
-}
 
 // Radix-2 butterflies along pair-index bit b: (P, Q) <- (P + Q, P - Q) on fp32 pairs.
 template <int NP>
@@ -602,6 +597,166 @@ __global__ void __launch_bounds__(Cfg<LOGN>::THREADS, 1) fwht_kernel(const Args 
   }
 }
 
+// ---------------------------------------------------------------- tensor-core first stage
+// Chunks of 2048 coordinates, bf16 input, quantised output. H_2048 = H_2^(x)11 factors over
+// the 11 coordinate bits e0..e10 (e = sum e_b 2^b), so the butterfly stages can be taken in
+// any order. The stages over {e0, e1, e2, e6} form one H_16, applied on the tensor cores to
+// the signed bf16 input (products with +-1 are exact, sums in fp32); the other seven stages
+// run on fp32 pairs in registers.
+//   MMA     m16n8k16 (bf16 in, fp32 out), D = X H_16 with X the 16 x 16 block of the chunk
+//           whose rows are coordinate blocks (row bits e3, e4, e5, e7) and columns the
+//           H_16 coordinates (k bits e0, e1, e2, e6); eight row tiles (e8, e9, e10).
+//           The A fragments come straight from the staged bf16 row with ldmatrix; the signs
+//           are XORed into them from a table kept in fragment order.
+//   phase A lane 4g + c holds e1e2 = c and e3e4e5 = g; its registers hold e0 (inside each
+//           fp32 pair), e6 (which of the two MMAs), e7 and e8..e10: butterflies over e7..e10.
+//   phase B after a transpose through shared memory (XOR-swizzled 16-byte chunks, no bank
+//           conflicts either way) lane l holds the contiguous coordinates 64 l .. 64 l + 63:
+//           butterflies over e3..e5, then group quantisation and packing as in fwht_kernel.
+constexpr int MMA_THREADS = 640;               // 20 warps, one chunk each
+constexpr int MMA_SLOTS = MMA_THREADS / 32;
+constexpr int MMA_SSTRIDE = 2048 + 4;          // floats per slot buffer
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr)
+               : "memory");
+}
+
+__device__ __forceinline__ void mma_h16(float2& d01, float2& d23, const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%10,%10,%10,%10};"
+      : "=f"(d01.x), "=f"(d01.y), "=f"(d23.x), "=f"(d23.y)
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "f"(0.0f));
+}
+
+// bf16 +-1 of the Sylvester entry (-1)^popcount(k & o)
+__host__ __device__ constexpr uint32_t h16_bf16(int k, int o) {
+  int v = k & o, par = 0;
+  while (v) { par ^= 1; v &= v - 1; }
+  return par ? 0xBF80u : 0x3F80u;
+}
+
+template <int BITS, int GT>
+__global__ void __launch_bounds__(MMA_THREADS, 1) fwht_mma_kernel(const Args a) {
+  constexpr int N = 2048, E = 64, NP = 32;
+  extern __shared__ __align__(128) float smem[];
+  float* sbuf = smem;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + MMA_SLOTS * MMA_SSTRIDE);
+  uint32_t* smf = reinterpret_cast<uint32_t*>(bars + MMA_SLOTS);  // sign masks, fragment order
+
+  const int slot = threadIdx.x >> 5;
+  const int l = threadIdx.x & 31;
+  const int g = l >> 2, c = l & 3;
+  float* buf = sbuf + slot * MMA_SSTRIDE;
+  uint64_t* bar = bars + slot;
+  const bool has_signs = a.signmask != nullptr;
+
+  const int64_t units = a.M * a.chunks;
+  const int64_t stride = (int64_t)gridDim.x * MMA_SLOTS;
+  int64_t u = (int64_t)blockIdx.x * MMA_SLOTS + slot;
+  const int64_t drow = stride / a.chunks;
+  const int dchunk = (int)(stride - drow * a.chunks);
+  int64_t row = u / a.chunks;
+  int chunk = (int)(u - row * a.chunks);
+  auto src_of = [&](int64_t r, int ch) -> const void* {
+    return static_cast<const uint8_t*>(a.A) + ((int64_t)r * a.lda + (int64_t)ch * N) * 2;
+  };
+
+  // prologue on plan memory only (see fwht_kernel): barrier, sign table in fragment order
+  if (l == 0) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_addr(bar)) : "memory");
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (has_signs) {
+    // word (ch * 1024 + i * 128 + lane * 4 + r): register r of lane's A fragment, tile i
+    for (int idx = threadIdx.x; idx < a.K / 2; idx += MMA_THREADS) {
+      const int ch = idx >> 10, i = (idx >> 7) & 7, ln = (idx >> 2) & 31, r = idx & 3;
+      const int off = ch * N + 8 * (ln >> 2) + 2 * (ln & 3) + 256 * i + ((r & 1) << 7) + ((r & 2) << 5);
+      smf[idx] = a.signmask[off >> 1];
+    }
+  }
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  if (l == 0 && u < units) stage_issue(bar, buf, src_of(row, chunk), N * 2);
+  __syncthreads();
+
+  // B fragments of H_16 for the two MMAs (outputs o3 = 0 / 1): n = g, k = 2c + {0,1} (+8)
+  uint32_t hb[2][2];
+#pragma unroll
+  for (int q = 0; q < 2; ++q) {
+    const int o = 8 * q + g;
+    hb[q][0] = h16_bf16(2 * c, o) | (h16_bf16(2 * c + 1, o) << 16);
+    hb[q][1] = h16_bf16(2 * c + 8, o) | (h16_bf16(2 * c + 9, o) << 16);
+  }
+  // ldmatrix row address of this lane (bytes): matrix l >> 3, row l & 7
+  const uint32_t lrow = (uint32_t)(8 * (l & 7) + ((l >> 3) & 1) * 128 + ((l >> 4) & 1) * 64) * 2;
+  const uint32_t sbase = smem_addr(buf);
+  // phase-A store base (element 2c + 8g of each 64-coordinate block, swizzle added per p)
+  const int abase = 2 * c + 8 * g;
+  uint32_t parity = 0;
+
+  for (; u < units; u += stride) {
+    const int cbase = chunk * N;
+    float2 xp[NP];
+    if (!stage_wait(bar, parity)) break;
+    parity ^= 1u;
+
+    // ---------------- MMA: H_16 over {e0, e1, e2, e6} for the 8 row tiles
+    const uint4* sm4 = reinterpret_cast<const uint4*>(smf + (cbase >> 1)) + l;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      uint32_t af[4];
+      ldsm_x4(sbase + lrow + i * 512, af);
+      if (has_signs) {
+        const uint4 m = sm4[i * 32];
+        af[0] ^= m.x; af[1] ^= m.y; af[2] ^= m.z; af[3] ^= m.w;
+      }
+      // xp index p = e6 + 2 e7 + 4 (e8..e10): MMA q gives e6 = q; rows g / g + 8 give e7
+      mma_h16(xp[4 * i + 0], xp[4 * i + 2], af, hb[0][0], hb[0][1]);
+      mma_h16(xp[4 * i + 1], xp[4 * i + 3], af, hb[1][0], hb[1][1]);
+    }
+    // ---------------- phase A: e7 .. e10 (pair-index bits 1 .. 4)
+#pragma unroll
+    for (int b = 1; b < 5; ++b) stage_pairs<NP>(xp, b);
+
+    // ---------------- transpose: element e = abase + 64 p (+ e0), physical e ^ ((p & 7) << 2)
+    __syncwarp();   // every lane's ldmatrix reads of the staged row are done
+#pragma unroll
+    for (int p = 0; p < NP; ++p)
+      *reinterpret_cast<float2*>(buf + ((abase ^ ((p & 7) << 2)) + 64 * p)) = xp[p];
+    __syncwarp();
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      const float4 q = *reinterpret_cast<const float4*>(buf + 64 * l + ((4 * j) ^ ((l & 7) << 2)));
+      xp[2 * j] = make_float2(q.x, q.y);
+      xp[2 * j + 1] = make_float2(q.z, q.w);
+    }
+    // the slot buffer is free: stage the next chunk while this one finishes
+    int64_t nrow = row + drow;
+    int nchunk = chunk + dchunk;
+    if (nchunk >= a.chunks) { nchunk -= a.chunks; ++nrow; }
+    if (u + stride < units) {
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      __syncwarp();
+      if (l == 0) stage_issue(bar, buf, src_of(nrow, nchunk), N * 2);
+    }
+    // ---------------- phase B: e3 .. e5 (pair-index bits 2 .. 4)
+#pragma unroll
+    for (int b = 2; b < 5; ++b) stage_pairs<NP>(xp, b);
+    const int64_t cur_row = row;
+    row = nrow;
+    chunk = nchunk;
+    quantise_store<11, BITS, GT, E, 32>(a, xp, cur_row, cbase + 64 * l, l);
+  }
+}
+
+size_t mma_smem_bytes(int K) {
+  return (size_t)MMA_SLOTS * MMA_SSTRIDE * 4 + (size_t)MMA_SLOTS * 8 + (size_t)(K / 2) * 4;
+}
+
 // Programmatic dependent launch (the kernel's prologue may overlap the previous kernel in
 // the stream); ROT_B200_PDL=0 in the environment turns it off.
 bool pdl_enabled() {
@@ -666,8 +821,56 @@ rot_status launch_one(const Args& a, cudaStream_t s) {
   return ROT_OK;
 }
 
+// Tensor-core first stage for 2048-coordinate chunks (ROT_B200_TC=0 in the environment
+// selects the all-CUDA-core kernel instead).
+bool tc_enabled() {
+  static const bool on = [] {
+    const char* e = std::getenv("ROT_B200_TC");
+    return !(e && e[0] == '0');
+  }();
+  return on;
+}
+
+template <int BITS, int GT>
+rot_status launch_mma(const Args& a, cudaStream_t s) {
+  const size_t smem = mma_smem_bytes(a.K);
+  if (smem > 227 * 1024) return set_error(ROT_EUNSUPPORTED, "fused rotation: sign table too large for shared memory");
+  auto kern = fwht_mma_kernel<BITS, GT>;
+  static int configured[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !configured[dev]) {
+    ROT_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024));
+    configured[dev] = 1;
+  }
+  const int64_t units = a.M * a.chunks;
+  int64_t grid = (units + MMA_SLOTS - 1) / MMA_SLOTS;
+  const int64_t cap = (int64_t)sm_count();
+  if (grid > cap) grid = cap;
+  if (grid < 1) return ROT_OK;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3(MMA_THREADS);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl_enabled() ? 1 : 0;
+  ROT_CUDA_TRY(cudaLaunchKernelEx(&cfg, kern, a));
+  return ROT_OK;
+}
+
 template <int LOGN, bool BF16, int MODE, int BITS>
 rot_status launch_g(const Args& a, cudaStream_t s) {
+  if constexpr (MODE == MODE_QUANT && BF16 && LOGN == 11) {
+    if (tc_enabled() && mma_smem_bytes(a.K) <= 227 * 1024) {
+      if (a.G == 32) return launch_mma<BITS, 32>(a, s);
+      if (a.G == 64) return launch_mma<BITS, 64>(a, s);
+      if (a.G == 128) return launch_mma<BITS, 128>(a, s);
+    }
+  }
   // compile-time group sizes for the common shapes (bf16 quantisation on large chunks)
   if constexpr (MODE == MODE_QUANT && BF16 && (LOGN == 8 || LOGN >= 11)) {
     if (a.G == 32) return launch_one<LOGN, BF16, MODE, BITS, 32>(a, s);
