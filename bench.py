@@ -240,10 +240,10 @@ def main():
 
     def step(i):
         c, s = outs[i % NSETS]
-        hbr.rot_quant(A_sets[i % NSETS], plan, bits, G, codes=c, scales=s, stream=stream)
+        hbr.rot_quant(A_sets[i % NSETS], plan, bits, G, codes=c, scales=s)
 
-    for i in range(args.warmup):
-        step(i)
+    # one period of the buffer rotation in a CUDA graph (warm-up steps run before capture)
+    steps_graph = StepGraph(step, NSETS, warm=args.warmup)
     torch.cuda.synchronize(dev)
     if world > 1:
         dist.barrier()
@@ -251,8 +251,7 @@ def main():
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(dev.index) as clk:
         ev0.record(stream)
-        for i in range(args.steps):
-            step(i)
+        steps_graph.run(args.steps)
         ev1.record(stream)
         torch.cuda.synchronize(dev)
     if world > 1:
@@ -320,6 +319,7 @@ def main():
         "config": {"workload": "llama32_1b: A[8192,2048] bf16, RHT K=2048 (signs + FWHT + 1/sqrt(K)), "
                                "int4 G=32, packed codes + fp16 scales",
                    "global_batch": M * world, "l2": "6 rotating input/output sets (258 MB > 126 MB L2)",
+                   "launch": "timed steps replayed from a CUDA graph holding one 6-step period",
                    "parallelism": f"dp{world} (independent rows)"},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
                      "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": profiled_traffic("rot_quant_llama32_1b"),
@@ -337,6 +337,7 @@ def main():
 
 
 def _time_loop(fn, n, stream, warm=5):
+    """Seconds per call of fn(i) over n direct launches (host launch cost included)."""
     import torch
     for i in range(warm):
         fn(i)
@@ -348,6 +349,46 @@ def _time_loop(fn, n, stream, warm=5):
     e1.record(stream)
     torch.cuda.synchronize()
     return e0.elapsed_time(e1) / n / 1e3  # seconds per call
+
+
+class StepGraph:
+    """Steps 0 .. period-1 of fn(i) (launching on the current stream) captured in one CUDA
+    graph, so that back-to-back steps are timed on the device without per-launch host cost.
+    run(n) issues exactly n steps: n // period graph replays, then the remaining steps
+    launched directly."""
+
+    def __init__(self, fn, period, warm=3):
+        import torch
+        self.fn, self.period = fn, period
+        for i in range(warm):
+            fn(i)
+        torch.cuda.synchronize()
+        self.g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.g):
+            for i in range(period):
+                fn(i)
+        self.g.replay()
+        torch.cuda.synchronize()
+
+    def run(self, n):
+        reps, rem = divmod(n, self.period)
+        for _ in range(reps):
+            self.g.replay()
+        for i in range(rem):
+            self.fn(i)
+
+
+def _graph_time(fn, n, period, warm=3):
+    """Seconds per step of fn(i), n steps replayed from a CUDA graph of `period` steps."""
+    import torch
+    sg = StepGraph(fn, period, warm)
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    sg.run(n)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / n / 1e3
 
 
 def run_extra(hbr, W, dev, stream, peaks):
@@ -370,8 +411,8 @@ def run_extra(hbr, W, dev, stream, peaks):
 
             def f(i):
                 c, s = outs[i % nsets]
-                hbr.rot_quant(As[i % nsets], plan, bits, G, codes=c, scales=s, stream=stream)
-            t = _time_loop(f, n, stream)
+                hbr.rot_quant(As[i % nsets], plan, bits, G, codes=c, scales=s)
+            t = _graph_time(f, n, nsets)
             b = algorithmic_bytes(wl.M, wl.K, bits, G)
             key = f"{name}{'_' + variant if variant else ''}_int{bits}_G{G}"
             out[key] = {"us": round(t * 1e6, 2), "GB/s": round(b / t / 1e9, 1), "frac_hbm": round(b / t / 1e9 / hbm, 4)}
@@ -387,7 +428,7 @@ def run_extra(hbr, W, dev, stream, peaks):
         N = Wq.shape[0]
         C = torch.empty((wl.M, N), dtype=torch.bfloat16, device=dev)
         n = 50 if wl.M > 16 else 200
-        t = _time_loop(lambda i: hbr.w4a4_linear(Aq, As_, Wq, Ws, G, out=C, stream=stream), n, stream)
+        t = _graph_time(lambda i: hbr.w4a4_linear(Aq, As_, Wq, Ws, G, out=C), n, 10)
         ops = 2.0 * wl.M * N * wl.K
         wbytes = Wq.numel() + Ws.numel() * 2 + Aq.numel() + As_.numel() * 2 + C.numel() * 2
         out[f"w4a4_{name}"] = {"us": round(t * 1e6, 2), "TOPS": round(ops / t / 1e12, 1),
@@ -413,7 +454,7 @@ def run_profile(args):
         Aq, As = hbr.rot_quant(torch.from_numpy(wl.A).to(torch.bfloat16).to(dev), plan, bits, G)
         Wq, Ws = hbr.rot_quant(torch.from_numpy(np.ascontiguousarray(wl.W.T)).to(dev), plan, bits, G)
         C = torch.empty((wl.M, Wq.shape[0]), dtype=torch.bfloat16, device=dev)
-        fn = lambda i: hbr.w4a4_linear(Aq, As, Wq, Ws, G, out=C, stream=stream)
+        fn = lambda i: hbr.w4a4_linear(Aq, As, Wq, Ws, G, out=C)
         work = 2.0 * wl.M * Wq.shape[0] * wl.K
         unit = "TOPS"
     else:
@@ -429,10 +470,10 @@ def run_profile(args):
         A = torch.from_numpy(wl.A).to(torch.bfloat16).to(dev)
         codes = torch.empty((wl.M, wl.K * bits // 8), dtype=torch.uint8, device=dev)
         scales = torch.empty((wl.M, wl.K // G), dtype=torch.float16, device=dev)
-        fn = lambda i: hbr.rot_quant(A, plan, bits, G, codes=codes, scales=scales, stream=stream)
+        fn = lambda i: hbr.rot_quant(A, plan, bits, G, codes=codes, scales=scales)
         work = algorithmic_bytes(wl.M, wl.K, bits, G)
         unit = "GB/s"
-    t = _time_loop(fn, args.steps, stream, warm=args.warmup)
+    t = _graph_time(fn, args.steps, 10, warm=args.warmup)
     print(json.dumps({"profile": name, "us_per_launch": round(t * 1e6, 3),
                       unit: round(work / t / 1e9 if unit == "GB/s" else work / t / 1e12, 2)}))
     return 0
