@@ -12,18 +12,25 @@
 // same K permutation is applied to both operands, so every group sum is unchanged.
 //
 // Tile: 128 rows of A x 256 rows of W per CTA; K in blocks of 128 (one 128-byte swizzle
-// atom of int8 per row), 4 UMMAs of K = 32 per block, 3-stage smem ring. (A 128 x 128 tile
-// avoids the epilogue's register spills but re-reads A twice as often and measured slower.)
+// atom of int8 per row), 4 UMMAs of K = 32 per block, 3-stage ring of unpacked int8 tiles fed
+// by a 2-stage ring of packed tiles. (A 128 x 128 tile re-reads A twice as often and
+// measured slower.)
 // Warp roles (512 threads, launched with 128 registers each). setmaxnreg acts on whole
-// warpgroups, so roles are aligned to them: warpgroups 0-1 (epilogue) grow to 168 registers,
-// warpgroups 2-3 (producers + MMA warp) shrink to 88: 256*168 + 256*88 = 512*128.
+// warpgroups, so roles are aligned to them: warpgroups 0-1 (epilogue) grow to 216 registers,
+// warpgroups 2-3 (loader, unpackers, MMA warp) shrink to 40: 256*216 + 256*40 = 512*128.
 //   warps 0-7   epilogue: two warpgroups, 128 columns each; after each group they read
-//               the int32 partials from TMEM, apply the group scales and accumulate in
-//               fp32 registers (packed f32x2 FMAs);
-//   warps 8-14  producers: load packed codes from global memory (register prefetch two
-//               K-blocks ahead), unpack, store into the swizzled K-major smem layout, then
-//               fence.proxy.async + mbarrier arrive;
+//               the int32 partials from TMEM (32 columns per load), apply the group scales
+//               and accumulate in fp32 registers (packed f32x2 FMAs);
+//   warp 8      loader: one bulk copy (cp.async.bulk) per tile row and K-block brings the
+//               packed codes into the packed ring, completing on an mbarrier;
+//   warps 9-14  unpackers: read a packed stage from shared memory, unpack, store into the
+//               swizzled K-major int8 layout, fence.proxy.async, then release both stages;
 //   warp 15     TMEM allocation and MMA issue (one elected lane).
+// Measured on B200 at M=2048, N=K=4096 (timestamps and role-by-role variants): the MMA warp
+// alone reaches 1529 TOPS; the epilogue's per-group TMEM traffic (read 256 partial columns,
+// rewrite the bias) slows the MMAs on the other accumulator several-fold while it runs, so
+// at G = 128 the epilogue's TMEM time, not the unpacking, bounds the kernel (G = 256 halves
+// it). Per-row bulk copies of the packed codes were 5x slower than the two 2-D TMA boxes.
 // TMEM holds two group accumulators (2 x 256 columns). Before a group's MMAs accumulate
 // into a buffer, the epilogue fills it with the bit pattern of 1.5 * 2^23; adding the
 // integer partial sum 256*P keeps the exponent, so the accumulator bits read back as the
@@ -32,6 +39,9 @@
 //
 // Every mbarrier wait is bounded (about 2 s of wall time); a wait that gives up records
 // ROT_ETIMEOUT in a device flag, and the CTA skips its remaining work and exits.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include <cstdint>
 
 #include "rot_internal.cuh"
@@ -42,22 +52,27 @@ namespace {
 constexpr int BM = 128;
 constexpr int BN = 256;
 constexpr int KB = 128;                  // K elements per stage
-constexpr int STAGES = 3;
+constexpr int STAGES = 3;                // unpacked int8 stages
+constexpr int PSTAGES = 2;               // packed stages
 constexpr int A_STAGE_BYTES = BM * KB;   // unpacked int8
 constexpr int B_STAGE_BYTES = BN * KB;
 constexpr int STAGE_BYTES = A_STAGE_BYTES + B_STAGE_BYTES;
+constexpr int PROW_BYTES = KB / 2;       // packed bytes of one row in one K-block
+constexpr int PSTAGE_BYTES = (BM + BN) * PROW_BYTES;
 constexpr int N_EPI = 256;               // epilogue threads (2 warpgroups)
-constexpr int N_PROD = 224;              // producer threads
-constexpr int THREADS = N_EPI + N_PROD + 32;
+constexpr int LOADER_WARP = N_EPI / 32;  // warp 8
+constexpr int N_UNP = 192;               // unpacker threads (warps 9-14)
+constexpr int N_UNP_WARPS = N_UNP / 32;
+constexpr int THREADS = N_EPI + 32 + N_UNP + 32;
 constexpr int N_CHUNKS = (BM + BN) * (KB / 32);                  // 16-byte packed chunks / stage
-constexpr int PROD_CHUNKS = (N_CHUNKS + N_PROD - 1) / N_PROD;     // per producer thread
+constexpr int UNP_CHUNKS = N_CHUNKS / N_UNP;                     // per unpacker thread
 constexpr int EPI_COLS = BN / 2;         // columns per epilogue warpgroup
-constexpr int MMA_WARP = (N_EPI + N_PROD) / 32;
+constexpr int MMA_WARP = (N_EPI + 32 + N_UNP) / 32;
 constexpr int LAUNCH_REGS = 128;         // 65536 / THREADS
-constexpr int EPI_REGS = 168, PROD_REGS = 88;  // per warpgroup role
+constexpr int EPI_REGS = 216, PROD_REGS = 40;  // per warpgroup role
 static_assert(THREADS == 512, "register split assumes 512 threads");
-static_assert(N_EPI == 256 && N_PROD + 32 == 256, "roles must fill whole warpgroups");
-static_assert(N_EPI * EPI_REGS + (N_PROD + 32) * PROD_REGS <= THREADS * LAUNCH_REGS, "register split");
+static_assert(N_CHUNKS % N_UNP == 0, "unpack work divides evenly");
+static_assert(N_EPI * EPI_REGS + (THREADS - N_EPI) * PROD_REGS <= THREADS * LAUNCH_REGS, "register split");
 constexpr uint32_t TMEM_COLS = 2 * BN;   // two group accumulators (all 512 columns)
 constexpr uint32_t BIAS_BITS = 0x4B400000u;  // 1.5 * 2^23
 constexpr float BIAS_F = 12582912.0f;
@@ -65,14 +80,18 @@ constexpr unsigned long long WAIT_NS = 2000000000ull;
 
 // smem layout (offsets from a 1024-byte aligned base)
 constexpr int OFF_STAGES = 0;
-constexpr int OFF_SCALES = STAGES * STAGE_BYTES;          // [2][2][BN] fp32: sW/256 and -1.5*2^23*sW/256
+constexpr int OFF_PSTAGES = STAGES * STAGE_BYTES;
+constexpr int OFF_SCALES = OFF_PSTAGES + PSTAGES * PSTAGE_BYTES;  // [2][2][BN] fp32: sW/256, -1.5*2^23*sW/256
 constexpr int OFF_BARS = OFF_SCALES + 2 * BN * 8;
 constexpr int OFF_TMEM = OFF_BARS + 16 * 8;
 constexpr int SMEM_BYTES = OFF_TMEM + 16 + 1024;          // + alignment slack
+static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
 
 __device__ int g_w4a4_error = 0;
 
 struct Params {
+  CUtensorMap tmA;   // packed A codes [M, K/2] uint8, box {64 bytes, BM rows}
+  CUtensorMap tmW;   // packed W codes [N, K/2] uint8, box {64 bytes, BN rows}
   const uint8_t* Aq;
   const uint16_t* As;
   const uint8_t* Wq;
@@ -164,12 +183,6 @@ __device__ __forceinline__ void umma_commit(uint64_t* bar) {
                : "memory");
 }
 
-__device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t (&r)[8]) {
-  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
-               : "r"(taddr)
-               : "memory");
-}
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_st16_const(uint32_t taddr, uint32_t v) {
   asm volatile(
@@ -193,15 +206,54 @@ __device__ __forceinline__ void named_bar(int id, int n) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
 }
 
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr)
+      : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
+}
+
+// 2-D tiled TMA load (no multicast) of box (x, y) of `tmap` into shared memory; the box's
+// bytes (out-of-range elements zero-filled) complete on `bar`
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* tmap, int x, int y, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::
+          "r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// Warp-uniform bounded wait: lane 0 waits on the mbarrier, the result is broadcast and the
+// warp re-converges (its memory accesses are ordered after lane 0's acquire by __syncwarp).
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag, int lane) {
+  int w = 1;
+  if (lane == 0) w = mbar_wait(bar, parity, abort_flag) ? 1 : 0;
+  w = __shfl_sync(0xffffffffu, w, 0);
+  __syncwarp();
+  return w != 0;
+}
+
 template <bool PARTIALS>
-__global__ void __launch_bounds__(THREADS, 1) w4a4_kernel(const Params p) {
+__global__ void __launch_bounds__(THREADS, 1) w4a4_kernel(const __grid_constant__ Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BARS);
-  uint64_t* full = bars;                 // [STAGES] producers -> MMA
-  uint64_t* empty = bars + STAGES;       // [STAGES] MMA commit -> producers
-  uint64_t* tfull = bars + 2 * STAGES;   // [2] MMA commit -> epilogue
-  uint64_t* tempty = bars + 2 * STAGES + 2;  // [2] epilogue -> MMA
+  uint64_t* full = bars;                      // [STAGES]  unpackers -> MMA (one arrival per warp)
+  uint64_t* empty = bars + STAGES;            // [STAGES]  MMA commit -> unpackers
+  uint64_t* tfull = bars + 2 * STAGES;        // [2]       MMA commit -> epilogue
+  uint64_t* tempty = bars + 2 * STAGES + 2;   // [2]       epilogue -> MMA
+  uint64_t* pfull = bars + 2 * STAGES + 4;    // [PSTAGES] bulk copies -> unpackers
+  uint64_t* pempty = bars + 2 * STAGES + 4 + PSTAGES;  // [PSTAGES] unpackers -> loader
+  static_assert(2 * STAGES + 4 + 2 * PSTAGES <= 16, "barrier slots");
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_TMEM);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + OFF_TMEM + 8);
   float* sc = reinterpret_cast<float*>(smem + OFF_SCALES);  // [buf][0: sW/256, 1: c][BN]
@@ -216,12 +268,16 @@ __global__ void __launch_bounds__(THREADS, 1) w4a4_kernel(const Params p) {
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&full[s], N_PROD);
+      mbar_init(&full[s], N_UNP_WARPS);
       mbar_init(&empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull[b], 1);
       mbar_init(&tempty[b], N_EPI);
+    }
+    for (int s = 0; s < PSTAGES; ++s) {
+      mbar_init(&pfull[s], 1);
+      mbar_init(&pempty[s], N_UNP_WARPS);
     }
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -239,7 +295,7 @@ __global__ void __launch_bounds__(THREADS, 1) w4a4_kernel(const Params p) {
 
   if (warp < N_EPI / 32) {
     // ======================= epilogue
-    asm volatile("setmaxnreg.inc.sync.aligned.u32 168;");
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 216;");
     const int wg = warp >> 2;                 // column block of EPI_COLS
     const int row = (warp & 3) * 32 + lane;   // TMEM lane = tile row
     const int m = m0 + row;
@@ -283,35 +339,36 @@ __global__ void __launch_bounds__(THREADS, 1) w4a4_kernel(const Params p) {
       }
       named_bar(1, N_EPI);
       const int b = g & 1;
-      if (!ok || !mbar_wait(&tfull[b], (g >> 1) & 1, abort_flag)) { ok = false; continue; }
+      ok = ok && warp_wait(&tfull[b], (g >> 1) & 1, abort_flag, lane);   // warp-uniform
+      if (!ok) continue;
       tc_fence_after();
       const uint32_t base = lane_addr + b * BN + wg * EPI_COLS;
       const float* scw = sc + ((g & 1) * 2 + 0) * BN + wg * EPI_COLS;
       const float* scc = sc + ((g & 1) * 2 + 1) * BN + wg * EPI_COLS;
       const float2 sa2 = make_float2(sa, sa);
 #pragma unroll
-      for (int c = 0; c < EPI_COLS / 8; ++c) {
-        uint32_t rr[8];
-        tmem_ld8(base + c * 8, rr);
+      for (int c = 0; c < EPI_COLS / 32; ++c) {
+        uint32_t rr[32];
+        tmem_ld32(base + c * 32, rr);
         tmem_wait_ld();
         if constexpr (!PARTIALS) {
 #pragma unroll
-          for (int j = 0; j < 8; j += 4) {
-            const float4 w4 = lds128(scw + c * 8 + j);
-            const float4 c4 = lds128(scc + c * 8 + j);
+          for (int j = 0; j < 32; j += 4) {
+            const float4 w4 = lds128(scw + c * 32 + j);
+            const float4 c4 = lds128(scc + c * 32 + j);
             const float2 u0 = make_float2(__uint_as_float(rr[j]), __uint_as_float(rr[j + 1]));
             const float2 u1 = make_float2(__uint_as_float(rr[j + 2]), __uint_as_float(rr[j + 3]));
             // exact P*sW (the bias cancels inside one rounding), then acc += (P*sW)*sA
             const float2 t0 = __ffma2_rn(u0, make_float2(w4.x, w4.y), make_float2(c4.x, c4.y));
             const float2 t1 = __ffma2_rn(u1, make_float2(w4.z, w4.w), make_float2(c4.z, c4.w));
-            acc[(c * 8 + j) / 2] = __ffma2_rn(t0, sa2, acc[(c * 8 + j) / 2]);
-            acc[(c * 8 + j) / 2 + 1] = __ffma2_rn(t1, sa2, acc[(c * 8 + j) / 2 + 1]);
+            acc[(c * 32 + j) / 2] = __ffma2_rn(t0, sa2, acc[(c * 32 + j) / 2]);
+            acc[(c * 32 + j) / 2 + 1] = __ffma2_rn(t1, sa2, acc[(c * 32 + j) / 2 + 1]);
           }
         } else {
           if (row_ok) {
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              const int n = n0 + wg * EPI_COLS + c * 8 + j;
+            for (int j = 0; j < 32; ++j) {
+              const int n = n0 + wg * EPI_COLS + c * 32 + j;
               if (n < p.N) p.P[((int64_t)m * p.N + n) * NG + g] = ((int32_t)(rr[j] - BIAS_BITS)) / 256;
             }
           }
@@ -352,51 +409,40 @@ __global__ void __launch_bounds__(THREADS, 1) w4a4_kernel(const Params p) {
         }
       }
     }
-  } else if (warp < MMA_WARP) {
-    // ======================= producers
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 88;");
-    const int pt = threadIdx.x - N_EPI;    // 0..N_PROD-1
-    const int64_t ldp = p.K / 2;           // packed bytes per row
-    // chunk q = pt + N_PROD*i: rows 0..BM-1 of A then 0..BN-1 of W, 4 chunks (16 B = 32 codes)
-    // per row. The global row pointers are fixed for the CTA; nullptr marks rows beyond M / N.
-    const uint8_t* gsrc[PROD_CHUNKS];
-#pragma unroll
-    for (int i = 0; i < PROD_CHUNKS; ++i) {
-      const int q = pt + N_PROD * i;
-      const int r = q >> 2, c = q & 3;
-      const uint8_t* src = nullptr;
-      if (q < N_CHUNKS) {
-        if (r < BM) {
-          if (m0 + r < p.M) src = p.Aq + (int64_t)(m0 + r) * ldp + c * 16;
-        } else {
-          if (n0 + r - BM < p.N) src = p.Wq + (int64_t)(n0 + r - BM) * ldp + c * 16;
-        }
+  } else if (warp == LOADER_WARP) {
+    // ======================= loader: the packed A and W tiles of one K-block -> packed stage
+    // (two 2-D TMA boxes; rows beyond M / N and bytes beyond K/2 arrive as zeros)
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 40;");
+    for (int kb = 0; kb < NKB; ++kb) {
+      const int ps = kb % PSTAGES;
+      if (kb >= PSTAGES && !warp_wait(&pempty[ps], ((kb / PSTAGES) + 1) & 1, abort_flag, lane)) break;
+      if (lane == 0) {
+        uint8_t* pst = smem + OFF_PSTAGES + ps * PSTAGE_BYTES;
+        mbar_arrive_expect_tx(&pfull[ps], (uint32_t)PSTAGE_BYTES);
+        // x = kb * 64 bytes: a multiple of 16, as a tiled TMA requires of the inner coordinate
+        tma_load_2d(pst, &p.tmA, kb * PROW_BYTES, m0, &pfull[ps]);
+        tma_load_2d(pst + BM * PROW_BYTES, &p.tmW, kb * PROW_BYTES, n0, &pfull[ps]);
       }
-      gsrc[i] = src;
+      __syncwarp();
     }
-    auto load = [&](int kb, uint4 (&dst)[PROD_CHUNKS]) {
-      const int64_t koff = (int64_t)kb * (KB / 2);
-#pragma unroll
-      for (int i = 0; i < PROD_CHUNKS; ++i) {
-        const int c = (pt + N_PROD * i) & 3;
-        uint4 v = make_uint4(0u, 0u, 0u, 0u);
-        if (gsrc[i] != nullptr && koff + c * 16 < ldp) v = __ldg(reinterpret_cast<const uint4*>(gsrc[i] + koff));
-        dst[i] = v;
-      }
-    };
-    // unpack one stage from registers, publish it, then refill the registers with K-block kb+2
-    auto stage = [&](int kb, uint4 (&cur)[PROD_CHUNKS]) -> bool {
-      const int s = kb % STAGES;
-      if (kb >= STAGES && !mbar_wait(&empty[s], ((kb / STAGES) + 1) & 1, abort_flag)) return false;
+  } else if (warp < MMA_WARP) {
+    // ======================= unpackers: packed stage -> swizzled int8 stage
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 40;");
+    const int ut = threadIdx.x - (LOADER_WARP + 1) * 32;   // 0..N_UNP-1
+    for (int kb = 0; kb < NKB; ++kb) {
+      const int s = kb % STAGES, ps = kb % PSTAGES;
+      if (!warp_wait(&pfull[ps], (kb / PSTAGES) & 1, abort_flag, lane)) break;
+      if (kb >= STAGES && !warp_wait(&empty[s], ((kb / STAGES) + 1) & 1, abort_flag, lane)) break;
+      const uint8_t* pst = smem + OFF_PSTAGES + ps * PSTAGE_BYTES;
       uint8_t* st = smem + OFF_STAGES + s * STAGE_BYTES;
-#pragma unroll
-      for (int i = 0; i < PROD_CHUNKS; ++i) {
-        const int q = pt + N_PROD * i;
-        if (q >= N_CHUNKS) continue;
+#pragma unroll 4
+      for (int i = 0; i < UNP_CHUNKS; ++i) {
+        // chunk q: row r (A rows 0..BM-1, then W rows), 16-byte piece c of the row's 64 bytes
+        const int q = ut + N_UNP * i;
         const int r = q >> 2, c = q & 3;
+        const uint4 w = *reinterpret_cast<const uint4*>(pst + q * 16);
         uint8_t* tile = r < BM ? st : st + A_STAGE_BYTES;
         const int rr = r < BM ? r : r - BM;
-        const uint4 w = cur[i];
         const uint4 lo = make_uint4((w.x << 4) & 0xF0F0F0F0u, (w.y << 4) & 0xF0F0F0F0u, (w.z << 4) & 0xF0F0F0F0u,
                                     (w.w << 4) & 0xF0F0F0F0u);
         const uint4 hi = make_uint4(w.x & 0xF0F0F0F0u, w.y & 0xF0F0F0F0u, w.z & 0xF0F0F0F0u, w.w & 0xF0F0F0F0u);
@@ -405,20 +451,15 @@ __global__ void __launch_bounds__(THREADS, 1) w4a4_kernel(const Params p) {
         *reinterpret_cast<uint4*>(rowp + (((2 * c + 1) ^ (rr & 7)) << 4)) = hi;
       }
       fence_proxy_async();
-      mbar_arrive(&full[s]);
-      if (kb + 2 < NKB) load(kb + 2, cur);
-      return true;
-    };
-    uint4 b0[PROD_CHUNKS], b1[PROD_CHUNKS];
-    load(0, b0);
-    if (NKB > 1) load(1, b1);
-    for (int kb = 0; kb < NKB; kb += 2) {
-      if (!stage(kb, b0)) break;
-      if (kb + 1 < NKB && !stage(kb + 1, b1)) break;
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&full[s]);
+        mbar_arrive(&pempty[ps]);
+      }
     }
   } else {
     // ======================= MMA issue
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 88;");  // same value as the producers of its warpgroup
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 40;");  // same value as the rest of its warpgroup
     const bool leader = lane == 0;
     const uint32_t sbase = smem_u32(smem + OFF_STAGES);
     for (int ks = 0; ks < KS; ++ks) {
@@ -454,7 +495,7 @@ __global__ void __launch_bounds__(THREADS, 1) w4a4_kernel(const Params p) {
   __syncthreads();
   if (warp == MMA_WARP) {
     if (*abort_flag) {
-      // let any in-flight MMA drain before the columns are released
+      // let any in-flight MMA or bulk copy drain before the columns and smem are released
       unsigned long long t0, now;
       asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t0));
       do { asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(now)); } while (now - t0 < 1000000ull);
@@ -487,6 +528,37 @@ rot_status w4a4_launch(const uint8_t* Aq, const uint16_t* As, const uint8_t* Wq,
     configured[dev] = 1;
   }
   Params p{};
+  {
+    static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
+    if (!encode) {
+      void* fn = nullptr;
+      cudaDriverEntryPointQueryResult q;
+      ROT_CUDA_TRY(cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q));
+      if (q != cudaDriverEntryPointSuccess || !fn)
+        return set_error(ROT_ECUDA, "w4a4_linear: cuTensorMapEncodeTiled not available");
+      encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    }
+    const cuuint64_t ldp = (cuuint64_t)(K / 2);
+    const cuuint32_t estr[2] = {1, 1};
+    {
+      const cuuint64_t dims[2] = {ldp, (cuuint64_t)(M > 0 ? M : 1)};
+      const cuuint64_t strides[1] = {ldp};
+      const cuuint32_t box[2] = {(cuuint32_t)PROW_BYTES, (cuuint32_t)BM};
+      if (encode(&p.tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(Aq), dims, strides, box, estr,
+                 CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return set_error(ROT_EINVAL, "w4a4_linear: tensor map for Aq rejected");
+    }
+    {
+      const cuuint64_t dims[2] = {ldp, (cuuint64_t)N};
+      const cuuint64_t strides[1] = {ldp};
+      const cuuint32_t box[2] = {(cuuint32_t)PROW_BYTES, (cuuint32_t)BN};
+      if (encode(&p.tmW, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(Wq), dims, strides, box, estr,
+                 CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return set_error(ROT_EINVAL, "w4a4_linear: tensor map for Wq rejected");
+    }
+  }
   p.Aq = Aq;
   p.As = As;
   p.Wq = Wq;
