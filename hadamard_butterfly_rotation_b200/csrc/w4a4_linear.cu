@@ -31,11 +31,11 @@
 // rewrite the bias) slows the MMAs on the other accumulator several-fold while it runs, so
 // at G = 128 the epilogue's TMEM time, not the unpacking, bounds the kernel (G = 256 halves
 // it). Per-row bulk copies of the packed codes were 5x slower than the two 2-D TMA boxes.
-// TMEM holds two group accumulators (2 x 256 columns). Before a group's MMAs accumulate
-// into a buffer, the epilogue fills it with the bit pattern of 1.5 * 2^23; adding the
-// integer partial sum 256*P keeps the exponent, so the accumulator bits read back as the
-// fp32 value 1.5 * 2^23 + 256*P: fma(u, sW/256, -1.5*2^23*sW/256) then gives P*sW exactly,
-// with no integer-to-float conversion. (|256*P| < 2^22 requires G <= 256.)
+// TMEM holds two group accumulators (2 x 256 columns); a group's first MMA overwrites its
+// accumulator. The epilogue adds the bit pattern of 1.5 * 2^23 to the int32 partial 256*P
+// (one integer add): the sum is the bit pattern of the fp32 value 1.5 * 2^23 + 256*P, and
+// fma(u, sW/256, -1.5*2^23*sW/256) then gives P*sW exactly, with no integer-to-float
+// conversion. (|256*P| < 2^22 requires G <= 256.)
 //
 // Every mbarrier wait is bounded (about 2 s of wall time); a wait that gives up records
 // ROT_ETIMEOUT in a device flag, and the CTA skips its remaining work and exits.
@@ -184,13 +184,6 @@ __device__ __forceinline__ void umma_commit(uint64_t* bar) {
 }
 
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
-__device__ __forceinline__ void tmem_st16_const(uint32_t taddr, uint32_t v) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1};" ::"r"(taddr),
-      "r"(v)
-      : "memory");
-}
-__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 // Ordered shared-memory vector load: kept next to the TMEM load it serves, so the scale loads
 // of all column chunks are not hoisted ahead (which would need a register per loaded value).
@@ -301,13 +294,7 @@ __global__ void __launch_bounds__(THREADS, 1) w4a4_kernel(const __grid_constant_
     const int m = m0 + row;
     const uint32_t lane_addr = tmem + ((uint32_t)((warp & 3) * 32) << 16);
     const int ep_tid = threadIdx.x;           // 0..N_EPI-1
-    // initial bias in both accumulators, then release them to the MMA warp
-#pragma unroll
-    for (int b = 0; b < 2; ++b)
-#pragma unroll
-      for (int c = 0; c < EPI_COLS / 16; ++c) tmem_st16_const(lane_addr + b * BN + wg * EPI_COLS + c * 16, BIAS_BITS);
-    tmem_wait_st();
-    tc_fence_before();
+    // both accumulators start free (a group's first MMA overwrites its accumulator)
     mbar_arrive(&tempty[0]);
     mbar_arrive(&tempty[1]);
 
@@ -356,8 +343,10 @@ __global__ void __launch_bounds__(THREADS, 1) w4a4_kernel(const __grid_constant_
           for (int j = 0; j < 32; j += 4) {
             const float4 w4 = lds128(scw + c * 32 + j);
             const float4 c4 = lds128(scc + c * 32 + j);
-            const float2 u0 = make_float2(__uint_as_float(rr[j]), __uint_as_float(rr[j + 1]));
-            const float2 u1 = make_float2(__uint_as_float(rr[j + 2]), __uint_as_float(rr[j + 3]));
+            // 256*P + bits(1.5 * 2^23) = bits of the float 1.5 * 2^23 + 256*P
+            const float2 u0 = make_float2(__uint_as_float(rr[j] + BIAS_BITS), __uint_as_float(rr[j + 1] + BIAS_BITS));
+            const float2 u1 =
+                make_float2(__uint_as_float(rr[j + 2] + BIAS_BITS), __uint_as_float(rr[j + 3] + BIAS_BITS));
             // exact P*sW (the bias cancels inside one rounding), then acc += (P*sW)*sA
             const float2 t0 = __ffma2_rn(u0, make_float2(w4.x, w4.y), make_float2(c4.x, c4.y));
             const float2 t1 = __ffma2_rn(u1, make_float2(w4.z, w4.w), make_float2(c4.z, c4.w));
@@ -369,15 +358,12 @@ __global__ void __launch_bounds__(THREADS, 1) w4a4_kernel(const __grid_constant_
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
               const int n = n0 + wg * EPI_COLS + c * 32 + j;
-              if (n < p.N) p.P[((int64_t)m * p.N + n) * NG + g] = ((int32_t)(rr[j] - BIAS_BITS)) / 256;
+              if (n < p.N) p.P[((int64_t)m * p.N + n) * NG + g] = ((int32_t)rr[j]) / 256;
             }
           }
         }
       }
-      // reset the accumulator to the bias for the group after next, then release it
-#pragma unroll
-      for (int c = 0; c < EPI_COLS / 16; ++c) tmem_st16_const(base + c * 16, BIAS_BITS);
-      tmem_wait_st();
+      // the partials are in registers: release the accumulator for the group after next
       tc_fence_before();
       mbar_arrive(&tempty[b]);
     }
@@ -479,7 +465,7 @@ __global__ void __launch_bounds__(THREADS, 1) w4a4_kernel(const __grid_constant_
       if (leader) {
         const uint32_t a_addr = sbase + s * STAGE_BYTES + k4 * 32;
         const uint32_t b_addr = sbase + s * STAGE_BYTES + A_STAGE_BYTES + k4 * 32;
-        umma_i8(tmem + b * BN, make_desc(a_addr), make_desc(b_addr), 1u);
+        umma_i8(tmem + b * BN, make_desc(a_addr), make_desc(b_addr), first ? 0u : 1u);
         if (last) umma_commit(&tfull[b]);
         if (k4 == 3 || ks == KS - 1) umma_commit(&empty[s]);
       }
