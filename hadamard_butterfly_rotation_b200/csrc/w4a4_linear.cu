@@ -42,6 +42,7 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <cstdint>
 
 #include "rot_internal.cuh"
@@ -100,6 +101,8 @@ struct Params {
   int32_t* P;
   int M, N, K, G;
   int c_bf16;
+  int kb_per_split;  // K-blocks per split (blockIdx.z); a multiple of the K-blocks per group
+  float* Cacc;       // split-K: fp32 [M, N] accumulated with atomics (zeroed beforehand), else null
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -255,9 +258,16 @@ __global__ void __launch_bounds__(THREADS, 1) w4a4_kernel(const __grid_constant_
   const int lane = threadIdx.x & 31;
   const int m0 = blockIdx.y * BM;
   const int n0 = blockIdx.x * BN;
-  const int KS = p.K / 32;                 // UMMA k-steps
-  const int NKB = (p.K + KB - 1) / KB;     // K blocks
-  const int NG = p.K / p.G;
+  const int NG = p.K / p.G;                // groups of the whole K (scale row length)
+  // this CTA's K range (split-K over blockIdx.z; the split is at group boundaries)
+  const int NKB_ALL = (p.K + KB - 1) / KB;
+  const int kb0 = blockIdx.z * p.kb_per_split;
+  const int kb1 = min(NKB_ALL, kb0 + p.kb_per_split);
+  const int NKB = kb1 - kb0;                       // K blocks of this CTA
+  const int ks0 = kb0 * (KB / 32);
+  const int KS = min(p.K / 32, kb1 * (KB / 32)) - ks0;   // UMMA k-steps of this CTA
+  const int g0 = (ks0 * 32) / p.G;                 // first group
+  const int NGL = (KS * 32) / p.G;                 // groups of this CTA
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -307,31 +317,32 @@ __global__ void __launch_bounds__(THREADS, 1) w4a4_kernel(const __grid_constant_
     // scales of the next group are fetched one group ahead
     float sw_next = 0.0f, sa_next = 0.0f;
     if (!PARTIALS) {
-      if (ep_tid < BN && n_col < p.N) sw_next = __half2float(__ushort_as_half(p.Ws[(int64_t)n_col * NG]));
-      if (row_ok) sa_next = __half2float(__ushort_as_half(p.As[(int64_t)m * NG]));
+      if (ep_tid < BN && n_col < p.N) sw_next = __half2float(__ushort_as_half(p.Ws[(int64_t)n_col * NG + g0]));
+      if (row_ok) sa_next = __half2float(__ushort_as_half(p.As[(int64_t)m * NG + g0]));
     }
     bool ok = true;
-    for (int g = 0; g < NG; ++g) {
+    for (int gl = 0; gl < NGL; ++gl) {
+      const int g = g0 + gl;
       const float sa = sa_next;
       if (!PARTIALS) {
         if (ep_tid < BN) {
           const float sw = sw_next * (1.0f / 256.0f);
-          sc[((g & 1) * 2 + 0) * BN + ep_tid] = sw;
-          sc[((g & 1) * 2 + 1) * BN + ep_tid] = -BIAS_F * sw;
+          sc[((gl & 1) * 2 + 0) * BN + ep_tid] = sw;
+          sc[((gl & 1) * 2 + 1) * BN + ep_tid] = -BIAS_F * sw;
         }
-        if (g + 1 < NG) {
+        if (gl + 1 < NGL) {
           if (ep_tid < BN && n_col < p.N) sw_next = __half2float(__ushort_as_half(p.Ws[(int64_t)n_col * NG + g + 1]));
           if (row_ok) sa_next = __half2float(__ushort_as_half(p.As[(int64_t)m * NG + g + 1]));
         }
       }
       named_bar(1, N_EPI);
-      const int b = g & 1;
-      ok = ok && warp_wait(&tfull[b], (g >> 1) & 1, abort_flag, lane);   // warp-uniform
+      const int b = gl & 1;
+      ok = ok && warp_wait(&tfull[b], (gl >> 1) & 1, abort_flag, lane);   // warp-uniform
       if (!ok) continue;
       tc_fence_after();
       const uint32_t base = lane_addr + b * BN + wg * EPI_COLS;
-      const float* scw = sc + ((g & 1) * 2 + 0) * BN + wg * EPI_COLS;
-      const float* scc = sc + ((g & 1) * 2 + 1) * BN + wg * EPI_COLS;
+      const float* scw = sc + ((gl & 1) * 2 + 0) * BN + wg * EPI_COLS;
+      const float* scc = sc + ((gl & 1) * 2 + 1) * BN + wg * EPI_COLS;
       const float2 sa2 = make_float2(sa, sa);
 #pragma unroll
       for (int c = 0; c < EPI_COLS / 32; ++c) {
@@ -369,7 +380,15 @@ __global__ void __launch_bounds__(THREADS, 1) w4a4_kernel(const __grid_constant_
     }
     if (!PARTIALS && ok && row_ok) {
       const int nb = n0 + wg * EPI_COLS;
-      if (!p.c_bf16) {
+      if (p.Cacc) {
+        // split-K: add this K range's contribution (fp32 vector atomics)
+        float* crow = p.Cacc + (int64_t)m * p.N + nb;
+#pragma unroll
+        for (int j = 0; j < EPI_COLS; j += 4)
+          if (nb + j < p.N)
+            atomicAdd(reinterpret_cast<float4*>(crow + j),
+                      make_float4(acc[j / 2].x, acc[j / 2].y, acc[j / 2 + 1].x, acc[j / 2 + 1].y));
+      } else if (!p.c_bf16) {
         float* crow = static_cast<float*>(p.C) + (int64_t)m * p.N + nb;
 #pragma unroll
         for (int j = 0; j < EPI_COLS; j += 4)
@@ -399,9 +418,9 @@ __global__ void __launch_bounds__(THREADS, 1) w4a4_kernel(const __grid_constant_
     // ======================= loader: the packed A and W tiles of one K-block -> packed stage
     // (two 2-D TMA boxes; rows beyond M / N and bytes beyond K/2 arrive as zeros)
     asm volatile("setmaxnreg.dec.sync.aligned.u32 40;");
-    for (int kb = 0; kb < NKB; ++kb) {
-      const int ps = kb % PSTAGES;
-      if (kb >= PSTAGES && !warp_wait(&pempty[ps], ((kb / PSTAGES) + 1) & 1, abort_flag, lane)) break;
+    for (int j = 0; j < NKB; ++j) {
+      const int kb = kb0 + j, ps = j % PSTAGES;
+      if (j >= PSTAGES && !warp_wait(&pempty[ps], ((j / PSTAGES) + 1) & 1, abort_flag, lane)) break;
       if (lane == 0) {
         uint8_t* pst = smem + OFF_PSTAGES + ps * PSTAGE_BYTES;
         mbar_arrive_expect_tx(&pfull[ps], (uint32_t)PSTAGE_BYTES);
@@ -415,10 +434,10 @@ __global__ void __launch_bounds__(THREADS, 1) w4a4_kernel(const __grid_constant_
     // ======================= unpackers: packed stage -> swizzled int8 stage
     asm volatile("setmaxnreg.dec.sync.aligned.u32 40;");
     const int ut = threadIdx.x - (LOADER_WARP + 1) * 32;   // 0..N_UNP-1
-    for (int kb = 0; kb < NKB; ++kb) {
-      const int s = kb % STAGES, ps = kb % PSTAGES;
-      if (!warp_wait(&pfull[ps], (kb / PSTAGES) & 1, abort_flag, lane)) break;
-      if (kb >= STAGES && !warp_wait(&empty[s], ((kb / STAGES) + 1) & 1, abort_flag, lane)) break;
+    for (int j = 0; j < NKB; ++j) {
+      const int s = j % STAGES, ps = j % PSTAGES;
+      if (!warp_wait(&pfull[ps], (j / PSTAGES) & 1, abort_flag, lane)) break;
+      if (j >= STAGES && !warp_wait(&empty[s], ((j / STAGES) + 1) & 1, abort_flag, lane)) break;
       const uint8_t* pst = smem + OFF_PSTAGES + ps * PSTAGE_BYTES;
       uint8_t* st = smem + OFF_STAGES + s * STAGE_BYTES;
 #pragma unroll 4
@@ -449,17 +468,18 @@ __global__ void __launch_bounds__(THREADS, 1) w4a4_kernel(const __grid_constant_
     const bool leader = lane == 0;
     const uint32_t sbase = smem_u32(smem + OFF_STAGES);
     for (int ks = 0; ks < KS; ++ks) {
+      // local k-step / K-block / group indices drive the rings; the split is group-aligned
       const int kb = ks >> 2, k4 = ks & 3, s = kb % STAGES;
       if (k4 == 0) {
         if (!mbar_wait(&full[s], (kb / STAGES) & 1, abort_flag)) break;
         tc_fence_after();
       }
-      const int g = (ks * 32) / p.G;
+      const int gl = (ks * 32) / p.G;
       const bool first = (ks * 32) % p.G == 0;
       const bool last = ((ks + 1) * 32) % p.G == 0;
-      const int b = g & 1;
+      const int b = gl & 1;
       if (first) {
-        if (!mbar_wait(&tempty[b], (g >> 1) & 1, abort_flag)) break;
+        if (!mbar_wait(&tempty[b], (gl >> 1) & 1, abort_flag)) break;
         tc_fence_after();
       }
       if (leader) {
@@ -492,6 +512,26 @@ __global__ void __launch_bounds__(THREADS, 1) w4a4_kernel(const __grid_constant_
 }
 
 }  // namespace
+
+// Split-K factor: only when the output tiles leave most SMs idle (decode-sized M); each
+// split then covers a whole number of groups.
+int split_count(int64_t tiles, int group_units, int sms) {
+  if (tiles * 2 > sms || group_units < 2) return 1;
+  int64_t sp = sms / tiles;
+  if (sp > group_units) sp = group_units;
+  return (int)(sp < 1 ? 1 : sp);
+}
+
+__global__ void f32_to_bf16_kernel(const float* __restrict__ src, __nv_bfloat16* __restrict__ dst, int64_t n4) {
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n4; i += (int64_t)gridDim.x * blockDim.x) {
+    const float4 v = reinterpret_cast<const float4*>(src)[i];
+    __nv_bfloat162 h0 = __floats2bfloat162_rn(v.x, v.y), h1 = __floats2bfloat162_rn(v.z, v.w);
+    uint2 o;
+    o.x = *reinterpret_cast<uint32_t*>(&h0);
+    o.y = *reinterpret_cast<uint32_t*>(&h1);
+    reinterpret_cast<uint2*>(dst)[i] = o;
+  }
+}
 
 rot_status w4a4_launch(const uint8_t* Aq, const uint16_t* As, const uint8_t* Wq, const uint16_t* Ws, int64_t M,
                        int64_t N, int64_t K, int G, void* C, int c_dtype, int32_t* partials, cudaStream_t s) {
@@ -556,10 +596,35 @@ rot_status w4a4_launch(const uint8_t* Aq, const uint16_t* As, const uint8_t* Wq,
   p.K = (int)K;
   p.G = G;
   p.c_bf16 = c_dtype == ROT_BF16;
-  dim3 grid((unsigned)((N + BN - 1) / BN), (unsigned)((M + BM - 1) / BM));
+  const int64_t gx = (N + BN - 1) / BN, gy = (M + BM - 1) / BM;
+  const int nkb = (int)((K + KB - 1) / KB);
+  const int unit = G > KB ? G / KB : 1;            // K-blocks per group (split granularity)
+  const int splits = partials ? 1 : split_count(gx * gy, nkb / unit, sm_count());
+  p.kb_per_split = ((nkb / unit + splits - 1) / splits) * unit;
+  const int zs = (nkb + p.kb_per_split - 1) / p.kb_per_split;
+  p.Cacc = nullptr;
+  float* scratch_owned = nullptr;
+  if (zs > 1) {
+    // split-K: fp32 accumulation target, zeroed on the stream before the kernel
+    if (c_dtype == ROT_F32) {
+      p.Cacc = static_cast<float*>(C);
+    } else {
+      ROT_CUDA_TRY(cudaMallocAsync(reinterpret_cast<void**>(&scratch_owned), (size_t)(M * N) * sizeof(float), s));
+      p.Cacc = scratch_owned;
+    }
+    ROT_CUDA_TRY(cudaMemsetAsync(p.Cacc, 0, (size_t)(M * N) * sizeof(float), s));
+  }
+  dim3 grid((unsigned)gx, (unsigned)gy, (unsigned)zs);
   if (partials) w4a4_kernel<true><<<grid, THREADS, SMEM_BYTES, s>>>(p);
   else w4a4_kernel<false><<<grid, THREADS, SMEM_BYTES, s>>>(p);
   ROT_CUDA_TRY(cudaGetLastError());
+  if (zs > 1 && c_dtype == ROT_BF16) {
+    const int64_t n4 = M * N / 4;   // N % 16 == 0
+    const int64_t blocks = std::min<int64_t>((n4 + 255) / 256, (int64_t)sm_count() * 8);
+    f32_to_bf16_kernel<<<(unsigned)blocks, 256, 0, s>>>(p.Cacc, static_cast<__nv_bfloat16*>(C), n4);
+    ROT_CUDA_TRY(cudaGetLastError());
+  }
+  if (scratch_owned) ROT_CUDA_TRY(cudaFreeAsync(scratch_owned, s));
   return ROT_OK;
 }
 
