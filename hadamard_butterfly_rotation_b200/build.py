@@ -1,4 +1,4 @@
-"""Build the sm_100a shared library in-tree: ``python -m hadamard_butterfly_rotation_b200.build``.
+"""Build the sm_100a shared library in-tree: ``python hadamard_butterfly_rotation_b200/build.py``.
 
 Compiles every ``csrc/*.cu`` with nvcc (``-gencode arch=compute_100a,code=sm_100a``) in
 parallel and links ``_lib/librot_b200.so``. Object files go to ``_build/`` next to this
