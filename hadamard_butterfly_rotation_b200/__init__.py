@@ -1,7 +1,7 @@
 """Python binding of the B200 rotation / group-quantisation / W4A4 library (``include/rot_b200.h``).
 
 Argument marshalling only: every step runs in the CUDA library ``_lib/librot_b200.so``
-(build it with ``python -m hadamard_butterfly_rotation_b200.build``). PyTorch supplies
+(build it with ``python hadamard_butterfly_rotation_b200/build.py``). PyTorch supplies
 device memory and the current CUDA stream. Importing this package without the built
 library raises ImportError; there is no CPU fallback.
 
@@ -22,7 +22,7 @@ LIB_PATH = os.environ.get("ROT_B200_LIB") or os.path.join(_HERE, "_lib", "librot
 if not os.path.exists(LIB_PATH):
     raise ImportError(
         f"{LIB_PATH} is missing: build the CUDA library first "
-        "(python -m hadamard_butterfly_rotation_b200.build)")
+        "(python hadamard_butterfly_rotation_b200/build.py)")
 
 _lib = C.CDLL(LIB_PATH)
 
@@ -39,6 +39,7 @@ _lib.rot_apply.argtypes = [_vp, _int, _i64, _i64, _vp, _int, _vp, _i64, _vp]
 _lib.rot_quant.argtypes = [_vp, _int, _i64, _i64, _vp, _int, _int, _vp, _vp, _vp]
 _lib.rot_dequant.argtypes = [_vp, _vp, _i64, _vp, _int, _int, _int, _vp, _vp]
 _lib.w4a4_linear.argtypes = [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _int, _vp, _int, _vp]
+_lib.w4a4_linear_noalloc.argtypes = [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _int, _vp, _int, _vp]
 _lib.w4a4_group_partials.argtypes = [_vp, _vp, _i64, _i64, _i64, _int, _vp, _vp]
 _lib.rot_harp_givens_blocks.argtypes = [C.POINTER(C.c_double), _i64, C.POINTER(C.c_float)]
 _lib.rot_harp_qr_block.argtypes = [C.POINTER(C.c_double), _int, C.POINTER(C.c_float)]
@@ -46,7 +47,7 @@ _lib.rot_check_device.argtypes = []
 _lib.rot_last_error.restype = C.c_char_p
 _lib.rot_version.restype = C.c_char_p
 for _f in ("rot_plan_create", "rot_plan_destroy", "rot_plan_info", "rot_apply", "rot_quant", "rot_dequant",
-           "w4a4_linear", "w4a4_group_partials", "rot_harp_givens_blocks", "rot_harp_qr_block",
+           "w4a4_linear", "w4a4_linear_noalloc", "w4a4_group_partials", "rot_harp_givens_blocks", "rot_harp_qr_block",
            "rot_check_device"):
     getattr(_lib, _f).restype = _int
 
@@ -217,6 +218,18 @@ def w4a4_linear(Aq, As, Wq, Ws, G: int, *, out_dtype=None, out=None, stream=None
         out = torch.empty((M, N), dtype=out_dtype or torch.float32, device=Wq.device)
     cd = ROT_BF16 if out.dtype == torch.bfloat16 else ROT_F32
     _check(_lib.w4a4_linear(_ptr(Aq), _ptr(As), _ptr(Wq), _ptr(Ws), M, N, K, G, _ptr(out), cd, _stream(stream)))
+    return out
+
+
+def w4a4_linear_noalloc(Aq, As, Wq, Ws, G: int, *, out_dtype=None, out=None, stream=None):
+    """w4a4_linear that never allocates device memory (static split-K buffer; see the header)."""
+    import torch
+    M, N, K = Aq.shape[0], Wq.shape[0], Wq.shape[1] * 2
+    if out is None:
+        out = torch.empty((M, N), dtype=out_dtype or torch.float32, device=Wq.device)
+    cd = ROT_BF16 if out.dtype == torch.bfloat16 else ROT_F32
+    _check(_lib.w4a4_linear_noalloc(_ptr(Aq), _ptr(As), _ptr(Wq), _ptr(Ws), M, N, K, G, _ptr(out), cd,
+                                    _stream(stream)))
     return out
 
 

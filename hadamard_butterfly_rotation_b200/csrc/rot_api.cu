@@ -105,6 +105,23 @@ extern "C" rot_status w4a4_linear(const uint8_t* Aq, const uint16_t* As, const u
   return w4a4_launch(Aq, As, Wq, Ws, M, N, K, G, C, c_dtype, nullptr, static_cast<cudaStream_t>(stream));
 }
 
+extern "C" rot_status w4a4_linear_noalloc(const uint8_t* Aq, const uint16_t* As, const uint8_t* Wq,
+                                          const uint16_t* Ws, int64_t M, int64_t N, int64_t K, int G, void* C,
+                                          int c_dtype, void* stream) {
+  rot_status st = check_w4a4(Aq, Wq, M, N, K, G, "w4a4_linear_noalloc");
+  if (st) return st;
+  if (c_dtype != ROT_F32 && c_dtype != ROT_BF16)
+    return set_error(ROT_EINVAL, "w4a4_linear_noalloc: c_dtype must be ROT_F32 or ROT_BF16");
+  if (M == 0) return ROT_OK;
+  if (!As || !Ws || !C || !aligned16(C))
+    return set_error(ROT_EINVAL, "w4a4_linear_noalloc: As, Ws, C must be non-NULL, C 16-byte aligned");
+  float* scratch = nullptr;
+  st = w4a4_noalloc_scratch(&scratch);
+  if (st) return st;
+  return w4a4_launch(Aq, As, Wq, Ws, M, N, K, G, C, c_dtype, nullptr, static_cast<cudaStream_t>(stream), scratch,
+                     W4A4_NOALLOC_SCRATCH_FLOATS);
+}
+
 extern "C" rot_status w4a4_group_partials(const uint8_t* Aq, const uint8_t* Wq, int64_t M, int64_t N,
                                           int64_t K, int G, int32_t* P, void* stream) {
   rot_status st = check_w4a4(Aq, Wq, M, N, K, G, "w4a4_group_partials");

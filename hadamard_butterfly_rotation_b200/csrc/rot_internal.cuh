@@ -69,9 +69,14 @@ rot_status stages_quant(const rot_plan_s* p, const void* A, int a_dtype, int64_t
 rot_status dequant_launch(const uint8_t* codes, const uint16_t* scales, int64_t M, int K, int bits,
                           int G, float* out, cudaStream_t s);
 // W4A4 linear (w4a4_linear.cu)
+// split-K accumulation: `scratch` (scratch_floats floats) if non-null, else a stream-ordered
+// temporary; only used for bf16 output on the split path
+constexpr int64_t W4A4_NOALLOC_SCRATCH_FLOATS = int64_t(1) << 20;
 rot_status w4a4_launch(const uint8_t* Aq, const uint16_t* As, const uint8_t* Wq,
                        const uint16_t* Ws, int64_t M, int64_t N, int64_t K, int G, void* C,
-                       int c_dtype, int32_t* partials, cudaStream_t s);
+                       int c_dtype, int32_t* partials, cudaStream_t s, float* scratch = nullptr,
+                       int64_t scratch_floats = 0);
+rot_status w4a4_noalloc_scratch(float** out);
 
 // ---------------------------------------------------------------- device helpers
 #ifdef __CUDACC__

@@ -90,6 +90,9 @@ static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
 
 __device__ int g_w4a4_error = 0;
 
+// Static split-K accumulation buffer for w4a4_linear_noalloc (bf16 output on the split path).
+__device__ __align__(256) float g_w4a4_scratch[W4A4_NOALLOC_SCRATCH_FLOATS];
+
 struct Params {
   CUtensorMap tmA;   // packed A codes [M, K/2] uint8, box {64 bytes, BM rows}
   CUtensorMap tmW;   // packed W codes [N, K/2] uint8, box {64 bytes, BN rows}
@@ -534,7 +537,8 @@ __global__ void f32_to_bf16_kernel(const float* __restrict__ src, __nv_bfloat16*
 }
 
 rot_status w4a4_launch(const uint8_t* Aq, const uint16_t* As, const uint8_t* Wq, const uint16_t* Ws, int64_t M,
-                       int64_t N, int64_t K, int G, void* C, int c_dtype, int32_t* partials, cudaStream_t s) {
+                       int64_t N, int64_t K, int G, void* C, int c_dtype, int32_t* partials, cudaStream_t s,
+                       float* scratch, int64_t scratch_floats) {
   if (G > 256) return set_error(ROT_EUNSUPPORTED, "w4a4_linear: G > 256 is not supported");
   if (M > (1ll << 30) || N > (1ll << 30) || K > (1ll << 30)) return set_error(ROT_EUNSUPPORTED, "w4a4_linear: size too large");
   static int configured[64] = {0};
@@ -608,6 +612,10 @@ rot_status w4a4_launch(const uint8_t* Aq, const uint16_t* As, const uint8_t* Wq,
     // split-K: fp32 accumulation target, zeroed on the stream before the kernel
     if (c_dtype == ROT_F32) {
       p.Cacc = static_cast<float*>(C);
+    } else if (scratch) {
+      if (M * N > scratch_floats)
+        return set_error(ROT_EINVAL, "w4a4_linear_noalloc: M * N exceeds the static split-K buffer");
+      p.Cacc = scratch;
     } else {
       ROT_CUDA_TRY(cudaMallocAsync(reinterpret_cast<void**>(&scratch_owned), (size_t)(M * N) * sizeof(float), s));
       p.Cacc = scratch_owned;
@@ -625,6 +633,16 @@ rot_status w4a4_launch(const uint8_t* Aq, const uint16_t* As, const uint8_t* Wq,
     ROT_CUDA_TRY(cudaGetLastError());
   }
   if (scratch_owned) ROT_CUDA_TRY(cudaFreeAsync(scratch_owned, s));
+  return ROT_OK;
+}
+
+rot_status w4a4_noalloc_scratch(float** out) {
+  static float* addr[64] = {nullptr};
+  int dev = 0;
+  ROT_CUDA_TRY(cudaGetDevice(&dev));
+  if (dev >= 64) return set_error(ROT_EUNSUPPORTED, "w4a4_linear_noalloc: device index too large");
+  if (!addr[dev]) ROT_CUDA_TRY(cudaGetSymbolAddress(reinterpret_cast<void**>(&addr[dev]), g_w4a4_scratch));
+  *out = addr[dev];
   return ROT_OK;
 }
 

@@ -127,6 +127,17 @@ rot_status w4a4_linear(const uint8_t* Aq, const uint16_t* As, const uint8_t* Wq,
                        const uint16_t* Ws, int64_t M, int64_t N, int64_t K, int G, void* C,
                        int c_dtype, void* stream);
 
+/* w4a4_linear without any device allocation: on the split-K path with bf16 output the
+ * fp32 partial results accumulate in a static device buffer of 2^20 floats owned by the
+ * library (located once per device with cudaGetSymbolAddress and zeroed on the stream
+ * before each use) instead of a stream-ordered temporary. Same arguments, results and
+ * constraints as w4a4_linear; ROT_EINVAL when that path is taken with M * N > 2^20.
+ * Calls that take that path share the buffer: issue them on one stream (or otherwise
+ * serialise them). */
+rot_status w4a4_linear_noalloc(const uint8_t* Aq, const uint16_t* As, const uint8_t* Wq,
+                               const uint16_t* Ws, int64_t M, int64_t N, int64_t K, int G, void* C,
+                               int c_dtype, void* stream);
+
 /* The exact int32 group partial sums P[m, n, g] of the same contraction, written to
  * P: int32 [M, N, K/G]. Same constraints as w4a4_linear. For checking only. */
 rot_status w4a4_group_partials(const uint8_t* Aq, const uint8_t* Wq, int64_t M, int64_t N,
