@@ -55,10 +55,13 @@ def load_peaks():
 
 
 def kernel_sources_sha() -> str:
+    """Hash of the fused rotation kernel's sources: rot_fwht.cu and the device helpers of
+    rot_internal.cuh (the host declarations there do not change the kernel)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "hadamard_butterfly_rotation_b200", "csrc")
-    for f in ("rot_fwht.cu", "rot_internal.cuh"):
-        h.update(open(os.path.join(csrc, f), "rb").read())
+    h.update(open(os.path.join(csrc, "rot_fwht.cu"), "rb").read())
+    hdr = open(os.path.join(csrc, "rot_internal.cuh"), "rb").read()
+    h.update(hdr[hdr.find(b"device helpers"):])
     return h.hexdigest()[:16]
 
 
