@@ -204,8 +204,8 @@ def main():
     ap.add_argument("--no-extra", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--profile", default=None,
-                    choices=["rot_quant", "down_proj_int4", "down_proj_int2", "harp_init", "harp_random",
-                             "w4a4_prefill", "w4a4_decode"],
+                    choices=["rot_quant", "q_proj_act_int4", "down_proj_int4", "down_proj_int2", "harp_init",
+                             "harp_random", "w4a4_prefill", "w4a4_decode"],
                     help="launch only this kernel --steps times (for ncu captures); prints timing only")
     args = ap.parse_args()
     if args.warmup < 3:
@@ -399,13 +399,15 @@ def run_extra(hbr, W, dev, stream, peaks):
     out = {}
     hbm = peaks["hbm_gbs"]
     # rotate + quantise on the other workloads
-    for name, variant in (("down_proj", None), ("harp11008", "init_identity"), ("harp11008", "random")):
+    for name, variant in (("q_proj_prefill", None), ("down_proj", None), ("harp11008", "init_identity"),
+                          ("harp11008", "random")):
         wl = W.make_workload(name)
         if variant is None:
             plan = hbr.Plan.rht(wl.K, wl.signs)
         else:
             plan = hbr.harp_plan(W.harp_draws(2, wl.extra["radices"]), wl.signs, variant)
-        nsets = 3 if wl.M * wl.K * 2 > 60e6 else 6
+        # enough rotating input/output sets to exceed twice the 126 MB L2
+        nsets = max(3, -(-256_000_000 // (wl.M * wl.K * 2 + wl.M * wl.K // 2)))
         As = [torch.from_numpy(wl.A).to(torch.bfloat16).to(dev) for _ in range(nsets)]
         for bits, G in wl.quant:
             outs = [(torch.empty((wl.M, wl.K * bits // 8), dtype=torch.uint8, device=dev),
@@ -461,7 +463,8 @@ def run_profile(args):
         work = 2.0 * wl.M * Wq.shape[0] * wl.K
         unit = "TOPS"
     else:
-        wname = {"rot_quant": "llama32_1b", "down_proj_int4": "down_proj", "down_proj_int2": "down_proj",
+        wname = {"rot_quant": "llama32_1b", "q_proj_act_int4": "q_proj_prefill",
+                 "down_proj_int4": "down_proj", "down_proj_int2": "down_proj",
                  "harp_init": "harp11008", "harp_random": "harp11008"}[name]
         wl = W.make_workload(wname)
         bits, G = wl.quant[1] if name == "down_proj_int2" else wl.quant[0]

@@ -615,6 +615,7 @@ __global__ void __launch_bounds__(Cfg<LOGN>::THREADS, 1) fwht_kernel(const Args 
 //           butterflies over e3..e5, then group quantisation and packing as in fwht_kernel.
 constexpr int MMA_THREADS = 640;               // 20 warps, one chunk each
 constexpr int MMA_SLOTS = MMA_THREADS / 32;
+static_assert(MMA_SLOTS % 2 == 0, "the sign table after the slot barriers must stay 16-byte aligned");
 constexpr int MMA_SSTRIDE = 2048 + 4;          // floats per slot buffer
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
