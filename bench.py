@@ -42,6 +42,27 @@ WORKLOAD = "llama32_1b"
 INT8_DENSE_SPEC_TOPS = 4500.0
 
 
+WORKLOAD_DESC = ("llama32_1b: A[8192,2048] bf16, RHT K=2048 (signs + FWHT + 1/sqrt(K)), int4 G=32, "
+                 "packed codes + fp16 scales")
+
+
+def max_over_ranks(x: float, device=None) -> float:
+    """Max of a per-rank scalar over the process group (identity without one). Measurement
+    only: the data path has no collective."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput_gbs(bytes_per_step: int, steps: int, world: int, ms: float) -> float:
+    """Whole-job GB/s: every rank processes its own full batch (weak scaling)."""
+    return bytes_per_step * steps * world / (ms / 1e3) / 1e9
+
+
 def algorithmic_bytes(M: int, K: int, bits: int, G: int, in_bytes: int = 2) -> int:
     return M * K * in_bytes + M * K * bits // 8 + M * (K // G) * 2
 
@@ -185,7 +206,7 @@ def run_reference(args):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(1000 * tot / len(step_times), 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": "llama32_1b A[8192,2048] bf16, RHT K=2048, int4 G=32", "rows_per_step": rows},
+        "config": {"workload": WORKLOAD_DESC, "global_batch": wl.M, "rows_per_step": rows},
         "cpu_baseline": {"value": round(gbs, 4), "unit": "GB/s", "cores": cores, "kind": "oracle", "sample": sample},
         "e2e": {"value": round(gbs, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -259,13 +280,9 @@ def main():
         torch.cuda.synchronize(dev)
     if world > 1:
         dist.barrier()
-    ms = ev0.elapsed_time(ev1)
-    if world > 1:
-        t = torch.tensor([ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ev0.elapsed_time(ev1), dev)
     bytes_step = algorithmic_bytes(M, K, bits, G)
-    gbs = bytes_step * args.steps * world / (ms / 1e3) / 1e9
+    gbs = job_throughput_gbs(bytes_step, args.steps, world, ms)
     per_launch_s = ms / 1e3 / args.steps
     achieved = bytes_step / per_launch_s / 1e9
     peaks, peak_kind = load_peaks()
@@ -312,11 +329,7 @@ def main():
         e2e_step(i + 2 * E_SETS)
     e1.record(s_out)
     torch.cuda.synchronize(dev)
-    e_ms = e0.elapsed_time(e1) / e_steps
-    if world > 1:
-        t = torch.tensor([e_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e_ms = float(t.item())
+    e_ms = max_over_ranks(e0.elapsed_time(e1) / e_steps, dev)
     e2e_gbs = bytes_step * world / (e_ms / 1e3) / 1e9
 
     extra = {}
@@ -339,8 +352,7 @@ def main():
         "metric": METRIC, "value": round(gbs, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 6), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": "llama32_1b: A[8192,2048] bf16, RHT K=2048 (signs + FWHT + 1/sqrt(K)), "
-                               "int4 G=32, packed codes + fp16 scales",
+        "config": {"workload": WORKLOAD_DESC,
                    "global_batch": M * world, "l2": "6 rotating input/output sets (258 MB > 126 MB L2)",
                    "launch": "timed steps replayed from a CUDA graph holding one 6-step period",
                    "parallelism": f"dp{world} (independent rows)"},
