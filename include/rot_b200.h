@@ -23,6 +23,12 @@
  *   - Calls that take a stream are asynchronous on that stream (a cudaStream_t passed as
  *     void*, NULL = legacy default stream) and never synchronise; argument errors are
  *     detected on the host and returned before any launch.
+ *   - The fused rotation kernels (rot_apply / rot_quant on RHT-type plans) are launched
+ *     with programmatic dependent launch: their prologue (barrier set-up, copying the
+ *     plan's sign table) may overlap the tail of the previous kernel in the stream, and
+ *     every access to A and to the outputs waits for that kernel to complete. Setting
+ *     ROT_B200_PDL=0 in the environment launches them normally. Stream capture into CUDA
+ *     graphs is supported (the dependency becomes a programmatic graph edge).
  *   - Device pointers must be 16-byte aligned; leading dimensions are in elements and
  *     lda * sizeof(element) must be a multiple of 16 bytes.
  *   - Layouts (row-major):
