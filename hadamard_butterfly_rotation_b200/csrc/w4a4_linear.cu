@@ -516,6 +516,122 @@ __global__ void __launch_bounds__(THREADS, 1) w4a4_kernel(const __grid_constant_
 
 }  // namespace
 
+// ---------------------------------------------------------------- decode-sized M
+// For M <= 64 the contraction is a weight stream: every weight byte is used by at most 64
+// tokens. One warp owns 8 weight rows (an n-tile) over a K range; per 64-byte span (128
+// codes) of those rows each lane loads one 16-byte piece of its row (lanes 4g..4g+3 cover
+// row g), unpacks it to 16*q int8 words (even codes, odd codes), and feeds four
+// mma.sync.m16n8k32 s8 MMAs per 16-token tile. A span's 128 codes are split over the four
+// MMAs in an order that both operands share, so every group sum is unchanged; the int32
+// group partials stay in registers, and the epilogue per group is 4 FMAs per lane.
+// Needs G % 128 == 0; the K range of a warp is a whole number of groups.
+constexpr int DEC_THREADS = 256;
+constexpr int DEC_MAXMT = 4;   // 16-token tiles
+
+__device__ __forceinline__ void mma_s8_16832(int (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+      : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+struct DecParams {
+  const uint8_t* Aq;
+  const uint16_t* As;
+  const uint8_t* Wq;
+  const uint16_t* Ws;
+  void* C;           // output when splits == 1
+  float* Cacc;       // fp32 accumulation target (zeroed) when splits > 1
+  int M, N, K, G;
+  int c_bf16;
+  int groups_per_split;
+};
+
+template <int MT>
+__global__ void __launch_bounds__(DEC_THREADS) w4a4_decode_kernel(const DecParams p) {
+  const int warp = threadIdx.x >> 5, l = threadIdx.x & 31;
+  const int g = l >> 2, c = l & 3;
+  const int nt = blockIdx.x * (DEC_THREADS / 32) + warp;   // n-tile of 8 weight rows
+  const int n0 = nt * 8;
+  if (n0 >= p.N) return;
+  const int NG = p.K / p.G;
+  const int ga = blockIdx.y * p.groups_per_split;
+  const int gb = min(NG, ga + p.groups_per_split);
+  if (ga >= gb) return;
+  const int64_t ldp = p.K / 2;
+  const int spans_per_group = p.G / 128;
+  const uint8_t* wrow = p.Wq + (int64_t)(n0 + g) * ldp + 16 * c;
+  float acc[MT][4];
+#pragma unroll
+  for (int t = 0; t < MT; ++t)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) acc[t][i] = 0.0f;
+
+  // the next span's weight piece is loaded one span ahead
+  int span = ga * spans_per_group;
+  const int span_end = gb * spans_per_group;
+  uint4 wnext = __ldg(reinterpret_cast<const uint4*>(wrow + (int64_t)span * 64));
+  for (int gg = ga; gg < gb; ++gg) {
+    int d[MT][4];
+#pragma unroll
+    for (int t = 0; t < MT; ++t)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) d[t][i] = 0;
+    for (int sp = 0; sp < spans_per_group; ++sp, ++span) {
+      const uint4 wv = wnext;
+      if (span + 1 < span_end) wnext = __ldg(reinterpret_cast<const uint4*>(wrow + (int64_t)(span + 1) * 64));
+      const uint32_t ww[4] = {wv.x, wv.y, wv.z, wv.w};
+#pragma unroll
+      for (int t = 0; t < MT; ++t) {
+        const int m_lo = t * 16 + g, m_hi = m_lo + 8;
+        uint4 alo = make_uint4(0u, 0u, 0u, 0u), ahi = make_uint4(0u, 0u, 0u, 0u);
+        if (m_lo < p.M) alo = __ldg(reinterpret_cast<const uint4*>(p.Aq + (int64_t)m_lo * ldp + (int64_t)span * 64 + 16 * c));
+        if (m_hi < p.M) ahi = __ldg(reinterpret_cast<const uint4*>(p.Aq + (int64_t)m_hi * ldp + (int64_t)span * 64 + 16 * c));
+        const uint32_t al[4] = {alo.x, alo.y, alo.z, alo.w}, ah[4] = {ahi.x, ahi.y, ahi.z, ahi.w};
+#pragma unroll
+        for (int s4 = 0; s4 < 4; ++s4) {
+          // A rows g / g + 8: even codes (low nibbles, as 16*q) then odd codes (high nibbles)
+          const uint32_t a[4] = {(al[s4] << 4) & 0xF0F0F0F0u, (ah[s4] << 4) & 0xF0F0F0F0u, al[s4] & 0xF0F0F0F0u,
+                                 ah[s4] & 0xF0F0F0F0u};
+          mma_s8_16832(d[t], a, (ww[s4] << 4) & 0xF0F0F0F0u, ww[s4] & 0xF0F0F0F0u);
+        }
+      }
+    }
+    // group scales: D[row][col] with rows m (tokens) and cols n0 + 2c (+1)
+    const float sw0 = __half2float(__ushort_as_half(p.Ws[(int64_t)(n0 + 2 * c) * NG + gg])) * (1.0f / 256.0f);
+    const float sw1 = __half2float(__ushort_as_half(p.Ws[(int64_t)(n0 + 2 * c + 1) * NG + gg])) * (1.0f / 256.0f);
+#pragma unroll
+    for (int t = 0; t < MT; ++t) {
+      const int m_lo = t * 16 + g, m_hi = m_lo + 8;
+      const float sa0 = m_lo < p.M ? __half2float(__ushort_as_half(p.As[(int64_t)m_lo * NG + gg])) : 0.0f;
+      const float sa1 = m_hi < p.M ? __half2float(__ushort_as_half(p.As[(int64_t)m_hi * NG + gg])) : 0.0f;
+      // exact int32 partials (|256 P| < 2^22) convert exactly; P*sW then acc += (P*sW)*sA
+      acc[t][0] = fmaf((float)d[t][0] * sw0, sa0, acc[t][0]);
+      acc[t][1] = fmaf((float)d[t][1] * sw1, sa0, acc[t][1]);
+      acc[t][2] = fmaf((float)d[t][2] * sw0, sa1, acc[t][2]);
+      acc[t][3] = fmaf((float)d[t][3] * sw1, sa1, acc[t][3]);
+    }
+  }
+#pragma unroll
+  for (int t = 0; t < MT; ++t) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int m = t * 16 + g + 8 * h;
+      if (m >= p.M) continue;
+      const int n = n0 + 2 * c;
+      const float v0 = acc[t][2 * h], v1 = acc[t][2 * h + 1];
+      if (p.Cacc) {
+        atomicAdd(reinterpret_cast<float2*>(p.Cacc + (int64_t)m * p.N + n), make_float2(v0, v1));
+      } else if (p.c_bf16) {
+        *reinterpret_cast<__nv_bfloat162*>(static_cast<__nv_bfloat16*>(p.C) + (int64_t)m * p.N + n) =
+            __floats2bfloat162_rn(v0, v1);
+      } else {
+        *reinterpret_cast<float2*>(static_cast<float*>(p.C) + (int64_t)m * p.N + n) = make_float2(v0, v1);
+      }
+    }
+  }
+}
+
 // Split-K factor: only when the output tiles leave most SMs idle (decode-sized M); each
 // split then covers a whole number of groups.
 int split_count(int64_t tiles, int group_units, int sms) {
@@ -541,6 +657,67 @@ rot_status w4a4_launch(const uint8_t* Aq, const uint16_t* As, const uint8_t* Wq,
                        float* scratch, int64_t scratch_floats) {
   if (G > 256) return set_error(ROT_EUNSUPPORTED, "w4a4_linear: G > 256 is not supported");
   if (M > (1ll << 30) || N > (1ll << 30) || K > (1ll << 30)) return set_error(ROT_EUNSUPPORTED, "w4a4_linear: size too large");
+  // fp32 accumulation target for K-split launches: C itself (fp32), the caller's scratch, or a
+  // stream-ordered temporary (bf16 output); zeroed on the stream
+  float* scratch_owned = nullptr;
+  auto acc_target = [&](float** out) -> rot_status {
+    if (c_dtype == ROT_F32) {
+      *out = static_cast<float*>(C);
+    } else if (scratch) {
+      if (M * N > scratch_floats)
+        return set_error(ROT_EINVAL, "w4a4_linear_noalloc: M * N exceeds the static split-K buffer");
+      *out = scratch;
+    } else {
+      ROT_CUDA_TRY(cudaMallocAsync(reinterpret_cast<void**>(&scratch_owned), (size_t)(M * N) * sizeof(float), s));
+      *out = scratch_owned;
+    }
+    ROT_CUDA_TRY(cudaMemsetAsync(*out, 0, (size_t)(M * N) * sizeof(float), s));
+    return ROT_OK;
+  };
+  auto finish_acc = [&](float* acc) -> rot_status {
+    if (c_dtype == ROT_BF16) {
+      const int64_t n4 = M * N / 4;   // N % 16 == 0
+      const int64_t blocks = std::min<int64_t>((n4 + 255) / 256, (int64_t)sm_count() * 8);
+      f32_to_bf16_kernel<<<(unsigned)blocks, 256, 0, s>>>(acc, static_cast<__nv_bfloat16*>(C), n4);
+      ROT_CUDA_TRY(cudaGetLastError());
+    }
+    if (scratch_owned) ROT_CUDA_TRY(cudaFreeAsync(scratch_owned, s));
+    return ROT_OK;
+  };
+  if (!partials && M <= 16 * DEC_MAXMT && G % 128 == 0) {
+    // decode-sized M: weight-streaming kernel, K split until about 16 warps per SM are busy
+    const int64_t ntiles = N / 8;
+    const int NG = (int)(K / G);
+    int64_t want = ((int64_t)sm_count() * 16 + ntiles - 1) / ntiles;
+    const int splits0 = (int)std::max<int64_t>(1, std::min<int64_t>(NG, want));
+    const int gps = (NG + splits0 - 1) / splits0;
+    const int splits = (NG + gps - 1) / gps;
+    DecParams d{};
+    d.Aq = Aq;
+    d.As = As;
+    d.Wq = Wq;
+    d.Ws = Ws;
+    d.C = C;
+    d.Cacc = nullptr;
+    d.M = (int)M;
+    d.N = (int)N;
+    d.K = (int)K;
+    d.G = G;
+    d.c_bf16 = c_dtype == ROT_BF16;
+    d.groups_per_split = gps;
+    if (splits > 1) {
+      rot_status st = acc_target(&d.Cacc);
+      if (st) return st;
+    }
+    const dim3 grid((unsigned)((ntiles + DEC_THREADS / 32 - 1) / (DEC_THREADS / 32)), (unsigned)splits);
+    const int mt = (int)((M + 15) / 16);
+    if (mt == 1) w4a4_decode_kernel<1><<<grid, DEC_THREADS, 0, s>>>(d);
+    else if (mt == 2) w4a4_decode_kernel<2><<<grid, DEC_THREADS, 0, s>>>(d);
+    else if (mt == 3) w4a4_decode_kernel<3><<<grid, DEC_THREADS, 0, s>>>(d);
+    else w4a4_decode_kernel<4><<<grid, DEC_THREADS, 0, s>>>(d);
+    ROT_CUDA_TRY(cudaGetLastError());
+    return splits > 1 ? finish_acc(d.Cacc) : ROT_OK;
+  }
   static int configured[64] = {0};
   int dev = 0;
   cudaGetDevice(&dev);
@@ -607,33 +784,15 @@ rot_status w4a4_launch(const uint8_t* Aq, const uint16_t* As, const uint8_t* Wq,
   p.kb_per_split = ((nkb / unit + splits - 1) / splits) * unit;
   const int zs = (nkb + p.kb_per_split - 1) / p.kb_per_split;
   p.Cacc = nullptr;
-  float* scratch_owned = nullptr;
   if (zs > 1) {
-    // split-K: fp32 accumulation target, zeroed on the stream before the kernel
-    if (c_dtype == ROT_F32) {
-      p.Cacc = static_cast<float*>(C);
-    } else if (scratch) {
-      if (M * N > scratch_floats)
-        return set_error(ROT_EINVAL, "w4a4_linear_noalloc: M * N exceeds the static split-K buffer");
-      p.Cacc = scratch;
-    } else {
-      ROT_CUDA_TRY(cudaMallocAsync(reinterpret_cast<void**>(&scratch_owned), (size_t)(M * N) * sizeof(float), s));
-      p.Cacc = scratch_owned;
-    }
-    ROT_CUDA_TRY(cudaMemsetAsync(p.Cacc, 0, (size_t)(M * N) * sizeof(float), s));
+    rot_status st = acc_target(&p.Cacc);
+    if (st) return st;
   }
   dim3 grid((unsigned)gx, (unsigned)gy, (unsigned)zs);
   if (partials) w4a4_kernel<true><<<grid, THREADS, SMEM_BYTES, s>>>(p);
   else w4a4_kernel<false><<<grid, THREADS, SMEM_BYTES, s>>>(p);
   ROT_CUDA_TRY(cudaGetLastError());
-  if (zs > 1 && c_dtype == ROT_BF16) {
-    const int64_t n4 = M * N / 4;   // N % 16 == 0
-    const int64_t blocks = std::min<int64_t>((n4 + 255) / 256, (int64_t)sm_count() * 8);
-    f32_to_bf16_kernel<<<(unsigned)blocks, 256, 0, s>>>(p.Cacc, static_cast<__nv_bfloat16*>(C), n4);
-    ROT_CUDA_TRY(cudaGetLastError());
-  }
-  if (scratch_owned) ROT_CUDA_TRY(cudaFreeAsync(scratch_owned, s));
-  return ROT_OK;
+  return zs > 1 ? finish_acc(p.Cacc) : ROT_OK;
 }
 
 rot_status w4a4_noalloc_scratch(float** out) {
