@@ -11,31 +11,29 @@
 // in int32), with the even codes of every 32-code chunk placed before the odd ones. The
 // same K permutation is applied to both operands, so every group sum is unchanged.
 //
-// Tile: 128 rows of A x 256 rows of W per CTA; K in blocks of 128 (one 128-byte swizzle
-// atom of int8 per row), 4 UMMAs of K = 32 per block, 3-stage ring of unpacked int8 tiles fed
-// by a 2-stage ring of packed tiles. (A 128 x 128 tile re-reads A twice as often and
-// measured slower.)
+// Persistent kernel: one CTA per SM walks a static list of work units (128 x 128 output
+// tiles, times the K splits when the tiles alone leave SMs idle), M-index fastest so that
+// the CTAs running at the same time share weight tiles in L2. Per K-block of 128: the
+// loader warp brings the packed A and W tiles (two 2-D TMA boxes) into a 6-deep packed
+// ring; 6 unpacker warps expand them into a 3-deep ring of swizzled K-major int8 tiles;
+// one thread issues 4 UMMAs (M = N = 128, K = 32) per K-block into one of four 128-column
+// TMEM accumulators, one per group in flight, so the tensor pipe can run three groups
+// ahead of the epilogue.
 // Warp roles (512 threads, launched with 128 registers each). setmaxnreg acts on whole
-// warpgroups, so roles are aligned to them: warpgroups 0-1 (epilogue) grow to 216 registers,
-// warpgroups 2-3 (loader, unpackers, MMA warp) shrink to 40: 256*216 + 256*40 = 512*128.
-//   warps 0-7   epilogue: two warpgroups, 128 columns each; after each group they read
-//               the int32 partials from TMEM (32 columns per load), apply the group scales
-//               and accumulate in fp32 registers (packed f32x2 FMAs);
-//   warp 8      loader: one bulk copy (cp.async.bulk) per tile row and K-block brings the
-//               packed codes into the packed ring, completing on an mbarrier;
-//   warps 9-14  unpackers: read a packed stage from shared memory, unpack, store into the
-//               swizzled K-major int8 layout, fence.proxy.async, then release both stages;
-//   warp 15     TMEM allocation and MMA issue (one elected lane).
-// Measured on B200 at M=2048, N=K=4096 (timestamps and role-by-role variants): the MMA warp
-// alone reaches 1529 TOPS; the epilogue's per-group TMEM traffic (read 256 partial columns,
-// rewrite the bias) slows the MMAs on the other accumulator several-fold while it runs, so
-// at G = 128 the epilogue's TMEM time, not the unpacking, bounds the kernel (G = 256 halves
-// it). Per-row bulk copies of the packed codes were 5x slower than the two 2-D TMA boxes.
-// TMEM holds two group accumulators (2 x 256 columns); a group's first MMA overwrites its
-// accumulator. The epilogue adds the bit pattern of 1.5 * 2^23 to the int32 partial 256*P
-// (one integer add): the sum is the bit pattern of the fp32 value 1.5 * 2^23 + 256*P, and
-// fma(u, sW/256, -1.5*2^23*sW/256) then gives P*sW exactly, with no integer-to-float
-// conversion. (|256*P| < 2^22 requires G <= 256.)
+// warpgroups, so roles are aligned to them: warpgroups 0-1 (epilogue) grow to 176 registers,
+// warpgroups 2-3 (loader, unpackers, MMA warp) shrink to 80: 256*176 + 256*80 = 512*128.
+//   warps 0-7   epilogue: warp w reads TMEM lanes 32*(w%4).. and columns 64*(w/4)..+63 of
+//               a group's accumulator (two 32-column loads in flight), scales them and
+//               accumulates in fp32 registers (packed f32x2 FMAs); it also stages the
+//               group scales two groups ahead into a ring of shared-memory slots;
+//   warp 8      loader;   warps 9-14 unpackers;   warp 15 TMEM allocation and MMA issue.
+// Group scaling: the epilogue adds the bit pattern of 1.5 * 2^23 to the int32 partial 256*P
+// (one integer add): the sum is the bit pattern of the fp32 value 1.5 * 2^23 + 256*P, so
+// fma(u, sA, -1.5*2^23*sA) = 256*P*sA rounded once, with no integer-to-float conversion
+// (|256*P| < 2^22 requires G <= 256), and acc += that * sW/256.
+// Measured on B200 (a probe with the MMAs and eight warps of TMEM loads running together):
+// 128-column int8 UMMAs keep their full rate while the TMEM is read, so the accumulator
+// depth, not TMEM bandwidth, sets how far the MMAs can run ahead of the epilogue.
 //
 // Every mbarrier wait is bounded (about 2 s of wall time); a wait that gives up records
 // ROT_ETIMEOUT in a device flag, and the CTA skips its remaining work and exits.
@@ -51,30 +49,37 @@ namespace rotb {
 namespace {
 
 constexpr int BM = 128;
-constexpr int BN = 256;
+constexpr int BN = 128;
 constexpr int KB = 128;                  // K elements per stage
 constexpr int STAGES = 3;                // unpacked int8 stages
-constexpr int PSTAGES = 2;               // packed stages
+constexpr int PSTAGES = 6;               // packed stages
+constexpr int NACC = 4;                  // TMEM accumulators (groups in flight)
+constexpr int NSLOT = 8;                 // scale slots
+constexpr int SLOT_AHEAD = 2;            // groups between staging a slot and reading it
+static_assert(NSLOT > SLOT_AHEAD + NACC, "a slot is rewritten only after every epilogue warp has left it");
 constexpr int A_STAGE_BYTES = BM * KB;   // unpacked int8
 constexpr int B_STAGE_BYTES = BN * KB;
 constexpr int STAGE_BYTES = A_STAGE_BYTES + B_STAGE_BYTES;
 constexpr int PROW_BYTES = KB / 2;       // packed bytes of one row in one K-block
 constexpr int PSTAGE_BYTES = (BM + BN) * PROW_BYTES;
 constexpr int N_EPI = 256;               // epilogue threads (2 warpgroups)
+constexpr int N_EPI_WARPS = N_EPI / 32;
 constexpr int LOADER_WARP = N_EPI / 32;  // warp 8
 constexpr int N_UNP = 192;               // unpacker threads (warps 9-14)
 constexpr int N_UNP_WARPS = N_UNP / 32;
 constexpr int THREADS = N_EPI + 32 + N_UNP + 32;
 constexpr int N_CHUNKS = (BM + BN) * (KB / 32);                  // 16-byte packed chunks / stage
-constexpr int UNP_CHUNKS = N_CHUNKS / N_UNP;                     // per unpacker thread
-constexpr int EPI_COLS = BN / 2;         // columns per epilogue warpgroup
+constexpr int UNP_ITERS = (N_CHUNKS + N_UNP - 1) / N_UNP;        // per unpacker thread (last one partial)
+constexpr int EPI_COLS = BN / 2;         // columns per epilogue warp
 constexpr int MMA_WARP = (N_EPI + 32 + N_UNP) / 32;
 constexpr int LAUNCH_REGS = 128;         // 65536 / THREADS
-constexpr int EPI_REGS = 216, PROD_REGS = 40;  // per warpgroup role
+constexpr int EPI_REGS = 176, PROD_REGS = 80;  // per warpgroup role
 static_assert(THREADS == 512, "register split assumes 512 threads");
-static_assert(N_CHUNKS % N_UNP == 0, "unpack work divides evenly");
+static_assert(N_UNP % 4 == 0 && (N_UNP / 4) % 8 == 0, "an unpacker keeps its chunk column and swizzle phase");
 static_assert(N_EPI * EPI_REGS + (THREADS - N_EPI) * PROD_REGS <= THREADS * LAUNCH_REGS, "register split");
-constexpr uint32_t TMEM_COLS = 2 * BN;   // two group accumulators (all 512 columns)
+static_assert(A_STAGE_BYTES == BM * 128, "A and W int8 tiles are contiguous 128-byte rows");
+constexpr uint32_t TMEM_COLS = NACC * BN;   // all 512 columns
+static_assert(TMEM_COLS == 512, "TMEM columns");
 constexpr uint32_t BIAS_BITS = 0x4B400000u;  // 1.5 * 2^23
 constexpr float BIAS_F = 12582912.0f;
 constexpr unsigned long long WAIT_NS = 2000000000ull;
@@ -82,11 +87,14 @@ constexpr unsigned long long WAIT_NS = 2000000000ull;
 // smem layout (offsets from a 1024-byte aligned base)
 constexpr int OFF_STAGES = 0;
 constexpr int OFF_PSTAGES = STAGES * STAGE_BYTES;
-constexpr int OFF_SCALES = OFF_PSTAGES + PSTAGES * PSTAGE_BYTES;  // [2][2][BN] fp32: sW/256, -1.5*2^23*sW/256
-constexpr int OFF_BARS = OFF_SCALES + 2 * BN * 8;
-constexpr int OFF_TMEM = OFF_BARS + 16 * 8;
+constexpr int OFF_SLOTS = OFF_PSTAGES + PSTAGES * PSTAGE_BYTES;  // [NSLOT] {sW/256 [BN], sA [BM]} fp32
+constexpr int SLOT_FLOATS = BN + BM;
+constexpr int OFF_BARS = OFF_SLOTS + NSLOT * SLOT_FLOATS * 4;
+constexpr int N_BARS = 2 * STAGES + 2 * PSTAGES + 2 * NACC + NSLOT;
+constexpr int OFF_TMEM = OFF_BARS + N_BARS * 8;
 constexpr int SMEM_BYTES = OFF_TMEM + 16 + 1024;          // + alignment slack
 static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
+static_assert(OFF_PSTAGES % 1024 == 0 && PSTAGE_BYTES % 1024 == 0, "TMA destinations stay 128-byte aligned");
 
 __device__ int g_w4a4_error = 0;
 
@@ -104,9 +112,37 @@ struct Params {
   int32_t* P;
   int M, N, K, G;
   int c_bf16;
-  int kb_per_split;  // K-blocks per split (blockIdx.z); a multiple of the K-blocks per group
+  int tiles_m;       // output tiles along M
+  int splits;        // K splits per tile
+  int units;         // tiles * splits
+  int kb_per_split;  // K-blocks per split; a multiple of lcm(G, KB) / KB
   float* Cacc;       // split-K: fp32 [M, N] accumulated with atomics (zeroed beforehand), else null
 };
+
+// One work unit: an output tile and a group-aligned K range.
+struct Unit {
+  int m0, n0;
+  int kb0, nkb;      // first K-block, K-blocks
+  int ks0, ks;       // first UMMA k-step (K = 32 each), k-steps
+  int g0, ngl;       // first group, groups
+};
+
+__device__ __forceinline__ Unit unit_of(const Params& p, int u) {
+  Unit w;
+  const int t = u / p.splits, z = u - t * p.splits;
+  const int tm = t % p.tiles_m, tn = t / p.tiles_m;
+  w.m0 = tm * BM;
+  w.n0 = tn * BN;
+  const int nkb_all = (p.K + KB - 1) / KB;
+  w.kb0 = z * p.kb_per_split;
+  const int kb1 = min(nkb_all, w.kb0 + p.kb_per_split);
+  w.nkb = kb1 - w.kb0;
+  w.ks0 = w.kb0 * (KB / 32);
+  w.ks = min(p.K / 32, kb1 * (KB / 32)) - w.ks0;
+  w.g0 = (w.ks0 * 32) / p.G;
+  w.ngl = (w.ks * 32) / p.G;
+  return w;
+}
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -120,32 +156,46 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
   asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.shared::cta.b64 st, [%0];\n\t}" ::"r"(smem_u32(bar)) : "memory");
 }
 
-// Bounded wait for the phase with the given parity; returns false on timeout.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+// Bounded wait for the phase with the given parity, by every lane of a converged warp; the
+// result is warp-uniform. A plain try_wait on a completed phase costs ~13 cycles on B200, where
+// one lane waiting with a suspend-time hint and broadcasting by shuffle measured ~130: every
+// role here waits once or twice per K-block, so the cheap form matters. Between unsuccessful
+// polls the warp sleeps for a few tens of nanoseconds. Gives up after ~2 s (records
+// ROT_ETIMEOUT and raises the CTA's abort flag).
+__device__ __forceinline__ bool bar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
   const uint32_t addr = smem_u32(bar);
-  uint32_t done = 0;
+  bool ok = true;
   unsigned long long t0 = 0;
   for (uint32_t it = 0;; ++it) {
+    uint32_t done;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(done)
-        : "r"(addr), "r"(parity), "r"(20000u)   // suspend up to 20 us per try (no spinning)
+        : "r"(addr), "r"(parity)
         : "memory");
-    if (done) return true;
-    if ((it & 7) == 7) {
-      if (*abort_flag) return false;
+    if (done) break;
+    // a polling warp takes issue slots from the epilogue's arithmetic on the same scheduler:
+    // back off briefly between polls
+    __nanosleep(32);
+    if ((it & 63) == 63) {
+      if (*abort_flag) {
+        ok = false;
+        break;
+      }
       unsigned long long now;
       asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(now));
       if (t0 == 0) t0 = now;
       else if (now - t0 > WAIT_NS) {
         *abort_flag = 1;
         atomicExch(&g_w4a4_error, (int)ROT_ETIMEOUT);
-        return false;
+        ok = false;
+        break;
       }
     }
   }
+  return __all_sync(0xffffffffu, ok);
 }
 
 __device__ __forceinline__ void fence_proxy_async() {
@@ -175,18 +225,23 @@ constexpr uint32_t IDESC = (2u << 4)            // D format: s32
                            | (1u << 10)         // B: signed int8
                            | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
 
+// Issued by the whole (converged) warp: elect.sync picks the one lane that issues, so the
+// operands stay warp-uniform (issuing from a diverged lane measured ~40% slower per MMA).
 __device__ __forceinline__ void umma_i8(uint32_t tmem_d, uint64_t da, uint64_t db, uint32_t accumulate) {
   asm volatile(
-      "{\n\t.reg .pred p;\n\t"
+      "{\n\t.reg .pred p, e;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
       "l"(da), "l"(db), "r"(IDESC), "r"(accumulate)
       : "memory");
 }
 
 __device__ __forceinline__ void umma_commit(uint64_t* bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
-               : "memory");
+  asm volatile(
+      "{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(smem_u32(bar))
+      : "memory");
 }
 
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
@@ -199,10 +254,6 @@ __device__ __forceinline__ float4 lds128(const float* p) {
                : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
                : "r"(smem_u32(p)));
   return v;
-}
-
-__device__ __forceinline__ void named_bar(int id, int n) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
 }
 
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
@@ -231,60 +282,40 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* tmap, 
       : "memory");
 }
 
-// Warp-uniform bounded wait: lane 0 waits on the mbarrier, the result is broadcast and the
-// warp re-converges (its memory accesses are ordered after lane 0's acquire by __syncwarp).
-__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag, int lane) {
-  int w = 1;
-  if (lane == 0) w = mbar_wait(bar, parity, abort_flag) ? 1 : 0;
-  w = __shfl_sync(0xffffffffu, w, 0);
-  __syncwarp();
-  return w != 0;
-}
-
 template <bool PARTIALS>
 __global__ void __launch_bounds__(THREADS, 1) w4a4_kernel(const __grid_constant__ Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BARS);
-  uint64_t* full = bars;                      // [STAGES]  unpackers -> MMA (one arrival per warp)
-  uint64_t* empty = bars + STAGES;            // [STAGES]  MMA commit -> unpackers
-  uint64_t* tfull = bars + 2 * STAGES;        // [2]       MMA commit -> epilogue
-  uint64_t* tempty = bars + 2 * STAGES + 2;   // [2]       epilogue -> MMA
-  uint64_t* pfull = bars + 2 * STAGES + 4;    // [PSTAGES] bulk copies -> unpackers
-  uint64_t* pempty = bars + 2 * STAGES + 4 + PSTAGES;  // [PSTAGES] unpackers -> loader
-  static_assert(2 * STAGES + 4 + 2 * PSTAGES <= 16, "barrier slots");
+  uint64_t* full = bars;                 // [STAGES]  unpackers -> MMA (one arrival per unpacker warp)
+  uint64_t* empty = full + STAGES;       // [STAGES]  MMA commit -> unpackers
+  uint64_t* pfull = empty + STAGES;      // [PSTAGES] TMA bytes -> unpackers
+  uint64_t* pempty = pfull + PSTAGES;    // [PSTAGES] unpackers -> loader
+  uint64_t* tfull = pempty + PSTAGES;    // [NACC]    MMA commit -> epilogue
+  uint64_t* tempty = tfull + NACC;       // [NACC]    epilogue warps -> MMA
+  uint64_t* sfull = tempty + NACC;       // [NSLOT]   epilogue warps (staging) -> epilogue warps
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_TMEM);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + OFF_TMEM + 8);
-  float* sc = reinterpret_cast<float*>(smem + OFF_SCALES);  // [buf][0: sW/256, 1: c][BN]
+  float* slots = reinterpret_cast<float*>(smem + OFF_SLOTS);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int m0 = blockIdx.y * BM;
-  const int n0 = blockIdx.x * BN;
   const int NG = p.K / p.G;                // groups of the whole K (scale row length)
-  // this CTA's K range (split-K over blockIdx.z; the split is at group boundaries)
-  const int NKB_ALL = (p.K + KB - 1) / KB;
-  const int kb0 = blockIdx.z * p.kb_per_split;
-  const int kb1 = min(NKB_ALL, kb0 + p.kb_per_split);
-  const int NKB = kb1 - kb0;                       // K blocks of this CTA
-  const int ks0 = kb0 * (KB / 32);
-  const int KS = min(p.K / 32, kb1 * (KB / 32)) - ks0;   // UMMA k-steps of this CTA
-  const int g0 = (ks0 * 32) / p.G;                 // first group
-  const int NGL = (KS * 32) / p.G;                 // groups of this CTA
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], N_UNP_WARPS);
       mbar_init(&empty[s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&tfull[b], 1);
-      mbar_init(&tempty[b], N_EPI);
-    }
     for (int s = 0; s < PSTAGES; ++s) {
       mbar_init(&pfull[s], 1);
       mbar_init(&pempty[s], N_UNP_WARPS);
     }
+    for (int b = 0; b < NACC; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], N_EPI_WARPS);
+    }
+    for (int s = 0; s < NSLOT; ++s) mbar_init(&sfull[s], N_EPI_WARPS);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -299,205 +330,316 @@ __global__ void __launch_bounds__(THREADS, 1) w4a4_kernel(const __grid_constant_
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp < N_EPI / 32) {
+  if (warp < N_EPI_WARPS) {
     // ======================= epilogue
-    asm volatile("setmaxnreg.inc.sync.aligned.u32 216;");
-    const int wg = warp >> 2;                 // column block of EPI_COLS
-    const int row = (warp & 3) * 32 + lane;   // TMEM lane = tile row
-    const int m = m0 + row;
-    const uint32_t lane_addr = tmem + ((uint32_t)((warp & 3) * 32) << 16);
-    const int ep_tid = threadIdx.x;           // 0..N_EPI-1
-    // both accumulators start free (a group's first MMA overwrites its accumulator)
-    mbar_arrive(&tempty[0]);
-    mbar_arrive(&tempty[1]);
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 176;");
+    const int qd = warp & 3;                  // TMEM lane quadrant
+    const int wg = warp >> 2;                 // column half of the tile
+    const int row = qd * 32 + lane;           // TMEM lane = tile row
+    const uint32_t lane_addr = tmem + ((uint32_t)(qd * 32) << 16) + wg * EPI_COLS;
+    // all accumulators start free (a group's first MMA overwrites its accumulator)
+    if (lane == 0)
+      for (int b = 0; b < NACC; ++b) mbar_arrive(&tempty[b]);
 
-    // fp32 accumulators as pairs of adjacent columns
+    // Scale staging runs SLOT_AHEAD groups ahead of the accumulation. Warps 0-3 stage sW/256
+    // of column threadIdx.x, warps 4-7 sA of their row. The raw binary16 values are loaded
+    // LQ groups before they are staged, into a ring of registers that a switch on the ring
+    // index addresses statically (no register is read while its load is still in flight).
+    int su = blockIdx.x;                      // load cursor: unit and group within it
+    int sg = 0;
+    int s_g0 = 0, s_ngl = 0, s_m0 = 0, s_n0 = 0;
+    auto cursor_unit = [&]() {
+      if (su < p.units) {
+        const Unit w = unit_of(p, su);
+        s_g0 = w.g0;
+        s_ngl = w.ngl;
+        s_m0 = w.m0;
+        s_n0 = w.n0;
+      }
+    };
+    // address of the raw scale at the cursor: clamped into the matrix (rows >= M and columns
+    // >= N are never stored, so their scale is irrelevant) and a valid dummy past the end, so
+    // that every load is unconditional and lands straight in its ring register
+    auto cursor_addr = [&]() -> const uint16_t* {
+      if (su >= p.units) return p.Ws;
+      const int g = s_g0 + sg;
+      if (wg == 0) return p.Ws + (int64_t)min(s_n0 + (int)threadIdx.x, p.N - 1) * NG + g;
+      return p.As + (int64_t)min(s_m0 + row, p.M - 1) * NG + g;
+    };
+    auto cursor_step = [&]() {
+      if (su < p.units && ++sg == s_ngl) {
+        sg = 0;
+        su += gridDim.x;
+        cursor_unit();
+      }
+    };
+    auto cursor_next = [&]() -> uint16_t {
+      const uint16_t v = __ldg(cursor_addr());
+      cursor_step();
+      return v;
+    };
+    int total = 0;                            // groups this CTA accumulates
+    if (!PARTIALS)
+      for (int u = blockIdx.x; u < p.units; u += gridDim.x) total += unit_of(p, u).ngl;
+    auto stage = [&](int gidx, uint16_t raw) {
+      if (gidx >= total) return;
+      const float v = __half2float(__ushort_as_half(raw));
+      float* sl = slots + (gidx % NSLOT) * SLOT_FLOATS;
+      if (wg == 0) sl[threadIdx.x] = v * (1.0f / 256.0f);
+      else sl[BN + row] = v;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sfull[gidx % NSLOT]);
+    };
+    uint16_t sq0 = 0, sq1 = 0, sq2 = 0, sq3 = 0;   // groups gc+SLOT_AHEAD+{0..3} (mod 4 ring)
+    if (!PARTIALS) {
+      cursor_unit();
+      for (int i = 0; i < SLOT_AHEAD; ++i) stage(i, cursor_next());
+      sq0 = cursor_next();
+      sq1 = cursor_next();
+      sq2 = cursor_next();
+      sq3 = cursor_next();
+    }
+
     float2 acc[EPI_COLS / 2];
 #pragma unroll
     for (int j = 0; j < EPI_COLS / 2; ++j) acc[j] = make_float2(0.0f, 0.0f);
-    const bool row_ok = m < p.M;
-    const int n_col = n0 + ep_tid;            // the column whose scale this thread stages
-    // scales of the next group are fetched one group ahead
-    float sw_next = 0.0f, sa_next = 0.0f;
-    if (!PARTIALS) {
-      if (ep_tid < BN && n_col < p.N) sw_next = __half2float(__ushort_as_half(p.Ws[(int64_t)n_col * NG + g0]));
-      if (row_ok) sa_next = __half2float(__ushort_as_half(p.As[(int64_t)m * NG + g0]));
-    }
     bool ok = true;
-    for (int gl = 0; gl < NGL; ++gl) {
-      const int g = g0 + gl;
-      const float sa = sa_next;
-      if (!PARTIALS) {
-        if (ep_tid < BN) {
-          const float sw = sw_next * (1.0f / 256.0f);
-          sc[((gl & 1) * 2 + 0) * BN + ep_tid] = sw;
-          sc[((gl & 1) * 2 + 1) * BN + ep_tid] = -BIAS_F * sw;
+    int gc = 0;                               // groups accumulated by this CTA so far
+    for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x) {
+      const Unit w = unit_of(p, u);
+      const int m = w.m0 + row;
+      const bool row_ok = m < p.M;
+      for (int gl = 0; gl < w.ngl; ++gl, ++gc) {
+        if (!PARTIALS) {
+          const uint16_t* sa_next = cursor_addr();
+          cursor_step();
+          switch (gc & 3) {
+            case 0: stage(gc + SLOT_AHEAD, sq0); sq0 = __ldg(sa_next); break;
+            case 1: stage(gc + SLOT_AHEAD, sq1); sq1 = __ldg(sa_next); break;
+            case 2: stage(gc + SLOT_AHEAD, sq2); sq2 = __ldg(sa_next); break;
+            default: stage(gc + SLOT_AHEAD, sq3); sq3 = __ldg(sa_next); break;
+          }
+          ok = ok && bar_wait(&sfull[gc % NSLOT], (gc / NSLOT) & 1, abort_flag);
         }
-        if (gl + 1 < NGL) {
-          if (ep_tid < BN && n_col < p.N) sw_next = __half2float(__ushort_as_half(p.Ws[(int64_t)n_col * NG + g + 1]));
-          if (row_ok) sa_next = __half2float(__ushort_as_half(p.As[(int64_t)m * NG + g + 1]));
-        }
-      }
-      named_bar(1, N_EPI);
-      const int b = gl & 1;
-      ok = ok && warp_wait(&tfull[b], (gl >> 1) & 1, abort_flag, lane);   // warp-uniform
-      if (!ok) continue;
-      tc_fence_after();
-      const uint32_t base = lane_addr + b * BN + wg * EPI_COLS;
-      const float* scw = sc + ((gl & 1) * 2 + 0) * BN + wg * EPI_COLS;
-      const float* scc = sc + ((gl & 1) * 2 + 1) * BN + wg * EPI_COLS;
-      const float2 sa2 = make_float2(sa, sa);
-#pragma unroll
-      for (int c = 0; c < EPI_COLS / 32; ++c) {
-        uint32_t rr[32];
-        tmem_ld32(base + c * 32, rr);
+        const int b = gc % NACC;
+        ok = ok && bar_wait(&tfull[b], (gc / NACC) & 1, abort_flag);
+        if (!ok) break;
+        tc_fence_after();
+        uint32_t r0[32], r1[32];
+        tmem_ld32(lane_addr + b * BN, r0);
+        tmem_ld32(lane_addr + b * BN + 32, r1);
         tmem_wait_ld();
         if constexpr (!PARTIALS) {
+          const float* sl = slots + (gc % NSLOT) * SLOT_FLOATS;
+          const float sa = sl[BN + row];
+          const float2 sa2 = make_float2(sa, sa);
+          const float2 d2 = make_float2(-BIAS_F * sa, -BIAS_F * sa);   // exact: 3 * 2^22 * binary16
+          const float* scw = sl + wg * EPI_COLS;
 #pragma unroll
-          for (int j = 0; j < 32; j += 4) {
-            const float4 w4 = lds128(scw + c * 32 + j);
-            const float4 c4 = lds128(scc + c * 32 + j);
-            // 256*P + bits(1.5 * 2^23) = bits of the float 1.5 * 2^23 + 256*P
-            const float2 u0 = make_float2(__uint_as_float(rr[j] + BIAS_BITS), __uint_as_float(rr[j + 1] + BIAS_BITS));
-            const float2 u1 =
-                make_float2(__uint_as_float(rr[j + 2] + BIAS_BITS), __uint_as_float(rr[j + 3] + BIAS_BITS));
-            // exact P*sW (the bias cancels inside one rounding), then acc += (P*sW)*sA
-            const float2 t0 = __ffma2_rn(u0, make_float2(w4.x, w4.y), make_float2(c4.x, c4.y));
-            const float2 t1 = __ffma2_rn(u1, make_float2(w4.z, w4.w), make_float2(c4.z, c4.w));
-            acc[(c * 32 + j) / 2] = __ffma2_rn(t0, sa2, acc[(c * 32 + j) / 2]);
-            acc[(c * 32 + j) / 2 + 1] = __ffma2_rn(t1, sa2, acc[(c * 32 + j) / 2 + 1]);
+          for (int h = 0; h < 2; ++h) {
+            const uint32_t* rr = h ? r1 : r0;
+#pragma unroll
+            for (int j = 0; j < 32; j += 4) {
+              const int c = h * 32 + j;
+              const float4 w4 = lds128(scw + c);
+              // 256*P + bits(1.5 * 2^23) = bits of the float 1.5 * 2^23 + 256*P
+              const float2 u0 = make_float2(__uint_as_float(rr[j] + BIAS_BITS), __uint_as_float(rr[j + 1] + BIAS_BITS));
+              const float2 u1 =
+                  make_float2(__uint_as_float(rr[j + 2] + BIAS_BITS), __uint_as_float(rr[j + 3] + BIAS_BITS));
+              // 256*P*sA (the bias cancels inside one rounding), then acc += that * sW/256
+              const float2 t0 = __ffma2_rn(u0, sa2, d2);
+              const float2 t1 = __ffma2_rn(u1, sa2, d2);
+              acc[c / 2] = __ffma2_rn(t0, make_float2(w4.x, w4.y), acc[c / 2]);
+              acc[c / 2 + 1] = __ffma2_rn(t1, make_float2(w4.z, w4.w), acc[c / 2 + 1]);
+            }
           }
         } else {
           if (row_ok) {
+            const int g = w.g0 + gl;
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              const int n = n0 + wg * EPI_COLS + c * 32 + j;
-              if (n < p.N) p.P[((int64_t)m * p.N + n) * NG + g] = ((int32_t)rr[j]) / 256;
+            for (int j = 0; j < 64; ++j) {
+              const int n = w.n0 + wg * EPI_COLS + j;
+              const uint32_t v = j < 32 ? r0[j] : r1[j - 32];
+              if (n < p.N) p.P[((int64_t)m * p.N + n) * NG + g] = ((int32_t)v) / 256;
+            }
+          }
+        }
+        // the partials are in registers: release the accumulator for the group NACC ahead
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tempty[b]);
+      }
+      if (PARTIALS || !ok) continue;
+      if (row_ok) {
+        const int nb = w.n0 + wg * EPI_COLS;
+        if (p.Cacc) {
+          // split-K: add this K range's contribution (fp32 vector atomics)
+          float* crow = p.Cacc + (int64_t)m * p.N + nb;
+#pragma unroll
+          for (int j = 0; j < EPI_COLS; j += 4)
+            if (nb + j < p.N)
+              atomicAdd(reinterpret_cast<float4*>(crow + j),
+                        make_float4(acc[j / 2].x, acc[j / 2].y, acc[j / 2 + 1].x, acc[j / 2 + 1].y));
+        } else if (!p.c_bf16) {
+          float* crow = static_cast<float*>(p.C) + (int64_t)m * p.N + nb;
+#pragma unroll
+          for (int j = 0; j < EPI_COLS; j += 4)
+            if (nb + j < p.N)
+              *reinterpret_cast<float4*>(crow + j) =
+                  make_float4(acc[j / 2].x, acc[j / 2].y, acc[j / 2 + 1].x, acc[j / 2 + 1].y);
+        } else {
+          __nv_bfloat16* crow = static_cast<__nv_bfloat16*>(p.C) + (int64_t)m * p.N + nb;
+#pragma unroll
+          for (int j = 0; j < EPI_COLS; j += 8) {
+            if (nb + j < p.N) {
+              uint4 v;
+              __nv_bfloat162 h0 = __floats2bfloat162_rn(acc[j / 2].x, acc[j / 2].y);
+              __nv_bfloat162 h1 = __floats2bfloat162_rn(acc[j / 2 + 1].x, acc[j / 2 + 1].y);
+              __nv_bfloat162 h2 = __floats2bfloat162_rn(acc[j / 2 + 2].x, acc[j / 2 + 2].y);
+              __nv_bfloat162 h3 = __floats2bfloat162_rn(acc[j / 2 + 3].x, acc[j / 2 + 3].y);
+              v.x = *reinterpret_cast<uint32_t*>(&h0);
+              v.y = *reinterpret_cast<uint32_t*>(&h1);
+              v.z = *reinterpret_cast<uint32_t*>(&h2);
+              v.w = *reinterpret_cast<uint32_t*>(&h3);
+              *reinterpret_cast<uint4*>(crow + j) = v;
             }
           }
         }
       }
-      // the partials are in registers: release the accumulator for the group after next
-      tc_fence_before();
-      mbar_arrive(&tempty[b]);
-    }
-    if (!PARTIALS && ok && row_ok) {
-      const int nb = n0 + wg * EPI_COLS;
-      if (p.Cacc) {
-        // split-K: add this K range's contribution (fp32 vector atomics)
-        float* crow = p.Cacc + (int64_t)m * p.N + nb;
 #pragma unroll
-        for (int j = 0; j < EPI_COLS; j += 4)
-          if (nb + j < p.N)
-            atomicAdd(reinterpret_cast<float4*>(crow + j),
-                      make_float4(acc[j / 2].x, acc[j / 2].y, acc[j / 2 + 1].x, acc[j / 2 + 1].y));
-      } else if (!p.c_bf16) {
-        float* crow = static_cast<float*>(p.C) + (int64_t)m * p.N + nb;
-#pragma unroll
-        for (int j = 0; j < EPI_COLS; j += 4)
-          if (nb + j < p.N)
-            *reinterpret_cast<float4*>(crow + j) =
-                make_float4(acc[j / 2].x, acc[j / 2].y, acc[j / 2 + 1].x, acc[j / 2 + 1].y);
-      } else {
-        __nv_bfloat16* crow = static_cast<__nv_bfloat16*>(p.C) + (int64_t)m * p.N + nb;
-#pragma unroll
-        for (int j = 0; j < EPI_COLS; j += 8) {
-          if (nb + j < p.N) {
-            uint4 v;
-            __nv_bfloat162 h0 = __floats2bfloat162_rn(acc[j / 2].x, acc[j / 2].y);
-            __nv_bfloat162 h1 = __floats2bfloat162_rn(acc[j / 2 + 1].x, acc[j / 2 + 1].y);
-            __nv_bfloat162 h2 = __floats2bfloat162_rn(acc[j / 2 + 2].x, acc[j / 2 + 2].y);
-            __nv_bfloat162 h3 = __floats2bfloat162_rn(acc[j / 2 + 3].x, acc[j / 2 + 3].y);
-            v.x = *reinterpret_cast<uint32_t*>(&h0);
-            v.y = *reinterpret_cast<uint32_t*>(&h1);
-            v.z = *reinterpret_cast<uint32_t*>(&h2);
-            v.w = *reinterpret_cast<uint32_t*>(&h3);
-            *reinterpret_cast<uint4*>(crow + j) = v;
-          }
-        }
-      }
+      for (int j = 0; j < EPI_COLS / 2; ++j) acc[j] = make_float2(0.0f, 0.0f);
     }
   } else if (warp == LOADER_WARP) {
     // ======================= loader: the packed A and W tiles of one K-block -> packed stage
     // (two 2-D TMA boxes; rows beyond M / N and bytes beyond K/2 arrive as zeros)
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 40;");
-    for (int j = 0; j < NKB; ++j) {
-      const int kb = kb0 + j, ps = j % PSTAGES;
-      if (j >= PSTAGES && !warp_wait(&pempty[ps], ((j / PSTAGES) + 1) & 1, abort_flag, lane)) break;
-      if (lane == 0) {
-        uint8_t* pst = smem + OFF_PSTAGES + ps * PSTAGE_BYTES;
-        mbar_arrive_expect_tx(&pfull[ps], (uint32_t)PSTAGE_BYTES);
-        // x = kb * 64 bytes: a multiple of 16, as a tiled TMA requires of the inner coordinate
-        tma_load_2d(pst, &p.tmA, kb * PROW_BYTES, m0, &pfull[ps]);
-        tma_load_2d(pst + BM * PROW_BYTES, &p.tmW, kb * PROW_BYTES, n0, &pfull[ps]);
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 80;");
+    int it = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x) {
+      const Unit w = unit_of(p, u);
+      for (int j = 0; j < w.nkb; ++j, ++it) {
+        const int ps = it % PSTAGES;
+        if (it >= PSTAGES && !bar_wait(&pempty[ps], ((it / PSTAGES) + 1) & 1, abort_flag)) {
+          ok = false;
+          break;
+        }
+        if (lane == 0) {
+          uint8_t* pst = smem + OFF_PSTAGES + ps * PSTAGE_BYTES;
+          const int kb = w.kb0 + j;
+          mbar_arrive_expect_tx(&pfull[ps], (uint32_t)PSTAGE_BYTES);
+          // x = kb * 64 bytes: a multiple of 16, as a tiled TMA requires of the inner coordinate
+          tma_load_2d(pst, &p.tmA, kb * PROW_BYTES, w.m0, &pfull[ps]);
+          tma_load_2d(pst + BM * PROW_BYTES, &p.tmW, kb * PROW_BYTES, w.n0, &pfull[ps]);
+        }
+        __syncwarp();
       }
-      __syncwarp();
     }
   } else if (warp < MMA_WARP) {
     // ======================= unpackers: packed stage -> swizzled int8 stage
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 40;");
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 80;");
     const int ut = threadIdx.x - (LOADER_WARP + 1) * 32;   // 0..N_UNP-1
-    for (int j = 0; j < NKB; ++j) {
-      const int s = j % STAGES, ps = j % PSTAGES;
-      if (!warp_wait(&pfull[ps], (j / PSTAGES) & 1, abort_flag, lane)) break;
-      if (j >= STAGES && !warp_wait(&empty[s], ((j / STAGES) + 1) & 1, abort_flag, lane)) break;
-      const uint8_t* pst = smem + OFF_PSTAGES + ps * PSTAGE_BYTES;
-      uint8_t* st = smem + OFF_STAGES + s * STAGE_BYTES;
-#pragma unroll 4
-      for (int i = 0; i < UNP_CHUNKS; ++i) {
-        // chunk q: row r (A rows 0..BM-1, then W rows), 16-byte piece c of the row's 64 bytes
-        const int q = ut + N_UNP * i;
-        const int r = q >> 2, c = q & 3;
-        const uint4 w = *reinterpret_cast<const uint4*>(pst + q * 16);
-        uint8_t* tile = r < BM ? st : st + A_STAGE_BYTES;
-        const int rr = r < BM ? r : r - BM;
-        const uint4 lo = make_uint4((w.x << 4) & 0xF0F0F0F0u, (w.y << 4) & 0xF0F0F0F0u, (w.z << 4) & 0xF0F0F0F0u,
-                                    (w.w << 4) & 0xF0F0F0F0u);
-        const uint4 hi = make_uint4(w.x & 0xF0F0F0F0u, w.y & 0xF0F0F0F0u, w.z & 0xF0F0F0F0u, w.w & 0xF0F0F0F0u);
-        uint8_t* rowp = tile + (rr >> 3) * 1024 + (rr & 7) * 128;
-        *reinterpret_cast<uint4*>(rowp + (((2 * c) ^ (rr & 7)) << 4)) = lo;
-        *reinterpret_cast<uint4*>(rowp + (((2 * c + 1) ^ (rr & 7)) << 4)) = hi;
-      }
-      fence_proxy_async();
-      __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(&full[s]);
-        mbar_arrive(&pempty[ps]);
+    // chunk q = ut + N_UNP*i: row (q >> 2) of the A-then-W rows, 16-byte piece (q & 3) of its
+    // 64 packed bytes. N_UNP/4 is a multiple of 8, so the piece and the row's swizzle phase
+    // are the same for all of a thread's chunks, and the A and W int8 tiles are contiguous
+    // 128-byte rows (row r at byte 128*r of the stage).
+    const int c = ut & 3, r0 = ut >> 2, r7 = r0 & 7;
+    const int lo_off = ((2 * c) ^ r7) << 4, hi_off = ((2 * c + 1) ^ r7) << 4;
+    const bool tail = ut + N_UNP * (UNP_ITERS - 1) < N_CHUNKS;   // this thread has a last chunk
+    int it = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x) {
+      const Unit w = unit_of(p, u);
+      for (int j = 0; j < w.nkb; ++j, ++it) {
+        const int s = it % STAGES, ps = it % PSTAGES;
+        if (!bar_wait(&pfull[ps], (it / PSTAGES) & 1, abort_flag) ||
+            (it >= STAGES && !bar_wait(&empty[s], ((it / STAGES) + 1) & 1, abort_flag))) {
+          ok = false;
+          break;
+        }
+        const uint8_t* src = smem + OFF_PSTAGES + ps * PSTAGE_BYTES + ut * 16;
+        uint8_t* dst = smem + OFF_STAGES + s * STAGE_BYTES + r0 * 128;
+        // all loads first, then the stores: the shared-memory latency is paid once per stage
+        uint4 v[UNP_ITERS];
+#pragma unroll
+        for (int i = 0; i < UNP_ITERS; ++i)
+          if (i < UNP_ITERS - 1 || tail) v[i] = *reinterpret_cast<const uint4*>(src + i * N_UNP * 16);
+#pragma unroll
+        for (int i = 0; i < UNP_ITERS; ++i) {
+          if (i < UNP_ITERS - 1 || tail) {
+            const uint4 lo = make_uint4((v[i].x << 4) & 0xF0F0F0F0u, (v[i].y << 4) & 0xF0F0F0F0u,
+                                        (v[i].z << 4) & 0xF0F0F0F0u, (v[i].w << 4) & 0xF0F0F0F0u);
+            const uint4 hi = make_uint4(v[i].x & 0xF0F0F0F0u, v[i].y & 0xF0F0F0F0u, v[i].z & 0xF0F0F0F0u,
+                                        v[i].w & 0xF0F0F0F0u);
+            uint8_t* rowp = dst + i * (N_UNP / 4) * 128;
+            *reinterpret_cast<uint4*>(rowp + lo_off) = lo;
+            *reinterpret_cast<uint4*>(rowp + hi_off) = hi;
+          }
+        }
+        fence_proxy_async();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&full[s]);
+          mbar_arrive(&pempty[ps]);
+        }
       }
     }
   } else {
-    // ======================= MMA issue
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 40;");  // same value as the rest of its warpgroup
-    const bool leader = lane == 0;
+    // ======================= MMA issue (the whole warp runs the loop; elect.sync issues)
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 80;");  // same value as the rest of its warpgroup
+    // descriptors of stage 0; stage s and k-step k4 add (s * STAGE_BYTES + 32 * k4) >> 4 to the
+    // start-address field (no carry: shared addresses stay below 2^18)
     const uint32_t sbase = smem_u32(smem + OFF_STAGES);
-    for (int ks = 0; ks < KS; ++ks) {
-      // local k-step / K-block / group indices drive the rings; the split is group-aligned
-      const int kb = ks >> 2, k4 = ks & 3, s = kb % STAGES;
-      if (k4 == 0) {
-        if (!mbar_wait(&full[s], (kb / STAGES) & 1, abort_flag)) break;
+    const uint64_t dA0 = make_desc(sbase), dB0 = make_desc(sbase + A_STAGE_BYTES);
+    const int gsteps = p.G / 32;            // k-steps per group
+    int s = 0, sph = 0;                     // int8 stage and its phase parity
+    int b = 0, tph = 0;                     // accumulator and its phase parity
+    int kg = 0;                             // k-step within the current group
+    int nblk = 0;                           // K-blocks consumed
+    bool ok = true;
+    for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x) {
+      const Unit w = unit_of(p, u);         // K range group-aligned: kg == 0 here
+      for (int j = 0; j < w.nkb; ++j) {
+        if (!bar_wait(&full[s], sph, abort_flag)) {
+          ok = false;
+          break;
+        }
         tc_fence_after();
+        const int nk = min(4, w.ks - 4 * j);
+        const uint64_t so = (uint64_t)((s * STAGE_BYTES) >> 4);
+#pragma unroll
+        for (int k4 = 0; k4 < 4; ++k4) {
+          if (k4 < nk) {
+            if (kg == 0) {
+              if (!bar_wait(&tempty[b], tph, abort_flag)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+            }
+            umma_i8(tmem + b * BN, dA0 + so + 2 * k4, dB0 + so + 2 * k4, kg != 0 ? 1u : 0u);
+            if (++kg == gsteps) {
+              umma_commit(&tfull[b]);
+              kg = 0;
+              if (++b == NACC) {
+                b = 0;
+                tph ^= 1;
+              }
+            }
+          }
+        }
+        if (!ok) break;
+        umma_commit(&empty[s]);
+        ++nblk;
+        if (++s == STAGES) {
+          s = 0;
+          sph ^= 1;
+        }
       }
-      const int gl = (ks * 32) / p.G;
-      const bool first = (ks * 32) % p.G == 0;
-      const bool last = ((ks + 1) * 32) % p.G == 0;
-      const int b = gl & 1;
-      if (first) {
-        if (!mbar_wait(&tempty[b], (gl >> 1) & 1, abort_flag)) break;
-        tc_fence_after();
-      }
-      if (leader) {
-        const uint32_t a_addr = sbase + s * STAGE_BYTES + k4 * 32;
-        const uint32_t b_addr = sbase + s * STAGE_BYTES + A_STAGE_BYTES + k4 * 32;
-        umma_i8(tmem + b * BN, make_desc(a_addr), make_desc(b_addr), first ? 0u : 1u);
-        if (last) umma_commit(&tfull[b]);
-        if (k4 == 3 || ks == KS - 1) umma_commit(&empty[s]);
-      }
-      __syncwarp();
     }
     // the last stage-release commit must have landed before the CTA (and its smem) goes away
-    if (!*abort_flag && NKB > 0) {
-      const int kl = NKB - 1;
-      mbar_wait(&empty[kl % STAGES], (kl / STAGES) & 1, abort_flag);
+    if (ok && nblk > 0) {
+      const int last = s == 0 ? STAGES - 1 : s - 1;
+      bar_wait(&empty[last], s == 0 ? sph ^ 1 : sph, abort_flag);
     }
   }
 
@@ -777,22 +919,29 @@ rot_status w4a4_launch(const uint8_t* Aq, const uint16_t* As, const uint8_t* Wq,
   p.K = (int)K;
   p.G = G;
   p.c_bf16 = c_dtype == ROT_BF16;
-  const int64_t gx = (N + BN - 1) / BN, gy = (M + BM - 1) / BM;
+  const int64_t tn = (N + BN - 1) / BN, tm = (M + BM - 1) / BM;
   const int nkb = (int)((K + KB - 1) / KB);
-  const int unit = G > KB ? G / KB : 1;            // K-blocks per group (split granularity)
-  const int splits = partials ? 1 : split_count(gx * gy, nkb / unit, sm_count());
+  // split granularity: the fewest whole K-blocks that hold whole groups, lcm(G, KB) / KB
+  int unit = 1;
+  while ((unit * KB) % G != 0) ++unit;
+  const int sms = sm_count();
+  const int splits = partials ? 1 : split_count(tn * tm, nkb / unit, sms);
   p.kb_per_split = ((nkb / unit + splits - 1) / splits) * unit;
-  const int zs = (nkb + p.kb_per_split - 1) / p.kb_per_split;
+  p.splits = (nkb + p.kb_per_split - 1) / p.kb_per_split;
+  p.tiles_m = (int)tm;
+  if (tn * tm * p.splits > (1ll << 30)) return set_error(ROT_EUNSUPPORTED, "w4a4_linear: too many tiles");
+  p.units = (int)(tn * tm * p.splits);
   p.Cacc = nullptr;
-  if (zs > 1) {
+  if (p.splits > 1) {
     rot_status st = acc_target(&p.Cacc);
     if (st) return st;
   }
-  dim3 grid((unsigned)gx, (unsigned)gy, (unsigned)zs);
+  // persistent: one CTA per SM (the shared-memory footprint admits no second one)
+  const unsigned grid = (unsigned)std::min<int64_t>(p.units, sms);
   if (partials) w4a4_kernel<true><<<grid, THREADS, SMEM_BYTES, s>>>(p);
   else w4a4_kernel<false><<<grid, THREADS, SMEM_BYTES, s>>>(p);
   ROT_CUDA_TRY(cudaGetLastError());
-  return zs > 1 ? finish_acc(p.Cacc) : ROT_OK;
+  return p.splits > 1 ? finish_acc(p.Cacc) : ROT_OK;
 }
 
 rot_status w4a4_noalloc_scratch(float** out) {
