@@ -827,10 +827,11 @@ rot_status w4a4_launch(const uint8_t* Aq, const uint16_t* As, const uint8_t* Wq,
     return ROT_OK;
   };
   if (!partials && M <= 16 * DEC_MAXMT && G % 128 == 0) {
-    // decode-sized M: weight-streaming kernel, K split until about 16 warps per SM are busy
+    // decode-sized M: weight-streaming kernel, K split until about 32 warps per SM are busy
+    // (more bytes in flight: 16 warps measured 9.7 us, 32 warps 8.8 us for q_proj at M = 16)
     const int64_t ntiles = N / 8;
     const int NG = (int)(K / G);
-    int64_t want = ((int64_t)sm_count() * 16 + ntiles - 1) / ntiles;
+    int64_t want = ((int64_t)sm_count() * 32 + ntiles - 1) / ntiles;
     const int splits0 = (int)std::max<int64_t>(1, std::min<int64_t>(NG, want));
     const int gps = (NG + splits0 - 1) / splits0;
     const int splits = (NG + gps - 1) / gps;
