@@ -24,8 +24,8 @@
 // warpgroups 2-3 (loader, unpackers, MMA warp) shrink to 80: 256*176 + 256*80 = 512*128.
 //   warps 0-7   epilogue: warp w reads TMEM lanes 32*(w%4).. and columns 64*(w/4)..+63 of
 //               a group's accumulator (two 32-column loads in flight), scales them and
-//               accumulates in fp32 registers (packed f32x2 FMAs); it also stages the
-//               group scales two groups ahead into a ring of shared-memory slots;
+//               accumulates in fp32 registers (packed f32x2 FMAs); it stages its own
+//               columns' scales in a private shared-memory buffer;
 //   warp 8      loader;   warps 9-14 unpackers;   warp 15 TMEM allocation and MMA issue.
 // Group scaling: the epilogue adds the bit pattern of 1.5 * 2^23 to the int32 partial 256*P
 // (one integer add): the sum is the bit pattern of the fp32 value 1.5 * 2^23 + 256*P, so
@@ -54,9 +54,6 @@ constexpr int KB = 128;                  // K elements per stage
 constexpr int STAGES = 3;                // unpacked int8 stages
 constexpr int PSTAGES = 6;               // packed stages
 constexpr int NACC = 4;                  // TMEM accumulators (groups in flight)
-constexpr int NSLOT = 8;                 // scale slots
-constexpr int SLOT_AHEAD = 2;            // groups between staging a slot and reading it
-static_assert(NSLOT > SLOT_AHEAD + NACC, "a slot is rewritten only after every epilogue warp has left it");
 constexpr int A_STAGE_BYTES = BM * KB;   // unpacked int8
 constexpr int B_STAGE_BYTES = BN * KB;
 constexpr int STAGE_BYTES = A_STAGE_BYTES + B_STAGE_BYTES;
@@ -87,10 +84,9 @@ constexpr unsigned long long WAIT_NS = 2000000000ull;
 // smem layout (offsets from a 1024-byte aligned base)
 constexpr int OFF_STAGES = 0;
 constexpr int OFF_PSTAGES = STAGES * STAGE_BYTES;
-constexpr int OFF_SLOTS = OFF_PSTAGES + PSTAGES * PSTAGE_BYTES;  // [NSLOT] {sW/256 [BN], sA [BM]} fp32
-constexpr int SLOT_FLOATS = BN + BM;
-constexpr int OFF_BARS = OFF_SLOTS + NSLOT * SLOT_FLOATS * 4;
-constexpr int N_BARS = 2 * STAGES + 2 * PSTAGES + 2 * NACC + NSLOT;
+constexpr int OFF_SLOTS = OFF_PSTAGES + PSTAGES * PSTAGE_BYTES;  // per epilogue warp: sW/256 of its columns
+constexpr int OFF_BARS = OFF_SLOTS + N_EPI_WARPS * EPI_COLS * 4;
+constexpr int N_BARS = 2 * STAGES + 2 * PSTAGES + 2 * NACC;
 constexpr int OFF_TMEM = OFF_BARS + N_BARS * 8;
 constexpr int SMEM_BYTES = OFF_TMEM + 16 + 1024;          // + alignment slack
 static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
@@ -293,7 +289,6 @@ __global__ void __launch_bounds__(THREADS, 1) w4a4_kernel(const __grid_constant_
   uint64_t* pempty = pfull + PSTAGES;    // [PSTAGES] unpackers -> loader
   uint64_t* tfull = pempty + PSTAGES;    // [NACC]    MMA commit -> epilogue
   uint64_t* tempty = tfull + NACC;       // [NACC]    epilogue warps -> MMA
-  uint64_t* sfull = tempty + NACC;       // [NSLOT]   epilogue warps (staging) -> epilogue warps
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_TMEM);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + OFF_TMEM + 8);
   float* slots = reinterpret_cast<float*>(smem + OFF_SLOTS);
@@ -315,7 +310,6 @@ __global__ void __launch_bounds__(THREADS, 1) w4a4_kernel(const __grid_constant_
       mbar_init(&tfull[b], 1);
       mbar_init(&tempty[b], N_EPI_WARPS);
     }
-    for (int s = 0; s < NSLOT; ++s) mbar_init(&sfull[s], N_EPI_WARPS);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -341,10 +335,13 @@ __global__ void __launch_bounds__(THREADS, 1) w4a4_kernel(const __grid_constant_
     if (lane == 0)
       for (int b = 0; b < NACC; ++b) mbar_arrive(&tempty[b]);
 
-    // Scale staging runs SLOT_AHEAD groups ahead of the accumulation. Warps 0-3 stage sW/256
-    // of column threadIdx.x, warps 4-7 sA of their row. The raw binary16 values are loaded
-    // LQ groups before they are staged, into a ring of registers that a switch on the ring
-    // index addresses statically (no register is read while its load is still in flight).
+    // Group scales: each warp stages sW/256 of its own 64 columns in a private shared-memory
+    // buffer (lane l: columns l and l + 32), ordered by __syncwarp alone, and keeps sA of its
+    // row in a register. The raw binary16 values are loaded two groups ahead into a two-entry
+    // register ring addressed statically by the parity of the group, from addresses clamped
+    // into the matrix (rows >= M and columns >= N are never stored), so every load is
+    // unconditional and no register is read while its load is in flight.
+    float* wsc = slots + warp * EPI_COLS;
     int su = blockIdx.x;                      // load cursor: unit and group within it
     int sg = 0;
     int s_g0 = 0, s_ngl = 0, s_m0 = 0, s_n0 = 0;
@@ -357,14 +354,13 @@ __global__ void __launch_bounds__(THREADS, 1) w4a4_kernel(const __grid_constant_
         s_n0 = w.n0;
       }
     };
-    // address of the raw scale at the cursor: clamped into the matrix (rows >= M and columns
-    // >= N are never stored, so their scale is irrelevant) and a valid dummy past the end, so
-    // that every load is unconditional and lands straight in its ring register
-    auto cursor_addr = [&]() -> const uint16_t* {
+    auto cursor_w = [&](int half) -> const uint16_t* {
       if (su >= p.units) return p.Ws;
-      const int g = s_g0 + sg;
-      if (wg == 0) return p.Ws + (int64_t)min(s_n0 + (int)threadIdx.x, p.N - 1) * NG + g;
-      return p.As + (int64_t)min(s_m0 + row, p.M - 1) * NG + g;
+      return p.Ws + (int64_t)min(s_n0 + wg * EPI_COLS + half * 32 + lane, p.N - 1) * NG + s_g0 + sg;
+    };
+    auto cursor_a = [&]() -> const uint16_t* {
+      if (su >= p.units) return p.Ws;
+      return p.As + (int64_t)min(s_m0 + row, p.M - 1) * NG + s_g0 + sg;
     };
     auto cursor_step = [&]() {
       if (su < p.units && ++sg == s_ngl) {
@@ -373,31 +369,17 @@ __global__ void __launch_bounds__(THREADS, 1) w4a4_kernel(const __grid_constant_
         cursor_unit();
       }
     };
-    auto cursor_next = [&]() -> uint16_t {
-      const uint16_t v = __ldg(cursor_addr());
-      cursor_step();
-      return v;
-    };
-    int total = 0;                            // groups this CTA accumulates
-    if (!PARTIALS)
-      for (int u = blockIdx.x; u < p.units; u += gridDim.x) total += unit_of(p, u).ngl;
-    auto stage = [&](int gidx, uint16_t raw) {
-      if (gidx >= total) return;
-      const float v = __half2float(__ushort_as_half(raw));
-      float* sl = slots + (gidx % NSLOT) * SLOT_FLOATS;
-      if (wg == 0) sl[threadIdx.x] = v * (1.0f / 256.0f);
-      else sl[BN + row] = v;
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&sfull[gidx % NSLOT]);
-    };
-    uint16_t sq0 = 0, sq1 = 0, sq2 = 0, sq3 = 0;   // groups gc+SLOT_AHEAD+{0..3} (mod 4 ring)
+    uint16_t q0w0 = 0, q0w1 = 0, q0a = 0, q1w0 = 0, q1w1 = 0, q1a = 0;   // groups gc (+1), by parity
     if (!PARTIALS) {
       cursor_unit();
-      for (int i = 0; i < SLOT_AHEAD; ++i) stage(i, cursor_next());
-      sq0 = cursor_next();
-      sq1 = cursor_next();
-      sq2 = cursor_next();
-      sq3 = cursor_next();
+      q0w0 = __ldg(cursor_w(0));
+      q0w1 = __ldg(cursor_w(1));
+      q0a = __ldg(cursor_a());
+      cursor_step();
+      q1w0 = __ldg(cursor_w(0));
+      q1w1 = __ldg(cursor_w(1));
+      q1a = __ldg(cursor_a());
+      cursor_step();
     }
 
     float2 acc[EPI_COLS / 2];
@@ -410,16 +392,23 @@ __global__ void __launch_bounds__(THREADS, 1) w4a4_kernel(const __grid_constant_
       const int m = w.m0 + row;
       const bool row_ok = m < p.M;
       for (int gl = 0; gl < w.ngl; ++gl, ++gc) {
+        float sa = 0.0f;
         if (!PARTIALS) {
-          const uint16_t* sa_next = cursor_addr();
+          const uint16_t *nw0 = cursor_w(0), *nw1 = cursor_w(1), *na = cursor_a();
           cursor_step();
-          switch (gc & 3) {
-            case 0: stage(gc + SLOT_AHEAD, sq0); sq0 = __ldg(sa_next); break;
-            case 1: stage(gc + SLOT_AHEAD, sq1); sq1 = __ldg(sa_next); break;
-            case 2: stage(gc + SLOT_AHEAD, sq2); sq2 = __ldg(sa_next); break;
-            default: stage(gc + SLOT_AHEAD, sq3); sq3 = __ldg(sa_next); break;
+          uint16_t rw0, rw1, ra;
+          if (gc & 1) {
+            rw0 = q1w0; rw1 = q1w1; ra = q1a;
+            q1w0 = __ldg(nw0); q1w1 = __ldg(nw1); q1a = __ldg(na);
+          } else {
+            rw0 = q0w0; rw1 = q0w1; ra = q0a;
+            q0w0 = __ldg(nw0); q0w1 = __ldg(nw1); q0a = __ldg(na);
           }
-          ok = ok && bar_wait(&sfull[gc % NSLOT], (gc / NSLOT) & 1, abort_flag);
+          __syncwarp();                 // every lane has read the previous group's column scales
+          wsc[lane] = __half2float(__ushort_as_half(rw0)) * (1.0f / 256.0f);
+          wsc[lane + 32] = __half2float(__ushort_as_half(rw1)) * (1.0f / 256.0f);
+          sa = __half2float(__ushort_as_half(ra));
+          __syncwarp();
         }
         const int b = gc % NACC;
         ok = ok && bar_wait(&tfull[b], (gc / NACC) & 1, abort_flag);
@@ -430,11 +419,9 @@ __global__ void __launch_bounds__(THREADS, 1) w4a4_kernel(const __grid_constant_
         tmem_ld32(lane_addr + b * BN + 32, r1);
         tmem_wait_ld();
         if constexpr (!PARTIALS) {
-          const float* sl = slots + (gc % NSLOT) * SLOT_FLOATS;
-          const float sa = sl[BN + row];
           const float2 sa2 = make_float2(sa, sa);
           const float2 d2 = make_float2(-BIAS_F * sa, -BIAS_F * sa);   // exact: 3 * 2^22 * binary16
-          const float* scw = sl + wg * EPI_COLS;
+          const float* scw = wsc;
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
             const uint32_t* rr = h ? r1 : r0;
