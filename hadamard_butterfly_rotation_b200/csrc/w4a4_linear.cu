@@ -343,30 +343,32 @@ __global__ void __launch_bounds__(THREADS, 1) w4a4_kernel(const __grid_constant_
     // unconditional and no register is read while its load is in flight.
     float* wsc = slots + warp * EPI_COLS;
     int su = blockIdx.x;                      // load cursor: unit and group within it
-    int sg = 0;
-    int s_g0 = 0, s_ngl = 0, s_m0 = 0, s_n0 = 0;
+    int sg = 0, s_ngl = 0;
+    const uint16_t *cw0 = p.Ws, *cw1 = p.Ws, *ca = p.Ws;   // the cursor group's scales (dummy past the end)
     auto cursor_unit = [&]() {
       if (su < p.units) {
         const Unit w = unit_of(p, su);
-        s_g0 = w.g0;
         s_ngl = w.ngl;
-        s_m0 = w.m0;
-        s_n0 = w.n0;
+        cw0 = p.Ws + (int64_t)min(w.n0 + wg * EPI_COLS + lane, p.N - 1) * NG + w.g0;
+        cw1 = p.Ws + (int64_t)min(w.n0 + wg * EPI_COLS + 32 + lane, p.N - 1) * NG + w.g0;
+        ca = p.As + (int64_t)min(w.m0 + row, p.M - 1) * NG + w.g0;
+      } else {
+        cw0 = cw1 = ca = p.Ws;
       }
     };
-    auto cursor_w = [&](int half) -> const uint16_t* {
-      if (su >= p.units) return p.Ws;
-      return p.Ws + (int64_t)min(s_n0 + wg * EPI_COLS + half * 32 + lane, p.N - 1) * NG + s_g0 + sg;
-    };
-    auto cursor_a = [&]() -> const uint16_t* {
-      if (su >= p.units) return p.Ws;
-      return p.As + (int64_t)min(s_m0 + row, p.M - 1) * NG + s_g0 + sg;
-    };
+    auto cursor_w = [&](int half) -> const uint16_t* { return half ? cw1 : cw0; };
+    auto cursor_a = [&]() -> const uint16_t* { return ca; };
     auto cursor_step = [&]() {
-      if (su < p.units && ++sg == s_ngl) {
-        sg = 0;
-        su += gridDim.x;
-        cursor_unit();
+      if (su < p.units) {
+        if (++sg == s_ngl) {
+          sg = 0;
+          su += gridDim.x;
+          cursor_unit();
+        } else {
+          ++cw0;
+          ++cw1;
+          ++ca;
+        }
       }
     };
     uint16_t q0w0 = 0, q0w1 = 0, q0a = 0, q1w0 = 0, q1w1 = 0, q1a = 0;   // groups gc (+1), by parity
