@@ -16,9 +16,9 @@
 // the CTAs running at the same time share weight tiles in L2. Per K-block of 128: the
 // loader warp brings the packed A and W tiles (two 2-D TMA boxes) into a 6-deep packed
 // ring; 6 unpacker warps expand them into a 3-deep ring of swizzled K-major int8 tiles;
-// one thread issues 4 UMMAs (M = N = 128, K = 32) per K-block into one of four 128-column
-// TMEM accumulators, one per group in flight, so the tensor pipe can run three groups
-// ahead of the epilogue.
+// the MMA warp, converged, issues 4 UMMAs (M = N = 128, K = 32) per K-block under an
+// elect.sync predicate into one of four 128-column TMEM accumulators, one per group in
+// flight, so the tensor pipe can run three groups ahead of the epilogue.
 // Warp roles (512 threads, launched with 128 registers each). setmaxnreg acts on whole
 // warpgroups, so roles are aligned to them: warpgroups 0-1 (epilogue) grow to 176 registers,
 // warpgroups 2-3 (loader, unpackers, MMA warp) shrink to 80: 256*176 + 256*80 = 512*128.

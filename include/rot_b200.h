@@ -125,8 +125,9 @@ rot_status rot_dequant(const uint8_t* codes, const uint16_t* scales, int64_t M, 
  * C:  [M, N] fp32 (c_dtype = ROT_F32) or bf16 (ROT_BF16), row-major, ldc = N.
  * Requires K % G == 0, G % 32 == 0, K % 64 == 0, N % 16 == 0; M >= 0 arbitrary.
  * Decode-sized M (M <= 64 with G % 128 == 0) runs a weight-streaming kernel (mma.sync
- * int8 per 8 weight rows); other shapes whose 128 x 256 output tiles leave most SMs idle
- * split K across CTAs of the tile kernel. When K is split, the partial results are added
+ * int8 per 8 weight rows); other shapes run a persistent tcgen05 kernel over 128 x 128
+ * output tiles, and shapes whose tiles leave most SMs idle split K into ranges aligned to
+ * lcm(G, 128). When K is split, the partial results are added
  * with fp32 atomics: C is zeroed on the stream first (fp32 output), or, for bf16 output, a
  * stream-ordered temporary of M * N floats is allocated (cudaMallocAsync), accumulated,
  * converted into C and freed on the stream. The summation order then varies between runs
