@@ -41,6 +41,7 @@ _lib.rot_dequant.argtypes = [_vp, _vp, _i64, _vp, _int, _int, _int, _vp, _vp]
 _lib.w4a4_linear.argtypes = [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _int, _vp, _int, _vp]
 _lib.w4a4_linear_noalloc.argtypes = [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _int, _vp, _int, _vp]
 _lib.w4a4_group_partials.argtypes = [_vp, _vp, _i64, _i64, _i64, _int, _vp, _vp]
+_lib.w4a4_tile_plan.argtypes = [_i64, _i64, _i64, _int, _int, _int, C.POINTER(_i64)]
 _lib.rot_harp_givens_blocks.argtypes = [C.POINTER(C.c_double), _i64, C.POINTER(C.c_float)]
 _lib.rot_harp_qr_block.argtypes = [C.POINTER(C.c_double), _int, C.POINTER(C.c_float)]
 _lib.rot_check_device.argtypes = []
@@ -241,6 +242,14 @@ def w4a4_group_partials(Aq, Wq, G: int, *, out=None, stream=None):
         out = torch.empty((M, N, K // G), dtype=torch.int32, device=Wq.device)
     _check(_lib.w4a4_group_partials(_ptr(Aq), _ptr(Wq), M, N, K, G, _ptr(out), _stream(stream)))
     return out
+
+
+def w4a4_tile_plan(M: int, N: int, K: int, G: int, sms: int, partials: bool = False) -> dict:
+    """Host: the tile kernel's work list for a shape (see ``include/rot_b200.h``)."""
+    out = (_i64 * 6)()
+    _check(_lib.w4a4_tile_plan(M, N, K, G, sms, int(partials), out))
+    keys = ("tiles_m", "tiles_n", "splits", "kb_per_split", "units", "grid")
+    return {k: int(v) for k, v in zip(keys, out)}
 
 
 def harp_givens_blocks(theta) -> np.ndarray:

@@ -122,6 +122,23 @@ extern "C" rot_status w4a4_linear_noalloc(const uint8_t* Aq, const uint16_t* As,
                      W4A4_NOALLOC_SCRATCH_FLOATS);
 }
 
+extern "C" rot_status w4a4_tile_plan(int64_t M, int64_t N, int64_t K, int G, int sms, int partials,
+                                     int64_t* out) {
+  if (!out) return set_error(ROT_EINVAL, "w4a4_tile_plan: out must be non-NULL");
+  if (K % 64 != 0 || N % 16 != 0)
+    return set_error(ROT_EINVAL, "w4a4_tile_plan: need K % 64 == 0 and N % 16 == 0");
+  W4A4TilePlan tp;
+  rot_status st = w4a4_tile_plan_compute(M, N, K, G, sms, partials != 0, &tp);
+  if (st) return st;
+  out[0] = tp.tiles_m;
+  out[1] = tp.tiles_n;
+  out[2] = tp.splits;
+  out[3] = tp.kb_per_split;
+  out[4] = tp.units;
+  out[5] = tp.grid;
+  return ROT_OK;
+}
+
 extern "C" rot_status w4a4_group_partials(const uint8_t* Aq, const uint8_t* Wq, int64_t M, int64_t N,
                                           int64_t K, int G, int32_t* P, void* stream) {
   rot_status st = check_w4a4(Aq, Wq, M, N, K, G, "w4a4_group_partials");

@@ -77,6 +77,12 @@ rot_status w4a4_launch(const uint8_t* Aq, const uint16_t* As, const uint8_t* Wq,
                        int c_dtype, int32_t* partials, cudaStream_t s, float* scratch = nullptr,
                        int64_t scratch_floats = 0);
 rot_status w4a4_noalloc_scratch(float** out);
+struct W4A4TilePlan {
+  int64_t tiles_m, tiles_n, units, grid;
+  int splits, kb_per_split;
+};
+rot_status w4a4_tile_plan_compute(int64_t M, int64_t N, int64_t K, int G, int sms, bool partials,
+                                  W4A4TilePlan* out);
 
 // ---------------------------------------------------------------- device helpers
 #ifdef __CUDACC__

@@ -783,6 +783,31 @@ __global__ void f32_to_bf16_kernel(const float* __restrict__ src, __nv_bfloat16*
   }
 }
 
+// Work list of the tile kernel: 128 x 128 output tiles, times K splits when the tiles alone
+// would leave more than half of the SMs idle. A split covers a whole number of lcm(G, 128)
+// K-ranges, so it starts and ends on both a K-block and a group boundary; every split is
+// non-empty; one persistent CTA per SM, at most one per unit.
+rot_status w4a4_tile_plan_compute(int64_t M, int64_t N, int64_t K, int G, int sms, bool partials,
+                                  W4A4TilePlan* out) {
+  if (M <= 0 || N <= 0 || K <= 0 || G <= 0 || G > 256 || K % G != 0 || G % 32 != 0 || sms <= 0)
+    return set_error(ROT_EINVAL, "w4a4 tile plan: need M, N, K, sms > 0, 0 < G <= 256, G % 32 == 0, K % G == 0");
+  W4A4TilePlan tp;
+  tp.tiles_n = (N + BN - 1) / BN;
+  tp.tiles_m = (M + BM - 1) / BM;
+  const int64_t nkb = (K + KB - 1) / KB;
+  int unit = 1;                                    // K-blocks per lcm(G, KB) range
+  while ((unit * KB) % G != 0) ++unit;
+  const int64_t ranges = (nkb + unit - 1) / unit;  // lcm ranges (the last one may be partial)
+  const int64_t want = partials ? 1 : split_count(tp.tiles_n * tp.tiles_m, (int)std::min<int64_t>(ranges, 1 << 20), sms);
+  tp.kb_per_split = (int)(((ranges + want - 1) / want) * unit);
+  tp.splits = (int)((nkb + tp.kb_per_split - 1) / tp.kb_per_split);
+  if (tp.tiles_n * tp.tiles_m * tp.splits > (1ll << 30)) return set_error(ROT_EUNSUPPORTED, "w4a4_linear: too many tiles");
+  tp.units = tp.tiles_n * tp.tiles_m * tp.splits;
+  tp.grid = std::min<int64_t>(tp.units, sms);
+  *out = tp;
+  return ROT_OK;
+}
+
 rot_status w4a4_launch(const uint8_t* Aq, const uint16_t* As, const uint8_t* Wq, const uint16_t* Ws, int64_t M,
                        int64_t N, int64_t K, int G, void* C, int c_dtype, int32_t* partials, cudaStream_t s,
                        float* scratch, int64_t scratch_floats) {
@@ -909,25 +934,22 @@ rot_status w4a4_launch(const uint8_t* Aq, const uint16_t* As, const uint8_t* Wq,
   p.K = (int)K;
   p.G = G;
   p.c_bf16 = c_dtype == ROT_BF16;
-  const int64_t tn = (N + BN - 1) / BN, tm = (M + BM - 1) / BM;
-  const int nkb = (int)((K + KB - 1) / KB);
-  // split granularity: the fewest whole K-blocks that hold whole groups, lcm(G, KB) / KB
-  int unit = 1;
-  while ((unit * KB) % G != 0) ++unit;
-  const int sms = sm_count();
-  const int splits = partials ? 1 : split_count(tn * tm, nkb / unit, sms);
-  p.kb_per_split = ((nkb / unit + splits - 1) / splits) * unit;
-  p.splits = (nkb + p.kb_per_split - 1) / p.kb_per_split;
-  p.tiles_m = (int)tm;
-  if (tn * tm * p.splits > (1ll << 30)) return set_error(ROT_EUNSUPPORTED, "w4a4_linear: too many tiles");
-  p.units = (int)(tn * tm * p.splits);
+  W4A4TilePlan tp;
+  {
+    rot_status st = w4a4_tile_plan_compute(M, N, K, G, sm_count(), partials != nullptr, &tp);
+    if (st) return st;
+  }
+  p.kb_per_split = tp.kb_per_split;
+  p.splits = tp.splits;
+  p.tiles_m = (int)tp.tiles_m;
+  p.units = (int)tp.units;
   p.Cacc = nullptr;
   if (p.splits > 1) {
     rot_status st = acc_target(&p.Cacc);
     if (st) return st;
   }
   // persistent: one CTA per SM (the shared-memory footprint admits no second one)
-  const unsigned grid = (unsigned)std::min<int64_t>(p.units, sms);
+  const unsigned grid = (unsigned)tp.grid;
   if (partials) w4a4_kernel<true><<<grid, THREADS, SMEM_BYTES, s>>>(p);
   else w4a4_kernel<false><<<grid, THREADS, SMEM_BYTES, s>>>(p);
   ROT_CUDA_TRY(cudaGetLastError());

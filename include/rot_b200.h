@@ -147,6 +147,15 @@ rot_status w4a4_linear_noalloc(const uint8_t* Aq, const uint16_t* As, const uint
                                const uint16_t* Ws, int64_t M, int64_t N, int64_t K, int G, void* C,
                                int c_dtype, void* stream);
 
+/* Host only (no device work): the work list the tcgen05 tile kernel of w4a4_linear uses for a
+ * shape (M > 64 or G % 128 != 0), given the device's SM count. out: int64 [6] =
+ * {tiles_m, tiles_n, splits, kb_per_split, units, grid}: 128 x 128 output tiles; K split into
+ * `splits` ranges of kb_per_split K-blocks of 128 (a multiple of lcm(G, 128) / 128, so every range
+ * starts and ends on a K-block and a group boundary; none is empty) when the tiles alone leave
+ * more than half of the SMs idle and partials == 0; units = tiles * splits; grid = min(units,
+ * sms) persistent CTAs. ROT_EINVAL for the shapes w4a4_linear rejects, M <= 0 or sms <= 0. */
+rot_status w4a4_tile_plan(int64_t M, int64_t N, int64_t K, int G, int sms, int partials, int64_t* out);
+
 /* The exact int32 group partial sums P[m, n, g] of the same contraction, written to
  * P: int32 [M, N, K/G]. Same constraints as w4a4_linear. For checking only. */
 rot_status w4a4_group_partials(const uint8_t* Aq, const uint8_t* Wq, int64_t M, int64_t N,

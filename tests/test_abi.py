@@ -82,3 +82,62 @@ def test_plan_create_rejects_bad_schedules(lib):
     rad2 = (C.c_int * 1)(2)
     st = lib._lib.rot_plan_create(C.byref(h), 2, 1, rad2, None, None, None, s)
     assert st == lib.ROT_EINVAL and "signs" in lib.last_error()
+
+
+def _w4a4_plan_cases():
+    cases = []
+    for M in (1, 65, 129, 2048, 5000):
+        for N in (16, 272, 4096, 11008):
+            for G in (32, 64, 96, 128, 160, 192, 224, 256):
+                for K in (192, 448, 1344, 4096, 11008):
+                    if K % G == 0 and K % 64 == 0:
+                        cases.append((M, N, K, G))
+    return cases
+
+
+def test_w4a4_tile_plan_invariants(lib):
+    """Host planner of the tcgen05 W4A4 kernel: every K split starts and ends on a K-block and a
+    group boundary, none is empty, the splits cover K, and K is split only when the output tiles
+    leave more than half of the SMs idle."""
+    from math import gcd
+    cases = _w4a4_plan_cases()
+    assert len(cases) > 100
+    for sms in (1, 20, 148):
+        for M, N, K, G in cases:
+            pl = lib.w4a4_tile_plan(M, N, K, G, sms)
+            unit = (G * 128 // gcd(G, 128)) // 128
+            nkb = -(-K // 128)
+            tiles = -(-M // 128) * -(-N // 128)
+            assert (pl["tiles_m"], pl["tiles_n"]) == (-(-M // 128), -(-N // 128))
+            kb = pl["kb_per_split"]
+            assert kb >= 1 and kb % unit == 0, (M, N, K, G, sms, pl)
+            assert pl["splits"] == -(-nkb // kb)
+            assert (pl["splits"] - 1) * kb < nkb                       # no empty split
+            assert all((s * kb * 128) % G == 0 for s in range(pl["splits"]))
+            assert pl["units"] == tiles * pl["splits"]
+            assert pl["grid"] == min(pl["units"], sms)
+            if 2 * tiles > sms:
+                assert pl["splits"] == 1
+            if pl["splits"] > 1:
+                assert pl["splits"] * tiles <= max(sms, tiles)
+
+
+def test_w4a4_tile_plan_k_below_one_lcm_range(lib):
+    """K smaller than lcm(G, 128): one split of one whole lcm range (a floor division here once
+    gave zero K-blocks per split)."""
+    for M, N, K, G in ((5, 640, 192, 192), (7, 96, 448, 224), (3, 48, 192, 96)):
+        pl = lib.w4a4_tile_plan(M, N, K, G, 148)
+        assert pl["splits"] == 1 and pl["kb_per_split"] >= -(-K // 128)
+
+
+def test_w4a4_tile_plan_partials_never_split(lib):
+    pl = lib.w4a4_tile_plan(16, 256, 4096, 128, 148, partials=True)
+    assert pl["splits"] == 1 and pl["units"] == 2
+
+
+def test_w4a4_tile_plan_rejects_bad_shapes(lib):
+    for args in ((0, 256, 4096, 128, 148), (16, 256, 4096, 96, 148), (16, 256, 4096, 512, 148),
+                 (16, 250, 4096, 128, 148), (16, 256, 4096, 128, 0), (16, 256, 4000, 32, 148)):
+        with pytest.raises(lib.RotError) as e:
+            lib.w4a4_tile_plan(*args)
+        assert e.value.status == lib.ROT_EINVAL

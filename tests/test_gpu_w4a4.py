@@ -29,7 +29,7 @@ def _dev(a):
 @pytest.mark.parametrize("M,N,K,G", [(1, 16, 128, 32), (3, 48, 256, 64), (128, 256, 512, 128),
                                      (129, 272, 384, 128), (64, 512, 4096, 128), (200, 176, 192, 32),
                                      (16, 256, 1024, 256), (300, 784, 640, 64), (5, 640, 1152, 96),
-                                     (33, 144, 640, 160)])
+                                     (33, 144, 640, 160), (5, 640, 192, 192)])
 def test_group_partials_exact(lib, M, N, K, G):
     qa, pa, sa = _codes(M + K, M, K, G)
     qw, pw, sw = _codes(N + K + 1, N, K, G)
@@ -40,7 +40,8 @@ def test_group_partials_exact(lib, M, N, K, G):
 @pytest.mark.parametrize("M,N,K,G", [(1, 16, 128, 32), (3, 48, 256, 64), (129, 272, 384, 128),
                                      (64, 512, 4096, 128), (200, 176, 192, 32), (16, 256, 1024, 256),
                                      (300, 784, 640, 64), (5, 640, 1152, 96), (130, 208, 1344, 192),
-                                     (7, 96, 896, 224), (33, 144, 640, 160)])
+                                     (7, 96, 896, 224), (33, 144, 640, 160), (5, 640, 192, 192),
+                                     (7, 96, 448, 224)])
 @pytest.mark.parametrize("out", ["f32", "bf16"])
 def test_w4a4_linear_small(lib, M, N, K, G, out):
     import torch
