@@ -61,6 +61,23 @@ def test_rht_quant(lib, K, G, bits):
     assert gflag.sum() <= max(6, 0.06 * gflag.size)
 
 
+@pytest.mark.parametrize("G", [32, 64, 128])
+@pytest.mark.parametrize("M", [1, 5, 2961])
+def test_rht_quant_k2048_strided_ragged(lib, M, G):
+    """K = 2048 bf16 int4 (the tensor-core first stage): rows with a pitch of K + 64 elements and
+    row counts just past one round of the persistent slots; sampled rows against the oracle."""
+    import torch
+    K = 2048
+    A, s = _acts(M, K, 7 * M + G)
+    big = torch.zeros((M, K + 64), dtype=torch.bfloat16, device="cuda")
+    big[:, :K] = to_device(A, True)
+    plan = lib.Plan.rht(K, s)
+    codes, scales = lib.rot_quant(big[:, :K], plan, 4, G)
+    rows = sample_rows(M, 64)
+    idx = rows.tolist()
+    assert_codes_match(codes[idx].cpu().numpy(), scales[idx].cpu().numpy(), Hd.rht_apply(A[rows], s), 4, G)
+
+
 def test_rht_quant_fp32_input_and_page2_probe_without_signs(lib):
     wl = W.make_workload("pr1")
     for signs in (wl.signs, None):
