@@ -48,8 +48,8 @@ _lib.rot_check_device.argtypes = []
 _lib.rot_last_error.restype = C.c_char_p
 _lib.rot_version.restype = C.c_char_p
 for _f in ("rot_plan_create", "rot_plan_destroy", "rot_plan_info", "rot_apply", "rot_quant", "rot_dequant",
-           "w4a4_linear", "w4a4_linear_noalloc", "w4a4_group_partials", "rot_harp_givens_blocks", "rot_harp_qr_block",
-           "rot_check_device"):
+           "w4a4_linear", "w4a4_linear_noalloc", "w4a4_group_partials", "w4a4_tile_plan", "rot_harp_givens_blocks",
+           "rot_harp_qr_block", "rot_check_device"):
     getattr(_lib, _f).restype = _int
 
 
@@ -92,6 +92,28 @@ def _dtype_code(t) -> int:
 
 def _ptr(t) -> C.c_void_p:
     return C.c_void_p(t.data_ptr()) if t is not None else C.c_void_p(0)
+
+
+def _arg(t, name: str, *, dtype=None, shape=None, strided_rows: bool = False):
+    """Check a tensor argument before its address reaches a kernel: on a CUDA device (a host
+    address would be dereferenced by the GPU), of the expected dtype and shape, and laid out as
+    the C ABI reads it (dense rows; with strided_rows, unit stride along a row only)."""
+    import torch
+    if not isinstance(t, torch.Tensor):
+        raise RotError(ROT_EINVAL, f"{name} must be a torch tensor")
+    if not t.is_cuda:
+        raise RotError(ROT_EINVAL, f"{name} must be on a CUDA device, not {t.device}")
+    if dtype is not None and t.dtype not in (dtype if isinstance(dtype, tuple) else (dtype,)):
+        raise RotError(ROT_EINVAL, f"{name} must be {dtype}, got {t.dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise RotError(ROT_EINVAL, f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if t.numel() > 0:
+        if strided_rows:
+            if t.dim() != 2 or t.stride(1) != 1:
+                raise RotError(ROT_EINVAL, f"{name} must be 2-D with unit stride along its rows")
+        elif not t.is_contiguous():
+            raise RotError(ROT_EINVAL, f"{name} must be contiguous")
+    return C.c_void_p(t.data_ptr())
 
 
 class Plan:
@@ -177,70 +199,96 @@ class Plan:
 def rot_apply(A, plan: Plan, *, inverse: bool = False, out=None, stream=None):
     """y = T a (or T^T a) for every row of A (cuda bf16/fp32 [M, >=K]); fp32 [M, K] out."""
     import torch
+    pa = _arg(A, "A", dtype=(torch.bfloat16, torch.float32), strided_rows=True)
     M = A.shape[0]
     if out is None:
         Kp = (plan.K + 3) // 4 * 4   # 16-byte aligned rows
         out = torch.empty((M, Kp), dtype=torch.float32, device=A.device)[:, :plan.K]
-    _check(_lib.rot_apply(_ptr(A), _dtype_code(A), M, A.stride(0), plan.handle, int(inverse), _ptr(out),
-                          out.stride(0), _stream(stream)))
+    po = _arg(out, "out", dtype=torch.float32, strided_rows=True)
+    _check(_lib.rot_apply(pa, _dtype_code(A), M, A.stride(0), plan.handle, int(inverse), po, out.stride(0),
+                          _stream(stream)))
     return out
 
 
 def rot_quant(A, plan: Plan, bits: int, G: int, *, codes=None, scales=None, stream=None):
     """Fused rotate + group quantise + pack. Returns (codes uint8 [M, K*bits/8], scales fp16 [M, K/G])."""
     import torch
+    pa = _arg(A, "A", dtype=(torch.bfloat16, torch.float32), strided_rows=True)
     M = A.shape[0]
     K = plan.K
     if codes is None:
         codes = torch.empty((M, K * bits // 8), dtype=torch.uint8, device=A.device)
     if scales is None:
         scales = torch.empty((M, K // G), dtype=torch.float16, device=A.device)
-    _check(_lib.rot_quant(_ptr(A), _dtype_code(A), M, A.stride(0), plan.handle, bits, G, _ptr(codes),
-                          _ptr(scales), _stream(stream)))
+    pc = _arg(codes, "codes", dtype=torch.uint8, shape=(M, K * bits // 8))
+    ps = _arg(scales, "scales", dtype=torch.float16, shape=(M, K // G) if G > 0 else None)
+    _check(_lib.rot_quant(pa, _dtype_code(A), M, A.stride(0), plan.handle, bits, G, pc, ps, _stream(stream)))
     return codes, scales
 
 
 def rot_dequant(codes, scales, plan: Plan, bits: int, G: int, *, inverse: bool = False, out=None, stream=None):
     """x_hat = q * s (rotated basis) or T^T (q * s) (original basis); fp32 [M, K]."""
     import torch
+    pc = _arg(codes, "codes", dtype=torch.uint8)
     M = codes.shape[0]
+    ps = _arg(scales, "scales", dtype=torch.float16)
     if out is None:
         out = torch.empty((M, plan.K), dtype=torch.float32, device=codes.device)
-    _check(_lib.rot_dequant(_ptr(codes), _ptr(scales), M, plan.handle, bits, G, int(inverse), _ptr(out),
-                            _stream(stream)))
+    po = _arg(out, "out", dtype=torch.float32, shape=(M, plan.K))
+    _check(_lib.rot_dequant(pc, ps, M, plan.handle, bits, G, int(inverse), po, _stream(stream)))
     return out
+
+
+def _w4a4_args(Aq, As, Wq, Ws, G: int):
+    """Shapes (M, N, K) and checked addresses of the W4A4 operands (As / Ws may be None)."""
+    import torch
+    pw = _arg(Wq, "Wq", dtype=torch.uint8)
+    if Wq.dim() != 2:
+        raise RotError(ROT_EINVAL, "Wq must be 2-D [N, K/2]")
+    N, K = Wq.shape[0], Wq.shape[1] * 2
+    if G <= 0 or K % G != 0:
+        raise RotError(ROT_EINVAL, f"G = {G} must divide K = {K}")
+    pa = _arg(Aq, "Aq", dtype=torch.uint8)
+    if Aq.dim() != 2 or Aq.shape[1] * 2 != K:
+        raise RotError(ROT_EINVAL, f"Aq must be [M, {K // 2}] like Wq")
+    M = Aq.shape[0]
+    ps_a = _arg(As, "As", dtype=torch.float16, shape=(M, K // G)) if As is not None else C.c_void_p(0)
+    ps_w = _arg(Ws, "Ws", dtype=torch.float16, shape=(N, K // G)) if Ws is not None else C.c_void_p(0)
+    return M, N, K, (pa, ps_a, pw, ps_w)
 
 
 def w4a4_linear(Aq, As, Wq, Ws, G: int, *, out_dtype=None, out=None, stream=None):
     """C = sum_g sA sW (qA qW^T)_g for int4 codes Aq [M, K/2], Wq [N, K/2]; fp32 or bf16 [M, N]."""
     import torch
-    M, N, K = Aq.shape[0], Wq.shape[0], Wq.shape[1] * 2
+    M, N, K, ptrs = _w4a4_args(Aq, As, Wq, Ws, G)
     if out is None:
         out = torch.empty((M, N), dtype=out_dtype or torch.float32, device=Wq.device)
+    po = _arg(out, "out", dtype=(torch.float32, torch.bfloat16), shape=(M, N))
     cd = ROT_BF16 if out.dtype == torch.bfloat16 else ROT_F32
-    _check(_lib.w4a4_linear(_ptr(Aq), _ptr(As), _ptr(Wq), _ptr(Ws), M, N, K, G, _ptr(out), cd, _stream(stream)))
+    _check(_lib.w4a4_linear(*ptrs, M, N, K, G, po, cd, _stream(stream)))
     return out
 
 
 def w4a4_linear_noalloc(Aq, As, Wq, Ws, G: int, *, out_dtype=None, out=None, stream=None):
     """w4a4_linear that never allocates device memory (static split-K buffer; see the header)."""
     import torch
-    M, N, K = Aq.shape[0], Wq.shape[0], Wq.shape[1] * 2
+    M, N, K, ptrs = _w4a4_args(Aq, As, Wq, Ws, G)
     if out is None:
         out = torch.empty((M, N), dtype=out_dtype or torch.float32, device=Wq.device)
+    po = _arg(out, "out", dtype=(torch.float32, torch.bfloat16), shape=(M, N))
     cd = ROT_BF16 if out.dtype == torch.bfloat16 else ROT_F32
-    _check(_lib.w4a4_linear_noalloc(_ptr(Aq), _ptr(As), _ptr(Wq), _ptr(Ws), M, N, K, G, _ptr(out), cd,
-                                    _stream(stream)))
+    _check(_lib.w4a4_linear_noalloc(*ptrs, M, N, K, G, po, cd, _stream(stream)))
     return out
 
 
 def w4a4_group_partials(Aq, Wq, G: int, *, out=None, stream=None):
     """Exact int32 group sums P[m, n, g] of the W4A4 contraction."""
     import torch
-    M, N, K = Aq.shape[0], Wq.shape[0], Wq.shape[1] * 2
+    M, N, K, ptrs = _w4a4_args(Aq, None, Wq, None, G)
     if out is None:
         out = torch.empty((M, N, K // G), dtype=torch.int32, device=Wq.device)
-    _check(_lib.w4a4_group_partials(_ptr(Aq), _ptr(Wq), M, N, K, G, _ptr(out), _stream(stream)))
+    po = _arg(out, "out", dtype=torch.int32, shape=(M, N, K // G))
+    _check(_lib.w4a4_group_partials(ptrs[0], ptrs[2], M, N, K, G, po, _stream(stream)))
     return out
 
 

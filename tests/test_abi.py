@@ -141,3 +141,26 @@ def test_w4a4_tile_plan_rejects_bad_shapes(lib):
         with pytest.raises(lib.RotError) as e:
             lib.w4a4_tile_plan(*args)
         assert e.value.status == lib.ROT_EINVAL
+
+
+def test_binding_rejects_host_tensors_before_any_kernel(lib):
+    """A host tensor's address must never reach a kernel: the binding refuses it (ROT_EINVAL)
+    before calling the library, with no device needed."""
+    import types
+    import torch
+    fake_plan = types.SimpleNamespace(K=256, handle=None)
+    A = torch.zeros((4, 256), dtype=torch.bfloat16)
+    for call in (lambda: lib.rot_quant(A, fake_plan, 4, 32),
+                 lambda: lib.rot_apply(A, fake_plan),
+                 lambda: lib.rot_dequant(torch.zeros((4, 128), dtype=torch.uint8),
+                                         torch.zeros((4, 8), dtype=torch.float16), fake_plan, 4, 32),
+                 lambda: lib.w4a4_linear(torch.zeros((4, 64), dtype=torch.uint8), torch.zeros((4, 1), dtype=torch.float16),
+                                         torch.zeros((16, 64), dtype=torch.uint8), torch.zeros((16, 1), dtype=torch.float16),
+                                         128),
+                 lambda: lib.w4a4_group_partials(torch.zeros((4, 64), dtype=torch.uint8),
+                                                 torch.zeros((16, 64), dtype=torch.uint8), 128),
+                 lambda: lib.rot_quant(np.zeros((4, 256), dtype=np.float32), fake_plan, 4, 32)):
+        with pytest.raises(lib.RotError) as e:
+            call()
+        assert e.value.status == lib.ROT_EINVAL
+        assert "CUDA" in str(e.value) or "torch tensor" in str(e.value)
