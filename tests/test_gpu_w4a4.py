@@ -66,7 +66,7 @@ def test_w4a4_empty_M(lib):
     assert C.shape == (0, 32)
 
 
-@pytest.mark.parametrize("name", ["q_proj_prefill", "q_proj_decode", "up_proj_decode"])
+@pytest.mark.parametrize("name", ["q_proj_prefill", "up_proj_prefill", "q_proj_decode", "up_proj_decode"])
 def test_w4a4_workload_oracle_codes(lib, name):
     """Full-size linear on oracle-quantised codes (parity isolates the GEMM; the codes of the
     workload's activation and weight shapes are quantised without rotation to keep the oracle fast)."""
