@@ -45,11 +45,12 @@ _lib.w4a4_tile_plan.argtypes = [_i64, _i64, _i64, _int, _int, _int, C.POINTER(_i
 _lib.rot_harp_givens_blocks.argtypes = [C.POINTER(C.c_double), _i64, C.POINTER(C.c_float)]
 _lib.rot_harp_qr_block.argtypes = [C.POINTER(C.c_double), _int, C.POINTER(C.c_float)]
 _lib.rot_check_device.argtypes = []
+_lib.rot_test_inject.argtypes = [_int, _i64]
 _lib.rot_last_error.restype = C.c_char_p
 _lib.rot_version.restype = C.c_char_p
 for _f in ("rot_plan_create", "rot_plan_destroy", "rot_plan_info", "rot_apply", "rot_quant", "rot_dequant",
            "w4a4_linear", "w4a4_linear_noalloc", "w4a4_group_partials", "w4a4_tile_plan", "rot_harp_givens_blocks",
-           "rot_harp_qr_block", "rot_check_device"):
+           "rot_harp_qr_block", "rot_check_device", "rot_test_inject"):
     getattr(_lib, _f).restype = _int
 
 
@@ -94,15 +95,25 @@ def _ptr(t) -> C.c_void_p:
     return C.c_void_p(t.data_ptr()) if t is not None else C.c_void_p(0)
 
 
+def _check_device(index, current: int, name: str):
+    """The library launches on the current CUDA device: an operand on another device would be
+    read and written from the wrong GPU. ROT_EINVAL unless ``index`` is the current device."""
+    if index is None or int(index) != int(current):
+        raise RotError(ROT_EINVAL, f"{name} is on cuda:{index}, but the current device is cuda:{current} "
+                                   "(call under torch.cuda.device(...) of the operands' device)")
+
+
 def _arg(t, name: str, *, dtype=None, shape=None, strided_rows: bool = False):
-    """Check a tensor argument before its address reaches a kernel: on a CUDA device (a host
-    address would be dereferenced by the GPU), of the expected dtype and shape, and laid out as
-    the C ABI reads it (dense rows; with strided_rows, unit stride along a row only)."""
+    """Check a tensor argument before its address reaches a kernel: on the current CUDA device
+    (a host address, or another GPU's memory, would be dereferenced by the wrong device), of the
+    expected dtype and shape, and laid out as the C ABI reads it (dense rows; with strided_rows,
+    unit stride along a row only)."""
     import torch
     if not isinstance(t, torch.Tensor):
         raise RotError(ROT_EINVAL, f"{name} must be a torch tensor")
     if not t.is_cuda:
         raise RotError(ROT_EINVAL, f"{name} must be on a CUDA device, not {t.device}")
+    _check_device(t.device.index, torch.cuda.current_device(), name)
     if dtype is not None and t.dtype not in (dtype if isinstance(dtype, tuple) else (dtype,)):
         raise RotError(ROT_EINVAL, f"{name} must be {dtype}, got {t.dtype}")
     if shape is not None and tuple(t.shape) != tuple(shape):
@@ -349,3 +360,12 @@ def harp_plan(draws, signs, variant: str) -> Plan:
 def check_device():
     """Synchronise and raise if a bounded device wait gave up since the last check."""
     _check(_lib.rot_check_device())
+
+
+ROT_TEST_NONE, ROT_TEST_ROTATION_COPY, ROT_TEST_W4A4_LOADS = 0, 1, 2
+
+
+def test_inject(fault: int, wait_ns: int = 0):
+    """Testing hook (rot_test_inject): make the next launch of one kernel family skip its copies
+    so that its bounded waits run out, and/or set the wait bound (0 = defaults)."""
+    _check(_lib.rot_test_inject(int(fault), int(wait_ns)))

@@ -88,6 +88,8 @@ struct Args {
   float norm;
   float cdiv;        // fp32(norm / qmax)
   float cf;          // fp32(norm * (1 + 2^-22))
+  unsigned long long wait_ns;  // bound of the staging waits
+  int skip_first;    // testing hook: slot 0 of CTA 0 never issues its first staging copy
 };
 
 enum { MODE_APPLY = 0, MODE_APPLY_INV = 1, MODE_QUANT = 2 };
@@ -160,8 +162,9 @@ __device__ __forceinline__ uint32_t smem_addr(const void* p) {
 }
 
 // Bounded wait on a slot's staging barrier (the bulk copy always completes; the bound only
-// protects against a programming error). Returns false after about 1 s.
-__device__ __forceinline__ bool stage_wait(uint64_t* bar, uint32_t parity) {
+// protects against a programming error, and lets the testing hook check this path). Returns
+// false after limit_ns of wall time (1 s by default) and records ROT_ETIMEOUT.
+__device__ __forceinline__ bool stage_wait(uint64_t* bar, uint32_t parity, unsigned long long limit_ns) {
   const uint32_t addr = smem_addr(bar);
   unsigned long long t0 = 0;
   for (uint32_t it = 0;; ++it) {
@@ -178,7 +181,7 @@ __device__ __forceinline__ bool stage_wait(uint64_t* bar, uint32_t parity) {
       unsigned long long now;
       asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(now));
       if (t0 == 0) t0 = now;
-      else if (now - t0 > 1000000000ull) {
+      else if (now - t0 > limit_ns) {
         atomicExch(&g_fwht_error, (int)ROT_ETIMEOUT);
         return false;
       }
@@ -436,7 +439,8 @@ __global__ void __launch_bounds__(Cfg<LOGN>::THREADS, 1) fwht_kernel(const Args 
   asm volatile("griddepcontrol.wait;" ::: "memory");
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   // the slot leader initialised its own barrier: it can start the first copy at once
-  if (t == 0 && u < units) stage_issue(bar, buf, src_of(row, chunk), chunk_bytes);
+  if (t == 0 && u < units && !(a.skip_first && blockIdx.x == 0 && slot == 0))
+    stage_issue(bar, buf, src_of(row, chunk), chunk_bytes);
   __syncthreads();
 
   // per-thread shared-memory bases (loop invariant); compile-time offsets are added per access
@@ -458,7 +462,7 @@ __global__ void __launch_bounds__(Cfg<LOGN>::THREADS, 1) fwht_kernel(const Args 
   for (; u < units; u += stride) {
     const int cbase = chunk * N;
     float2 xp[NP];
-    if (!stage_wait(bar, parity)) break;
+    if (!stage_wait(bar, parity, a.wait_ns)) break;
     parity ^= 1u;
 
     // ---------------- phase A: runs of NV elements from the staged chunk, signs, fp32 pairs
@@ -681,7 +685,8 @@ __global__ void __launch_bounds__(MMA_THREADS, 1) fwht_mma_kernel(const Args a) 
   }
   asm volatile("griddepcontrol.wait;" ::: "memory");
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  if (l == 0 && u < units) stage_issue(bar, buf, src_of(row, chunk), N * 2);
+  if (l == 0 && u < units && !(a.skip_first && blockIdx.x == 0 && slot == 0))
+    stage_issue(bar, buf, src_of(row, chunk), N * 2);
   __syncthreads();
 
   // B fragments of H_16 for the two MMAs (outputs o3 = 0 / 1): n = g, k = 2c + {0,1} (+8)
@@ -702,7 +707,7 @@ __global__ void __launch_bounds__(MMA_THREADS, 1) fwht_mma_kernel(const Args a) 
   for (; u < units; u += stride) {
     const int cbase = chunk * N;
     float2 xp[NP];
-    if (!stage_wait(bar, parity)) break;
+    if (!stage_wait(bar, parity, a.wait_ns)) break;
     parity ^= 1u;
 
     // ---------------- MMA: H_16 over {e0, e1, e2, e6} for the 8 row tiles
@@ -906,6 +911,8 @@ Args make_args(const rot_plan_s* p, const void* A, int64_t M, int64_t lda) {
   a.chunks = p->K >> p->chunk_log2;
   a.signmask = p->has_signs ? p->d_signmask : nullptr;
   a.norm = (float)(1.0 / std::sqrt((double)(1 << p->chunk_log2)));
+  a.wait_ns = wait_limit_ns(1000000000ull);
+  a.skip_first = take_test_fault(TEST_FAULT_ROTATION_COPY) ? 1 : 0;
   return a;
 }
 

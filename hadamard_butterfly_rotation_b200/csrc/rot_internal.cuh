@@ -24,6 +24,12 @@ rot_status cuda_error(cudaError_t e, const char* what);
 
 int sm_count();  // SMs of the current device (cached per device)
 
+// Testing hook (rot_test_inject): a one-shot fault for the next launch of one kernel family
+// and an optional bound for the kernels' device-side waits.
+enum { TEST_FAULT_NONE = 0, TEST_FAULT_ROTATION_COPY = 1, TEST_FAULT_W4A4_LOADS = 2 };
+bool take_test_fault(int which);                        // true once after rot_test_inject(which, .)
+unsigned long long wait_limit_ns(unsigned long long dflt);  // the injected bound, else dflt
+
 // ---------------------------------------------------------------- plan
 struct Stage {
   int b = 0;            // radix

@@ -8,6 +8,7 @@
 // Sylvester-Hadamard stages over the leading digits are, per contiguous chunk of
 // 2^n coordinates, a signed Walsh-Hadamard transform [HARP abstract: the processor
 // initialises to the RHT]; those run on the fused butterfly kernel.
+#include <atomic>
 #include <cmath>
 #include <cstring>
 #include <mutex>
@@ -44,6 +45,19 @@ int sm_count() {
   return cache[dev];
 }
 
+static std::atomic<int> g_test_fault{TEST_FAULT_NONE};
+static std::atomic<long long> g_test_wait_ns{0};
+
+bool take_test_fault(int which) {
+  int expected = which;
+  return which != TEST_FAULT_NONE && g_test_fault.compare_exchange_strong(expected, TEST_FAULT_NONE);
+}
+
+unsigned long long wait_limit_ns(unsigned long long dflt) {
+  const long long v = g_test_wait_ns.load();
+  return v > 0 ? (unsigned long long)v : dflt;
+}
+
 static bool is_pow2(int64_t x) { return x >= 1 && (x & (x - 1)) == 0; }
 
 // Entry (r, c) of the Sylvester matrix H_b: (-1)^popcount(r & c).
@@ -65,7 +79,15 @@ using namespace rotb;
 
 extern "C" const char* rot_last_error(void) { return g_last_error.c_str(); }
 
-extern "C" const char* rot_version(void) { return "rot_b200 1.0 (sm_100a)"; }
+extern "C" const char* rot_version(void) { return "rot_b200 1.1 (sm_100a)"; }
+
+extern "C" rot_status rot_test_inject(int fault, int64_t wait_ns) {
+  if (fault < TEST_FAULT_NONE || fault > TEST_FAULT_W4A4_LOADS || wait_ns < 0)
+    return set_error(ROT_EINVAL, "rot_test_inject: unknown fault or negative wait bound");
+  g_test_wait_ns.store(wait_ns);
+  g_test_fault.store(fault);
+  return ROT_OK;
+}
 
 extern "C" rot_status rot_plan_create(rot_plan_t* out, int K, int n_stages, const int* radices,
                                       const float* const* stage_params, const int64_t* n_blocks,

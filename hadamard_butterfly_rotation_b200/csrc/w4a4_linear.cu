@@ -113,6 +113,8 @@ struct Params {
   int units;         // tiles * splits
   int kb_per_split;  // K-blocks per split; a multiple of lcm(G, KB) / KB
   float* Cacc;       // split-K: fp32 [M, N] accumulated with atomics (zeroed beforehand), else null
+  unsigned long long wait_ns;  // bound of every mbarrier wait
+  int skip_loads;    // testing hook: the loader issues no TMA load, so every wait runs out
 };
 
 // One work unit: an output tile and a group-aligned K range.
@@ -158,7 +160,8 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
 // role here waits once or twice per K-block, so the cheap form matters. Between unsuccessful
 // polls the warp sleeps for a few tens of nanoseconds. Gives up after ~2 s (records
 // ROT_ETIMEOUT and raises the CTA's abort flag).
-__device__ __forceinline__ bool bar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+__device__ __forceinline__ bool bar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                         unsigned long long limit_ns) {
   const uint32_t addr = smem_u32(bar);
   bool ok = true;
   unsigned long long t0 = 0;
@@ -183,7 +186,7 @@ __device__ __forceinline__ bool bar_wait(uint64_t* bar, uint32_t parity, volatil
       unsigned long long now;
       asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(now));
       if (t0 == 0) t0 = now;
-      else if (now - t0 > WAIT_NS) {
+      else if (now - t0 > limit_ns) {
         *abort_flag = 1;
         atomicExch(&g_w4a4_error, (int)ROT_ETIMEOUT);
         ok = false;
@@ -413,7 +416,7 @@ __global__ void __launch_bounds__(THREADS, 1) w4a4_kernel(const __grid_constant_
           __syncwarp();
         }
         const int b = gc % NACC;
-        ok = ok && bar_wait(&tfull[b], (gc / NACC) & 1, abort_flag);
+        ok = ok && bar_wait(&tfull[b], (gc / NACC) & 1, abort_flag, p.wait_ns);
         if (!ok) break;
         tc_fence_after();
         uint32_t r0[32], r1[32];
@@ -503,12 +506,12 @@ __global__ void __launch_bounds__(THREADS, 1) w4a4_kernel(const __grid_constant_
     // (two 2-D TMA boxes; rows beyond M / N and bytes beyond K/2 arrive as zeros)
     asm volatile("setmaxnreg.dec.sync.aligned.u32 80;");
     int it = 0;
-    bool ok = true;
+    bool ok = !p.skip_loads;   // testing hook: no load is ever issued (nothing in flight)
     for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x) {
       const Unit w = unit_of(p, u);
       for (int j = 0; j < w.nkb; ++j, ++it) {
         const int ps = it % PSTAGES;
-        if (it >= PSTAGES && !bar_wait(&pempty[ps], ((it / PSTAGES) + 1) & 1, abort_flag)) {
+        if (it >= PSTAGES && !bar_wait(&pempty[ps], ((it / PSTAGES) + 1) & 1, abort_flag, p.wait_ns)) {
           ok = false;
           break;
         }
@@ -540,8 +543,8 @@ __global__ void __launch_bounds__(THREADS, 1) w4a4_kernel(const __grid_constant_
       const Unit w = unit_of(p, u);
       for (int j = 0; j < w.nkb; ++j, ++it) {
         const int s = it % STAGES, ps = it % PSTAGES;
-        if (!bar_wait(&pfull[ps], (it / PSTAGES) & 1, abort_flag) ||
-            (it >= STAGES && !bar_wait(&empty[s], ((it / STAGES) + 1) & 1, abort_flag))) {
+        if (!bar_wait(&pfull[ps], (it / PSTAGES) & 1, abort_flag, p.wait_ns) ||
+            (it >= STAGES && !bar_wait(&empty[s], ((it / STAGES) + 1) & 1, abort_flag, p.wait_ns))) {
           ok = false;
           break;
         }
@@ -588,7 +591,7 @@ __global__ void __launch_bounds__(THREADS, 1) w4a4_kernel(const __grid_constant_
     for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x) {
       const Unit w = unit_of(p, u);         // K range group-aligned: kg == 0 here
       for (int j = 0; j < w.nkb; ++j) {
-        if (!bar_wait(&full[s], sph, abort_flag)) {
+        if (!bar_wait(&full[s], sph, abort_flag, p.wait_ns)) {
           ok = false;
           break;
         }
@@ -599,7 +602,7 @@ __global__ void __launch_bounds__(THREADS, 1) w4a4_kernel(const __grid_constant_
         for (int k4 = 0; k4 < 4; ++k4) {
           if (k4 < nk) {
             if (kg == 0) {
-              if (!bar_wait(&tempty[b], tph, abort_flag)) {
+              if (!bar_wait(&tempty[b], tph, abort_flag, p.wait_ns)) {
                 ok = false;
                 break;
               }
@@ -628,7 +631,7 @@ __global__ void __launch_bounds__(THREADS, 1) w4a4_kernel(const __grid_constant_
     // the last stage-release commit must have landed before the CTA (and its smem) goes away
     if (ok && nblk > 0) {
       const int last = s == 0 ? STAGES - 1 : s - 1;
-      bar_wait(&empty[last], s == 0 ? sph ^ 1 : sph, abort_flag);
+      bar_wait(&empty[last], s == 0 ? sph ^ 1 : sph, abort_flag, p.wait_ns);
     }
   }
 
@@ -944,6 +947,8 @@ rot_status w4a4_launch(const uint8_t* Aq, const uint16_t* As, const uint8_t* Wq,
   p.tiles_m = (int)tp.tiles_m;
   p.units = (int)tp.units;
   p.Cacc = nullptr;
+  p.wait_ns = wait_limit_ns(WAIT_NS);
+  p.skip_loads = take_test_fault(TEST_FAULT_W4A4_LOADS) ? 1 : 0;
   if (p.splits > 1) {
     rot_status st = acc_target(&p.Cacc);
     if (st) return st;

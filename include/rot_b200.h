@@ -174,6 +174,24 @@ rot_status rot_harp_qr_block(const double* g, int b, float* out);
  * waits (ROT_ETIMEOUT) since the last call; clears the record. */
 rot_status rot_check_device(void);
 
+/* Testing hook for the bounded-wait failure path (the pages have no counterpart). Every
+ * device-side wait of the fused rotation kernels (staging copies) and of the W4A4 tile kernel
+ * (its mbarrier pipeline) gives up after a bound of wall time, records ROT_ETIMEOUT for
+ * rot_check_device and returns without leaving a copy or an MMA in flight. This call makes
+ * that happen on purpose, so tests can check the path without faulting the GPU:
+ *   fault = 0  no fault (only sets the bound)
+ *   fault = 1  ROT_TEST_ROTATION_COPY: the next rot_quant / rot_apply launch of the fused
+ *              rotation kernel does not issue the first staging copy of CTA 0's first slot;
+ *              that slot's waits run out, every other slot completes normally
+ *   fault = 2  ROT_TEST_W4A4_LOADS: the next launch of the W4A4 tile kernel (M > 64 or
+ *              G % 128 != 0) issues no TMA load; every role's waits run out
+ * The fault is one-shot (consumed by the next launch of that kernel family on any thread).
+ * wait_ns > 0 sets the bound of those waits (default: 1 s rotation, 2 s W4A4) until the
+ * next call; 0 restores the defaults. Outputs of a launch that gave up are unspecified.
+ * ROT_EINVAL for an unknown fault or wait_ns < 0. Host only. */
+enum { ROT_TEST_NONE = 0, ROT_TEST_ROTATION_COPY = 1, ROT_TEST_W4A4_LOADS = 2 };
+rot_status rot_test_inject(int fault, int64_t wait_ns);
+
 /* Last error message of the calling host thread ("" if none). */
 const char* rot_last_error(void);
 

@@ -14,7 +14,7 @@ Sources (HARP, arXiv 2605.29843):
   matrix for powers of two, the QR fallback otherwise; Q is a Givens rotation for
   b_t = 2; at theta = 0, Q = I so B = G and HARP equals the RHT.
 
-Readings where the pages leave a step open (each listed in the design doc):
+Readings where the pages leave a step open:
 * digit addressing: coordinate i = sum_t d_t s_t with s_t = prod_{u<t} b_u
   (digit 0 least significant). Stage t mixes the b_t coordinates that differ only
   in digit t, base + r*s_t for r = 0..b_t-1, with block index

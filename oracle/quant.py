@@ -2,11 +2,18 @@
 
 Source: Hadamard-Int4-Accuracy wiki, Method: ``q_dequant_vec(x, out, K, G, bits)``
 is per-group symmetric integer quantise -> dequantise for any bit-width; Hypothesis:
-outliers blow out the per-group absmax scale. The probe works in fp32 ("exactly in
-fp32"), so the integer decisions below are taken in fp32; the inputs (rotated
-values) come from the fp64 rotation rounded once to fp32.
+outliers blow out the per-group absmax scale.
 
-Readings (listed in DESIGN.md):
+Decision precision: the pages fix no precision for the quantiser's decisions (the
+wiki's "exactly in fp32" is said of the identity A.B = (A.Q)(Q.B), not of the
+quantiser). Where floating point decides an integer, this oracle takes the decision in
+the precision the CUDA kernels compute in, fp32: the fp64 rotated value is rounded
+once to fp32, the scale is fp32(absmax / qmax) rounded to binary16, and the quotient
+y / s is an fp32 division. Against an all-fp64 decision this moves |y/s| by about
+1e-6 (relative 2^-24 per rounding) and absmax/qmax by about 1e-7 relative, so the two
+readings differ only inside the 1e-5 boundary windows that ``boundary_flags`` marks.
+
+Readings where the pages are silent:
 * levels are symmetric: qmax = 2^(bits-1) - 1 (int4: -7..7, int2: -1..1, int8:
   -127..127); the code -2^(bits-1) is never produced;
 * scale s = fp16_rn(fp32(absmax / qmax)); codes use that stored fp16 value, so

@@ -164,3 +164,24 @@ def test_binding_rejects_host_tensors_before_any_kernel(lib):
             call()
         assert e.value.status == lib.ROT_EINVAL
         assert "CUDA" in str(e.value) or "torch tensor" in str(e.value)
+
+
+def test_binding_rejects_operands_on_another_device(lib):
+    """Operands must live on the current device (the library launches there): the binding's
+    device check raises ROT_EINVAL for any other index, before an address reaches a kernel."""
+    lib._check_device(0, 0, "A")
+    lib._check_device(3, 3, "A")
+    for idx, cur in ((1, 0), (0, 2), (None, 0)):
+        with pytest.raises(lib.RotError) as e:
+            lib._check_device(idx, cur, "Wq")
+        assert e.value.status == lib.ROT_EINVAL and "Wq" in str(e.value)
+
+
+def test_test_inject_rejects_unknown_faults(lib):
+    """The testing hook refuses unknown faults and negative bounds (host only, no device)."""
+    with pytest.raises(lib.RotError) as e:
+        lib.test_inject(7, 0)
+    assert e.value.status == lib.ROT_EINVAL
+    with pytest.raises(lib.RotError):
+        lib.test_inject(0, -1)
+    lib.test_inject(lib.ROT_TEST_NONE, 0)

@@ -6,7 +6,8 @@ import workloads as W
 from oracle import hadamard as Hd
 from oracle import harp as Hp
 from oracle import quant as Q
-from parity import (assert_codes_match, assert_rotated_close, padded_rows, sample_rows, to_device)
+from parity import (assert_codes_match, assert_rotated_close, guarded_apply, guarded_quant, padded_rows,
+                    sample_rows, to_device)
 
 pytestmark = pytest.mark.gpu
 
@@ -24,9 +25,9 @@ def test_rht_apply(lib, K, bf16):
     A, s = _acts(37, K, K, bf16)
     plan = lib.Plan.rht(K, s)
     assert plan.info()["chunk"] == K
-    y = lib.rot_apply(to_device(A, bf16), plan).cpu().numpy()
+    y = guarded_apply(lib, to_device(A, bf16), plan).cpu().numpy()
     assert_rotated_close(y, Hd.rht_apply(A, s))
-    yi = lib.rot_apply(to_device(A, bf16), plan, inverse=True).cpu().numpy()
+    yi = guarded_apply(lib, to_device(A, bf16), plan, inverse=True).cpu().numpy()
     assert_rotated_close(yi, Hd.rht_apply(A, s, inverse=True))
 
 
@@ -38,7 +39,7 @@ def test_rht_apply_ragged_rows_and_stride(lib, M):
     big = torch.zeros((M, K + 64), dtype=torch.bfloat16, device="cuda")
     big[:, :K] = to_device(A, True)
     plan = lib.Plan.rht(K, s)
-    y = lib.rot_apply(big[:, :K], plan).cpu().numpy()
+    y = guarded_apply(lib, big[:, :K], plan).cpu().numpy()
     assert_rotated_close(y, Hd.rht_apply(A, s))
 
 
@@ -51,9 +52,9 @@ def test_rht_apply_ragged_rows_and_stride(lib, M):
 def test_rht_quant(lib, K, G, bits):
     A, s = _acts(67, K, K + G + bits)
     plan = lib.Plan.rht(K, s)
-    codes, scales = lib.rot_quant(to_device(A, True), plan, bits, G)
+    codes, scales = guarded_quant(lib, to_device(A, True), plan, bits, G)
     y = Hd.rht_apply(A, s)
-    assert_codes_match(codes.cpu().numpy(), scales.cpu().numpy(), y, bits, G)
+    assert_codes_match(codes, scales, y, bits, G)
     # exclusions stay rare: per-code windows well under 1e-3 of the codes, and scale windows
     # (binary16 midpoints are 2^-10 apart, the window 2e-5 wide) under 5% of the groups
     cflag, gflag = Q.boundary_flags(y, bits, G)
@@ -72,7 +73,7 @@ def test_rht_quant_k2048_strided_ragged(lib, M, G):
     big = torch.zeros((M, K + 64), dtype=torch.bfloat16, device="cuda")
     big[:, :K] = to_device(A, True)
     plan = lib.Plan.rht(K, s)
-    codes, scales = lib.rot_quant(big[:, :K], plan, 4, G)
+    codes, scales = guarded_quant(lib, big[:, :K], plan, 4, G)
     rows = sample_rows(M, 64)
     idx = rows.tolist()
     assert_codes_match(codes[idx].cpu().numpy(), scales[idx].cpu().numpy(), Hd.rht_apply(A[rows], s), 4, G)
@@ -83,8 +84,8 @@ def test_rht_quant_fp32_input_and_page2_probe_without_signs(lib):
     for signs in (wl.signs, None):
         plan = lib.Plan.rht(2048, signs)
         for bits, G in wl.quant:
-            codes, scales = lib.rot_quant(to_device(wl.A, False), plan, bits, G)
-            assert_codes_match(codes.cpu().numpy(), scales.cpu().numpy(), Hd.rht_apply(wl.A, signs), bits, G)
+            codes, scales = guarded_quant(lib, to_device(wl.A, False), plan, bits, G)
+            assert_codes_match(codes, scales, Hd.rht_apply(wl.A, signs), bits, G)
 
 
 def test_quant_edge_cases(lib):
@@ -99,8 +100,8 @@ def test_quant_edge_cases(lib):
     A[5] = W.rng(3).standard_normal(K)
     A = W.to_bf16_exact(A)
     plan = lib.Plan.rht(K, s)
-    codes, scales = lib.rot_quant(to_device(A, True), plan, 4, G)
-    assert_codes_match(codes.cpu().numpy(), scales.cpu().numpy(), Hd.rht_apply(A, s), 4, G)
+    codes, scales = guarded_quant(lib, to_device(A, True), plan, 4, G)
+    assert_codes_match(codes, scales, Hd.rht_apply(A, s), 4, G)
     # empty input is a no-op
     e = torch.empty((0, K), dtype=torch.bfloat16, device="cuda")
     c0, s0 = lib.rot_quant(e, plan, 4, G)
@@ -127,10 +128,10 @@ def test_workload_full_size_sampled_rows(lib, name):
     dA = to_device(wl.A, True)
     rows = sample_rows(wl.M, 48)
     y_ref = Hd.rht_apply(wl.A[rows], wl.signs)
-    y = lib.rot_apply(dA, plan)[rows.tolist()].cpu().numpy()
+    y = guarded_apply(lib, dA, plan)[rows.tolist()].cpu().numpy()
     assert_rotated_close(y, y_ref)
     for bits, G in wl.quant:
-        codes, scales = lib.rot_quant(dA, plan, bits, G)
+        codes, scales = guarded_quant(lib, dA, plan, bits, G)
         idx = rows.tolist()
         assert_codes_match(codes[idx].cpu().numpy(), scales[idx].cpu().numpy(), y_ref, bits, G)
 
@@ -142,7 +143,7 @@ def test_dequant_roundtrip(lib, bits, G):
     K = 8192
     A, s = _acts(9, K, 77)
     plan = lib.Plan.rht(K, s)
-    codes, scales = lib.rot_quant(to_device(A, True), plan, bits, G)
+    codes, scales = guarded_quant(lib, to_device(A, True), plan, bits, G)
     c_np, s_np = codes.cpu().numpy(), scales.cpu().numpy()
     # rotated basis: exact q * s of the GPU's own codes
     xh = lib.rot_dequant(codes, scales, plan, bits, G).cpu().numpy()
@@ -183,13 +184,13 @@ def test_harp_generic_apply_and_quant(lib, radices, per_block):
     assert plan.info()["chunk"] == 0
     dA = padded_rows(A)            # leading dimension rounded up to 16 bytes
     y_ref = Hp.harp_apply(A, spec)
-    y = lib.rot_apply(dA, plan).cpu().numpy()
+    y = guarded_apply(lib, dA, plan).cpu().numpy()
     assert_rotated_close(y, y_ref)
-    yi = lib.rot_apply(dA, plan, inverse=True).cpu().numpy()
+    yi = guarded_apply(lib, dA, plan, inverse=True).cpu().numpy()
     assert_rotated_close(yi, Hp.harp_apply(A, spec, inverse=True))
     if K % 8 == 0:
-        codes, scales = lib.rot_quant(dA, plan, 4, 8)
-        assert_codes_match(codes.cpu().numpy(), scales.cpu().numpy(), y_ref, 4, 8)
+        codes, scales = guarded_quant(lib, dA, plan, 4, 8)
+        assert_codes_match(codes, scales, y_ref, 4, 8)
 
 
 @pytest.mark.parametrize("variant", ["init_identity", "init_qr", "random"])
@@ -203,9 +204,42 @@ def test_harp11008_full_size(lib, variant):
     dA = to_device(wl.A, True)
     rows = sample_rows(wl.M, 24)
     y_ref = Hp.harp_apply(wl.A[rows], spec)
-    y = lib.rot_apply(dA, plan)[rows.tolist()].cpu().numpy()
+    y = guarded_apply(lib, dA, plan)[rows.tolist()].cpu().numpy()
     assert_rotated_close(y, y_ref)
     for bits, G in wl.quant:
-        codes, scales = lib.rot_quant(dA, plan, bits, G)
+        codes, scales = guarded_quant(lib, dA, plan, bits, G)
         idx = rows.tolist()
         assert_codes_match(codes[idx].cpu().numpy(), scales[idx].cpu().numpy(), y_ref, bits, G)
+
+
+# ----------------------------------------------------------------------------- fp32 input at large K
+
+@pytest.mark.parametrize("K,G,bits", [(4096, 128, 4), (4096, 32, 4), (8192, 128, 4), (8192, 64, 2)])
+def test_rht_quant_fp32_input_large_k(lib, K, G, bits):
+    """fp32 activations (the weight-preparation input type) at K = 4096 / 8192, every element."""
+    A, s = _acts(41, K, 3 * K + G + bits, bf16=False)
+    plan = lib.Plan.rht(K, s)
+    codes, scales = guarded_quant(lib, to_device(A, False), plan, bits, G)
+    assert_codes_match(codes, scales, Hd.rht_apply(A, s), bits, G)
+    y = guarded_apply(lib, to_device(A, False), plan).cpu().numpy()
+    assert_rotated_close(y, Hd.rht_apply(A, s))
+
+
+# ----------------------------------------------------------------------------- offline weight preparation
+
+@pytest.mark.parametrize("name", ["q_proj_prefill", "up_proj_prefill"])
+def test_weight_prep_full_size(lib, name):
+    """The offline step of the linear: the fp32 rows of W^T ([N, K] = [4096 or 11008, 4096]) through
+    the same RHT plan as the activations and quantised to int4 G = 128, at full size; codes and
+    scales of sampled rows bit-exact against the oracle's quantize(rht_apply(W^T)) outside the
+    rounding-boundary windows [Hadamard-Int4-Accuracy wiki, Hypothesis: A.B = (A.Q)(Q.B), the
+    weights take the rotation offline]."""
+    wl = W.make_workload(name, M=16)
+    bits, G = wl.quant[0]
+    Wt = np.ascontiguousarray(wl.W.T)            # [N, K] fp32
+    plan = lib.Plan.rht(wl.K, wl.signs)
+    codes, scales = guarded_quant(lib, to_device(Wt, False), plan, bits, G)
+    rows = sample_rows(Wt.shape[0], 64, seed=5)
+    idx = rows.tolist()
+    assert_codes_match(codes[idx].cpu().numpy(), scales[idx].cpu().numpy(), Hd.rht_apply(Wt[rows], wl.signs),
+                       bits, G, what=f"W^T {Wt.shape[0]}x{wl.K} int{bits} G={G}")

@@ -7,7 +7,7 @@ import workloads as W
 from oracle import hadamard as Hd
 from oracle import linear as L
 from oracle import quant as Q
-from parity import assert_linear_close, sample_rows, to_device
+from parity import assert_codes_match, assert_linear_close, guarded_linear, guarded_quant, sample_rows, to_device
 
 pytestmark = pytest.mark.gpu
 
@@ -33,7 +33,11 @@ def _dev(a):
 def test_group_partials_exact(lib, M, N, K, G):
     qa, pa, sa = _codes(M + K, M, K, G)
     qw, pw, sw = _codes(N + K + 1, N, K, G)
-    P = lib.w4a4_group_partials(_dev(pa), _dev(pw), G).cpu().numpy()
+    import torch
+    from parity import POISON, Guarded
+    out = Guarded((M, N, K // G), torch.int32, POISON["i32"])
+    P = lib.w4a4_group_partials(_dev(pa), _dev(pw), G, out=out.t).cpu().numpy()
+    out.check()
     assert np.array_equal(P, L.group_partials(qa, qw, G))
 
 
@@ -47,8 +51,8 @@ def test_w4a4_linear_small(lib, M, N, K, G, out):
     import torch
     qa, pa, sa = _codes(M + K + 7, M, K, G)
     qw, pw, sw = _codes(N + K + 9, N, K, G)
-    C = lib.w4a4_linear(_dev(pa), _dev(sa), _dev(pw), _dev(sw), G,
-                        out_dtype=torch.float32 if out == "f32" else torch.bfloat16)
+    C = guarded_linear(lib, lib.w4a4_linear, _dev(pa), _dev(sa), _dev(pw), _dev(sw), G,
+                       torch.float32 if out == "f32" else torch.bfloat16)
     C_ref = L.w4a4_reference(qa, sa, qw, sw, G)
     if out == "f32":
         assert_linear_close(C.cpu().numpy(), C_ref)
@@ -70,33 +74,43 @@ def test_w4a4_empty_M(lib):
 def test_w4a4_workload_oracle_codes(lib, name):
     """Full-size linear on oracle-quantised codes (parity isolates the GEMM; the codes of the
     workload's activation and weight shapes are quantised without rotation to keep the oracle fast)."""
+    import torch
     wl = W.make_workload(name)
     bits, G = wl.quant[0]
     rows = sample_rows(wl.M, 24)
     qa, sa = Q.quantize(wl.A, bits, G)
     qw, sw = Q.quantize(np.ascontiguousarray(wl.W.T), bits, G)
-    C = lib.w4a4_linear(_dev(Q.pack(qa, 4)), _dev(sa), _dev(Q.pack(qw, 4)), _dev(sw), G).cpu().numpy()
+    C = guarded_linear(lib, lib.w4a4_linear, _dev(Q.pack(qa, 4)), _dev(sa), _dev(Q.pack(qw, 4)), _dev(sw), G,
+                       torch.float32).cpu().numpy()
     C_ref = L.w4a4_reference(qa[rows], sa[rows], qw, sw, G)
     assert_linear_close(C[rows], C_ref)
 
 
-def test_w4a4_end_to_end_rotated_pipeline(lib):
-    """GPU rotate+quantise of A and W^T, then the GPU linear: close to the oracle pipeline
-    (codes may differ only at boundary elements) and the page-2 accuracy trend holds."""
+@pytest.mark.parametrize("M", [16, 256])
+def test_w4a4_end_to_end_rotated_pipeline(lib, M):
+    """The whole path on the GPU: rotate + quantise the activations (bf16) and the rows of W^T
+    (fp32, the offline step) with one RHT plan, then the linear. Checked element by element:
+    the GPU codes and scales of both operands equal the oracle's outside the rounding-boundary
+    windows, and the GPU linear on the GPU codes is within 1e-4 of the oracle linear on those
+    same codes. The page-2 accuracy trend (rotation lowers the W4A4 error against the exact
+    product) holds as well [Hadamard-Int4-Accuracy wiki, Hypothesis and Results]."""
     import torch
-    wl = W.make_workload("q_proj_prefill", M=64)
+    wl = W.make_workload("q_proj_prefill", M=M)
     bits, G = wl.quant[0]
+    N = 512                                           # the first 512 output columns of q_proj
+    Wt = np.ascontiguousarray(wl.W.T[:N])             # [N, K]
     plan = lib.Plan.rht(wl.K, wl.signs)
-    Aq, As = lib.rot_quant(to_device(wl.A, True), plan, bits, G)
-    Wq, Ws = lib.rot_quant(to_device(wl.W.T.copy(), False), plan, bits, G)
-    C = lib.w4a4_linear(Aq, As, Wq, Ws, G, out_dtype=torch.bfloat16).float().cpu().numpy()
-    qa, sa = Q.quantize(Hd.rht_apply(wl.A, wl.signs), bits, G)
-    qw, sw = Q.quantize(Hd.rht_apply(wl.W.T, wl.signs), bits, G)
-    C_ref = L.w4a4_reference(qa, sa, qw, sw, G)
-    assert np.linalg.norm(C - C_ref) / np.linalg.norm(C_ref) < 5e-3
-    exact = wl.A.astype(np.float64) @ wl.W.astype(np.float64)
+    Aq, As = guarded_quant(lib, to_device(wl.A, True), plan, bits, G)
+    Wq, Ws = guarded_quant(lib, to_device(Wt, False), plan, bits, G)
+    assert_codes_match(Aq, As, Hd.rht_apply(wl.A, wl.signs), bits, G, what="A int4 G=128")
+    assert_codes_match(Wq, Ws, Hd.rht_apply(Wt, wl.signs), bits, G, what="W^T int4 G=128")
+    C = guarded_linear(lib, lib.w4a4_linear, Aq, As, Wq, Ws, G, torch.float32).cpu().numpy()
+    qa, sa = Q.unpack(Aq.cpu().numpy(), 4, wl.K), As.cpu().numpy()
+    qw, sw = Q.unpack(Wq.cpu().numpy(), 4, wl.K), Ws.cpu().numpy()
+    assert_linear_close(C, L.w4a4_reference(qa, sa, qw, sw, G))
+    exact = wl.A.astype(np.float64) @ wl.W[:, :N].astype(np.float64)
     err_rot = np.linalg.norm(C - exact) / np.linalg.norm(exact)
     qa0, sa0 = Q.quantize(wl.A, bits, G)
-    qw0, sw0 = Q.quantize(wl.W.T, bits, G)
+    qw0, sw0 = Q.quantize(Wt, bits, G)
     err_plain = np.linalg.norm(L.w4a4_reference(qa0, sa0, qw0, sw0, G) - exact) / np.linalg.norm(exact)
     assert err_rot < 0.8 * err_plain

@@ -400,3 +400,42 @@ def test_error_benefit_scales_with_outlier_severity():
         had = L.matmul_q_err(A, B, 4, 4, rot, 128)
         gains.append(plain - had)
     assert gains[1] > gains[0] > 0
+
+
+# ----------------------------------------------------------------------------- plain CPU baseline
+
+@pytest.mark.parametrize("K,G,bits", [(2, 2, 4), (64, 16, 2), (256, 32, 4), (2048, 32, 4), (2048, 128, 4),
+                                      (4096, 64, 2)])
+def test_plain_cpu_baseline_matches_the_oracle(K, G, bits):
+    """The scalar O(K log K) C baseline (fp32 butterflies) gives the oracle's codes and scales
+    (fp64 dense RHT) everywhere outside the 1e-5 rounding-boundary windows, on heavy-tailed rows
+    with outlier channels, with and without signs (the wiki's probe has none)."""
+    from oracle import plain
+    g = W.rng(K + G + bits)
+    A = W.activations(g, 24, K, dist="student_t", t_scale=0.5, outlier_frac=0.01, outlier_scale=50.0, bf16=False)
+    for s in (W.signs(g, K), None):
+        codes, scales = plain.rht_quant(A, s, bits, G)
+        y = Hd.rht_apply(A, s)
+        q_ref, s_ref = Q.quantize(y, bits, G)
+        cflag, gflag = Q.boundary_flags(y, bits, G)
+        assert not ((scales.view(np.uint16) != s_ref.view(np.uint16)) & ~gflag).any()
+        assert not ((Q.unpack(codes, bits, K) != q_ref) & ~cflag).any()
+
+
+def test_plain_cpu_baseline_edge_cases():
+    """Zero rows, scales in the binary16 subnormal range and past its largest finite value (inf
+    scale, zero codes) take the same decisions as the oracle."""
+    from oracle import plain
+    K, G = 256, 32
+    A = np.zeros((4, K), dtype=np.float32)
+    A[1] = W.rng(2).standard_normal(K) * 1e-6
+    A[2] = 3.0e5
+    A[3, 5] = -4.0
+    codes, scales = plain.rht_quant(A, None, 4, G)
+    y = Hd.rht_apply(A, None)
+    q_ref, s_ref = Q.quantize(y, 4, G)
+    cflag, gflag = Q.boundary_flags(y, 4, G)
+    assert np.array_equal(scales.view(np.uint16)[~gflag], s_ref.view(np.uint16)[~gflag])
+    assert not ((Q.unpack(codes, 4, K) != q_ref) & ~cflag).any()
+    # a constant row puts all its energy in coordinate 0 (no signs): group 0's scale overflows to inf
+    assert np.isinf(scales[2, 0].astype(np.float32)) and (Q.unpack(codes, 4, K)[2] == 0).all()
