@@ -306,6 +306,7 @@ def main():
 
     # one period of the buffer rotation in a CUDA graph (warm-up steps run before capture)
     steps_graph = StepGraph(step, NSETS, warm=args.warmup)
+    steps_graph.prepare(args.steps)
     torch.cuda.synchronize(dev)
     if world > 1:
         dist.barrier()
@@ -397,7 +398,7 @@ def main():
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": WORKLOAD_DESC,
                    "global_batch": M * world, "l2": "6 rotating input/output sets (258 MB > 126 MB L2)",
-                   "launch": "timed steps replayed from a CUDA graph holding one 6-step period",
+                   "launch": "every timed step replayed from CUDA graphs (6-step periods plus one remainder graph)",
                    "parallelism": f"dp{world} (independent rows)"},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
                      "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": profiled_traffic("rot_quant_llama32_1b"),
@@ -435,8 +436,8 @@ def _time_loop(fn, n, stream, warm=5):
 class StepGraph:
     """Steps 0 .. period-1 of fn(i) (launching on the current stream) captured in one CUDA
     graph, so that back-to-back steps are timed on the device without per-launch host cost.
-    run(n) issues exactly n steps: n // period graph replays, then the remaining steps
-    launched directly."""
+    run(n) issues exactly n steps: n // period replays of that graph, then one replay of a
+    graph holding steps 0 .. (n % period) - 1 (captured by prepare(n), before timing)."""
 
     def __init__(self, fn, period, warm=3):
         import torch
@@ -444,25 +445,38 @@ class StepGraph:
         for i in range(warm):
             fn(i)
         torch.cuda.synchronize()
-        self.g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(self.g):
-            for i in range(period):
-                fn(i)
-        self.g.replay()
+        self.g = self._capture(period)
+        self.tail = {}
+
+    def _capture(self, k):
+        import torch
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for i in range(k):
+                self.fn(i)
+        g.replay()
         torch.cuda.synchronize()
+        return g
+
+    def prepare(self, n):
+        rem = n % self.period
+        if rem and rem not in self.tail:
+            self.tail[rem] = self._capture(rem)
 
     def run(self, n):
+        self.prepare(n)
         reps, rem = divmod(n, self.period)
         for _ in range(reps):
             self.g.replay()
-        for i in range(rem):
-            self.fn(i)
+        if rem:
+            self.tail[rem].replay()
 
 
 def _graph_time(fn, n, period, warm=3):
     """Seconds per step of fn(i), n steps replayed from a CUDA graph of `period` steps."""
     import torch
     sg = StepGraph(fn, period, warm)
+    sg.prepare(n)
     stream = torch.cuda.current_stream()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
