@@ -6,7 +6,8 @@ device memory and the current CUDA stream. Importing this package without the bu
 library raises ImportError; there is no CPU fallback.
 
 Names follow the C ABI: ``Plan`` (rot_plan_create / rot_plan_destroy), ``rot_apply``,
-``rot_quant``, ``rot_dequant``, ``w4a4_linear``, ``w4a4_group_partials``,
+``rot_quant``, ``rot_dequant``, ``w4a4_linear``, ``w4a4_group_partials``, ``w4a8_linear``,
+``w4a8_group_partials``,
 ``harp_givens_blocks``, ``harp_qr_block``, ``check_device``.
 """
 from __future__ import annotations
@@ -41,16 +42,27 @@ _lib.rot_dequant.argtypes = [_vp, _vp, _i64, _vp, _int, _int, _int, _vp, _vp]
 _lib.w4a4_linear.argtypes = [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _int, _vp, _int, _vp]
 _lib.w4a4_linear_noalloc.argtypes = [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _int, _vp, _int, _vp]
 _lib.w4a4_group_partials.argtypes = [_vp, _vp, _i64, _i64, _i64, _int, _vp, _vp]
+_lib.w4a8_linear.argtypes = [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _int, _vp, _int, _vp]
+_lib.w4a4_linear_rot.argtypes = [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _int, _vp, _vp, _int, _vp]
+_lib.w4a4_linear_act_workspace.argtypes = [_i64, _i64, _int, C.POINTER(C.c_size_t)]
+_lib.w4a4_linear_act.argtypes = [_vp, _int, _i64, _i64, _vp, _vp, _vp, _i64, _int, _vp, _int, _vp, C.c_size_t, _vp]
+_lib.w4a8_group_partials.argtypes = [_vp, _vp, _i64, _i64, _i64, _int, _vp, _vp]
 _lib.w4a4_tile_plan.argtypes = [_i64, _i64, _i64, _int, _int, _int, C.POINTER(_i64)]
 _lib.rot_harp_givens_blocks.argtypes = [C.POINTER(C.c_double), _i64, C.POINTER(C.c_float)]
 _lib.rot_harp_qr_block.argtypes = [C.POINTER(C.c_double), _int, C.POINTER(C.c_float)]
+_lib.rot_harp_cayley_block.argtypes = [C.POINTER(C.c_double), _int, C.POINTER(C.c_float), C.POINTER(C.c_float)]
+_lib.rot_plan_create_q8.argtypes = [C.POINTER(_vp), _int, _int, C.POINTER(_int), C.POINTER(C.POINTER(C.c_int8)),
+                                    C.POINTER(C.c_float), C.POINTER(_i64), C.POINTER(C.POINTER(C.c_float)),
+                                    C.POINTER(C.POINTER(_i32)), C.POINTER(C.c_int8)]
 _lib.rot_check_device.argtypes = []
 _lib.rot_test_inject.argtypes = [_int, _i64]
 _lib.rot_last_error.restype = C.c_char_p
 _lib.rot_version.restype = C.c_char_p
 for _f in ("rot_plan_create", "rot_plan_destroy", "rot_plan_info", "rot_apply", "rot_quant", "rot_dequant",
-           "w4a4_linear", "w4a4_linear_noalloc", "w4a4_group_partials", "w4a4_tile_plan", "rot_harp_givens_blocks",
-           "rot_harp_qr_block", "rot_check_device", "rot_test_inject"):
+           "w4a4_linear", "w4a4_linear_noalloc", "w4a4_group_partials", "w4a8_linear", "w4a8_group_partials",
+           "w4a4_linear_rot", "w4a4_linear_act_workspace", "w4a4_linear_act",
+           "w4a4_tile_plan", "rot_harp_givens_blocks",
+           "rot_harp_qr_block", "rot_check_device", "rot_test_inject", "rot_harp_cayley_block", "rot_plan_create_q8"):
     getattr(_lib, _f).restype = _int
 
 
@@ -179,6 +191,59 @@ class Plan:
         self._h = h
 
     @classmethod
+    def q8(cls, K: int, radices, codes, scales, mixers=None, perms=None, signs=None) -> "Plan":
+        """Plan from int8-stored HARP parameters (rot_plan_create_q8): codes[t] None or int8
+        ([n_blocks] for radix 2, [n_blocks, b(b-1)/2] otherwise), scales[t] fp32 (theta =
+        code * scale), mixers[t] None or a b x b fp32 base mixer, perms / signs as for Plan."""
+        import torch  # noqa: F401
+        m = len(radices)
+        radices = [int(b) for b in radices]
+        keep = []
+        cp = (C.POINTER(C.c_int8) * m)()
+        nb = (_i64 * m)()
+        for t, q in enumerate(codes):
+            if q is None:
+                cp[t] = C.POINTER(C.c_int8)()
+            else:
+                a = np.ascontiguousarray(q, dtype=np.int8)
+                keep.append(a)
+                cp[t] = a.ctypes.data_as(C.POINTER(C.c_int8))
+                nb[t] = a.shape[0]
+        sc = (C.c_float * m)(*[float(x) for x in scales])
+        mp = None
+        if mixers is not None and any(x is not None for x in mixers):
+            mp = (C.POINTER(C.c_float) * m)()
+            for t, g in enumerate(mixers):
+                if g is None:
+                    mp[t] = C.POINTER(C.c_float)()
+                else:
+                    a = np.ascontiguousarray(g, dtype=np.float32)
+                    keep.append(a)
+                    mp[t] = a.ctypes.data_as(C.POINTER(C.c_float))
+        pp = None
+        if perms is not None and any(p is not None for p in perms):
+            pp = (C.POINTER(_i32) * m)()
+            for t, P in enumerate(perms):
+                if P is None:
+                    pp[t] = C.POINTER(_i32)()
+                else:
+                    a = np.ascontiguousarray(P, dtype=np.int32)
+                    keep.append(a)
+                    pp[t] = a.ctypes.data_as(C.POINTER(_i32))
+        sg = None
+        if signs is not None:
+            sgn = np.ascontiguousarray(signs, dtype=np.int8)
+            keep.append(sgn)
+            sg = sgn.ctypes.data_as(C.POINTER(C.c_int8))
+        h = _vp()
+        _check(_lib.rot_plan_create_q8(C.byref(h), int(K), m, (_int * m)(*radices), cp, sc, nb, mp, pp, sg))
+        self = cls.__new__(cls)
+        self.K = int(K)
+        self.radices = radices
+        self._h = h
+        return self
+
+    @classmethod
     def rht(cls, K: int, signs=None) -> "Plan":
         """Randomized Hadamard transform of size K (power of two): radix-2 base mixers."""
         n = int(K).bit_length() - 1
@@ -222,7 +287,8 @@ def rot_apply(A, plan: Plan, *, inverse: bool = False, out=None, stream=None):
 
 
 def rot_quant(A, plan: Plan, bits: int, G: int, *, codes=None, scales=None, stream=None):
-    """Fused rotate + group quantise + pack. Returns (codes uint8 [M, K*bits/8], scales fp16 [M, K/G])."""
+    """Fused rotate + group quantise + pack (bits 2, 4 or 8). Returns (codes uint8 [M, K*bits/8],
+    scales fp16 [M, K/G]); int8 codes can be viewed as torch.int8 for w4a8_linear."""
     import torch
     pa = _arg(A, "A", dtype=(torch.bfloat16, torch.float32), strided_rows=True)
     M = A.shape[0]
@@ -280,6 +346,48 @@ def w4a4_linear(Aq, As, Wq, Ws, G: int, *, out_dtype=None, out=None, stream=None
     return out
 
 
+def w4a4_linear_rot(Aq, As, Wq, Ws, G: int, out_plan: Plan, *, out_dtype=None, out=None, stream=None):
+    """Two-sided processor: the linear on weights prepared as B~ = T B U^T, then every output row
+    returned to c = U^T c~ with the output-side plan U (size N)."""
+    import torch
+    M, N, K, ptrs = _w4a4_args(Aq, As, Wq, Ws, G)
+    if out is None:
+        out = torch.empty((M, N), dtype=out_dtype or torch.float32, device=Wq.device)
+    po = _arg(out, "out", dtype=(torch.float32, torch.bfloat16), shape=(M, N))
+    cd = ROT_BF16 if out.dtype == torch.bfloat16 else ROT_F32
+    _check(_lib.w4a4_linear_rot(*ptrs, M, N, K, G, out_plan.handle, po, cd, _stream(stream)))
+    return out
+
+
+def w4a4_linear_act_workspace(M: int, K: int, G: int) -> int:
+    n = C.c_size_t()
+    _check(_lib.w4a4_linear_act_workspace(M, K, G, C.byref(n)))
+    return int(n.value)
+
+
+def w4a4_linear_act(A, plan: Plan, Wq, Ws, G: int, *, out_dtype=None, out=None, workspace=None, stream=None):
+    """rot_quant of the activations A (bf16/fp32 [M, >=K]) into a workspace, then the linear.
+    Returns C; the workspace (uint8, allocated here if not given) holds the codes and scales."""
+    import torch
+    pa = _arg(A, "A", dtype=(torch.bfloat16, torch.float32), strided_rows=True)
+    pw = _arg(Wq, "Wq", dtype=torch.uint8)
+    M, K, N = A.shape[0], plan.K, Wq.shape[0]
+    if Wq.dim() != 2 or Wq.shape[1] * 2 != K:
+        raise RotError(ROT_EINVAL, f"Wq must be [N, {K // 2}]")
+    ps_w = _arg(Ws, "Ws", dtype=torch.float16, shape=(N, K // G) if G > 0 and K % G == 0 else None)
+    nbytes = w4a4_linear_act_workspace(M, K, G)
+    if workspace is None:
+        workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=A.device)
+    pws = _arg(workspace, "workspace", dtype=torch.uint8)
+    if out is None:
+        out = torch.empty((M, N), dtype=out_dtype or torch.float32, device=A.device)
+    po = _arg(out, "out", dtype=(torch.float32, torch.bfloat16), shape=(M, N))
+    cd = ROT_BF16 if out.dtype == torch.bfloat16 else ROT_F32
+    _check(_lib.w4a4_linear_act(pa, _dtype_code(A), M, A.stride(0), plan.handle, pw, ps_w, N, G, po, cd, pws,
+                                workspace.numel(), _stream(stream)))
+    return out
+
+
 def w4a4_linear_noalloc(Aq, As, Wq, Ws, G: int, *, out_dtype=None, out=None, stream=None):
     """w4a4_linear that never allocates device memory (static split-K buffer; see the header)."""
     import torch
@@ -300,6 +408,47 @@ def w4a4_group_partials(Aq, Wq, G: int, *, out=None, stream=None):
         out = torch.empty((M, N, K // G), dtype=torch.int32, device=Wq.device)
     po = _arg(out, "out", dtype=torch.int32, shape=(M, N, K // G))
     _check(_lib.w4a4_group_partials(ptrs[0], ptrs[2], M, N, K, G, po, _stream(stream)))
+    return out
+
+
+def _w4a8_args(Aq, As, Wq, Ws, G: int):
+    """Shapes (M, N, K) and checked addresses of the W4A8 operands (int8 Aq [M, K]; As / Ws may be None)."""
+    import torch
+    pw = _arg(Wq, "Wq", dtype=torch.uint8)
+    if Wq.dim() != 2:
+        raise RotError(ROT_EINVAL, "Wq must be 2-D [N, K/2]")
+    N, K = Wq.shape[0], Wq.shape[1] * 2
+    if G <= 0 or K % G != 0:
+        raise RotError(ROT_EINVAL, f"G = {G} must divide K = {K}")
+    pa = _arg(Aq, "Aq", dtype=(torch.int8, torch.uint8))
+    if Aq.dim() != 2 or Aq.shape[1] != K:
+        raise RotError(ROT_EINVAL, f"Aq must be int8 [M, {K}]")
+    M = Aq.shape[0]
+    ps_a = _arg(As, "As", dtype=torch.float16, shape=(M, K // G)) if As is not None else C.c_void_p(0)
+    ps_w = _arg(Ws, "Ws", dtype=torch.float16, shape=(N, K // G)) if Ws is not None else C.c_void_p(0)
+    return M, N, K, (pa, ps_a, pw, ps_w)
+
+
+def w4a8_linear(Aq, As, Wq, Ws, G: int, *, out_dtype=None, out=None, stream=None):
+    """C = sum_g sA sW (qA qW^T)_g for int8 codes Aq [M, K] (rot_quant bits=8) and int4 Wq [N, K/2]."""
+    import torch
+    M, N, K, ptrs = _w4a8_args(Aq, As, Wq, Ws, G)
+    if out is None:
+        out = torch.empty((M, N), dtype=out_dtype or torch.float32, device=Wq.device)
+    po = _arg(out, "out", dtype=(torch.float32, torch.bfloat16), shape=(M, N))
+    cd = ROT_BF16 if out.dtype == torch.bfloat16 else ROT_F32
+    _check(_lib.w4a8_linear(*ptrs, M, N, K, G, po, cd, _stream(stream)))
+    return out
+
+
+def w4a8_group_partials(Aq, Wq, G: int, *, out=None, stream=None):
+    """Exact int32 group sums P[m, n, g] of the W4A8 contraction."""
+    import torch
+    M, N, K, ptrs = _w4a8_args(Aq, None, Wq, None, G)
+    if out is None:
+        out = torch.empty((M, N, K // G), dtype=torch.int32, device=Wq.device)
+    po = _arg(out, "out", dtype=torch.int32, shape=(M, N, K // G))
+    _check(_lib.w4a8_group_partials(ptrs[0], ptrs[2], M, N, K, G, po, _stream(stream)))
     return out
 
 
@@ -328,6 +477,27 @@ def harp_qr_block(g) -> np.ndarray:
     _check(_lib.rot_harp_qr_block(a.ctypes.data_as(C.POINTER(C.c_double)), b,
                                   out.ctypes.data_as(C.POINTER(C.c_float))))
     return out
+
+
+def harp_cayley_block(params, b: int, mixer=None) -> np.ndarray:
+    """Host: B = Q(theta) G (Cayley map of the b(b-1)/2 parameters times the mixer), float32 [b, b]."""
+    p = np.ascontiguousarray(params, dtype=np.float64)
+    out = np.empty((b, b), dtype=np.float32)
+    mx = None
+    if mixer is not None:
+        mx = np.ascontiguousarray(mixer, dtype=np.float32)
+    _check(_lib.rot_harp_cayley_block(p.ctypes.data_as(C.POINTER(C.c_double)), int(b),
+                                      mx.ctypes.data_as(C.POINTER(C.c_float)) if mx is not None else None,
+                                      out.ctypes.data_as(C.POINTER(C.c_float))))
+    return out
+
+
+def harp_q8_plan(draws, signs) -> Plan:
+    """Plan of an int8-stored HARP processor (``workloads.harp_q8_draws``): the fallback mixers of
+    non-power-of-two radices are the library's QR of the drawn Gaussians."""
+    mixers = [None if gm is None else harp_qr_block(gm) for gm in draws.mixer_gaussians]
+    K = int(np.prod(draws.radices))
+    return Plan.q8(K, draws.radices, draws.codes, draws.scales, mixers, draws.perms, signs)
 
 
 def harp_plan(draws, signs, variant: str) -> Plan:

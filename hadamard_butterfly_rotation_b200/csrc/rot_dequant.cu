@@ -1,6 +1,6 @@
-// Dequantisation x_hat = q * s of packed int4 / int2 codes with binary16 group scales
+// Dequantisation x_hat = q * s of packed int8 / int4 / int2 codes with binary16 group scales
 // [Hadamard-Int4-Accuracy wiki, Method: q_dequant_vec quantise -> dequantise].
-// One thread per 32-bit code word (8 int4 or 16 int2 codes); fp32 output rows.
+// One thread per 32-bit code word (4 int8, 8 int4 or 16 int2 codes); fp32 output rows.
 #include "rot_internal.cuh"
 
 namespace rotb {
@@ -40,7 +40,9 @@ rot_status dequant_launch(const uint8_t* codes, const uint16_t* scales, int64_t 
   const int64_t n_words = M * (K / cpw);
   if (n_words == 0) return ROT_OK;
   const int64_t grid = std::min<int64_t>((n_words + 255) / 256, (int64_t)sm_count() * 8);
-  if (bits == 4)
+  if (bits == 8)
+    dequant_kernel<8><<<(unsigned)grid, 256, 0, s>>>(reinterpret_cast<const uint32_t*>(codes), scales, n_words, K, G, out);
+  else if (bits == 4)
     dequant_kernel<4><<<(unsigned)grid, 256, 0, s>>>(reinterpret_cast<const uint32_t*>(codes), scales, n_words, K, G, out);
   else
     dequant_kernel<2><<<(unsigned)grid, 256, 0, s>>>(reinterpret_cast<const uint32_t*>(codes), scales, n_words, K, G, out);

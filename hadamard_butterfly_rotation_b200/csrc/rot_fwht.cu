@@ -147,6 +147,10 @@ __device__ __forceinline__ uint32_t pack8_int4(const uint32_t (&t)[8]) {
   const uint32_t x45 = t[5] * 16u + t[4], x67 = t[7] * 16u + t[6];
   return prmt(prmt(x01, x23, 0x0040u), prmt(x45, x67, 0x0040u), 0x5410u) ^ 0x88888888u;
 }
+// Pack 4 offset codes (low bytes of t[0..3], each 128 + q) into one int8 word, two's complement.
+__device__ __forceinline__ uint32_t pack4_int8(const uint32_t (&t)[4]) {
+  return prmt(prmt(t[0], t[1], 0x0040u), prmt(t[2], t[3], 0x0040u), 0x5410u) ^ 0x80808080u;
+}
 // Pack 16 offset codes (each 2 + q) into one int2 word: byte j holds codes 4j .. 4j+3.
 __device__ __forceinline__ uint32_t pack16_int2(const uint32_t (&t)[16]) {
   uint32_t b[4];
@@ -156,6 +160,10 @@ __device__ __forceinline__ uint32_t pack16_int2(const uint32_t (&t)[16]) {
 }
 
 __device__ int g_fwht_error = 0;
+
+#ifndef ROT_STAGE_SLEEP
+#define ROT_STAGE_SLEEP 0
+#endif
 
 __device__ __forceinline__ uint32_t smem_addr(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -177,6 +185,9 @@ __device__ __forceinline__ bool stage_wait(uint64_t* bar, uint32_t parity, unsig
         : "r"(addr), "r"(parity)
         : "memory");
     if (done) return true;
+#if ROT_STAGE_SLEEP > 0
+    __nanosleep(ROT_STAGE_SLEEP);
+#endif
     if ((it & 255) == 255) {
       unsigned long long now;
       asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(now));
@@ -216,8 +227,8 @@ __device__ __forceinline__ void stage_pairs(float2 (&xp)[NP], int b) {
 // packed codes and scales. GT > 0: compile-time group size; GT == 0: runtime a.G.
 template <int LOGN, int BITS, int GT, int E, int TPC>
 __device__ __forceinline__ void quantise_store(const Args& a, const float2 (&xp)[E / 2], int64_t row, int c0, int t) {
-  constexpr float QMAX = BITS == 4 ? 7.0f : 1.0f;
-  constexpr float MAGIC = BITS == 4 ? 8388616.0f : 8388610.0f;  // 2^23 + qmax + 1
+  constexpr float QMAX = qmax_of_bits(BITS);
+  constexpr float MAGIC = magic_of_bits(BITS);  // 2^23 + qmax + 1
   constexpr int CPW = 32 / BITS;   // codes per 32-bit word
   constexpr int NWD = E / CPW;     // words per thread
   uint16_t* srow = a.scales + row * a.ngroups;
@@ -279,7 +290,8 @@ __device__ __forceinline__ void quantise_store(const Args& a, const float2 (&xp)
           tt[j] = __float_as_uint(r.x);
           tt[j + 1] = __float_as_uint(r.y);
         }
-        if constexpr (BITS == 4) words[w] = pack8_int4(*reinterpret_cast<const uint32_t(*)[8]>(tt));
+        if constexpr (BITS == 8) words[w] = pack4_int8(*reinterpret_cast<const uint32_t(*)[4]>(tt));
+        else if constexpr (BITS == 4) words[w] = pack8_int4(*reinterpret_cast<const uint32_t(*)[8]>(tt));
         else words[w] = pack16_int2(*reinterpret_cast<const uint32_t(*)[16]>(tt));
       }
     } else {
@@ -292,7 +304,8 @@ __device__ __forceinline__ void quantise_store(const Args& a, const float2 (&xp)
           tt[j] = code_magic_clamped(xp[(CPW * w + j) / 2].x, fg, QMAX, MAGIC);
           tt[j + 1] = code_magic_clamped(xp[(CPW * w + j) / 2].y, fg, QMAX, MAGIC);
         }
-        if constexpr (BITS == 4) words[w] = pack8_int4(*reinterpret_cast<const uint32_t(*)[8]>(tt));
+        if constexpr (BITS == 8) words[w] = pack4_int8(*reinterpret_cast<const uint32_t(*)[4]>(tt));
+        else if constexpr (BITS == 4) words[w] = pack8_int4(*reinterpret_cast<const uint32_t(*)[8]>(tt));
         else words[w] = pack16_int2(*reinterpret_cast<const uint32_t(*)[16]>(tt));
       }
     }
@@ -343,7 +356,7 @@ __device__ __forceinline__ void quantise_store(const Args& a, const float2 (&xp)
     const float2 mg = make_float2(MAGIC, MAGIC);
 #pragma unroll
     for (int w = 0; w < NWD; ++w) {
-      const int gi = w * (CPW / 8);
+      const int gi = (w * CPW) / 8;        // granule of 8 codes holding the word's first code
       uint32_t tt[CPW];
       if (!slow[gi]) {
         const float2 ff = make_float2(fw[gi], fw[gi]);
@@ -360,7 +373,8 @@ __device__ __forceinline__ void quantise_store(const Args& a, const float2 (&xp)
           tt[j + 1] = code_magic_clamped(xp[(CPW * w + j) / 2].y, fw[gi], QMAX, MAGIC);
         }
       }
-      if constexpr (BITS == 4) words[w] = pack8_int4(*reinterpret_cast<const uint32_t(*)[8]>(tt));
+      if constexpr (BITS == 8) words[w] = pack4_int8(*reinterpret_cast<const uint32_t(*)[4]>(tt));
+      else if constexpr (BITS == 4) words[w] = pack8_int4(*reinterpret_cast<const uint32_t(*)[8]>(tt));
       else words[w] = pack16_int2(*reinterpret_cast<const uint32_t(*)[16]>(tt));
     }
   }
@@ -759,6 +773,143 @@ __global__ void __launch_bounds__(MMA_THREADS, 1) fwht_mma_kernel(const Args a) 
   }
 }
 
+// ---------------------------------------------------------------- double-buffered variant
+// The same per-chunk work as fwht_mma_kernel, with two staging buffers per warp so that the
+// copy of the chunk two units ahead is in flight while the warp computes the current one and
+// the next. A warp's 12 KB region is [S0 | X | S1] (4 KB each): chunk i is staged in S_(i&1),
+// and its fp32 transpose uses the 8 KB window S_(i&1) + X (S0+X or X+S1, contiguous), so the
+// other staging buffer is never touched while its copy is in flight. The copy into S_(i&1) is
+// issued as soon as the transpose has been read back.
+#ifndef ROT_DB_WARPS
+#define ROT_DB_WARPS 18
+#endif
+constexpr int DB_WARPS = ROT_DB_WARPS;         // chunk slots (warps) per CTA
+constexpr int DB_THREADS = DB_WARPS * 32;
+constexpr int DB_REGION = 3 * 1024;            // floats per warp
+
+size_t db_smem_bytes(int K) {
+  return (size_t)DB_WARPS * DB_REGION * 4 + (size_t)DB_WARPS * 2 * 8 + (size_t)(K / 2) * 4;
+}
+
+template <int BITS, int GT>
+__global__ void __launch_bounds__(DB_THREADS, 1) fwht_mma_db_kernel(const Args a) {
+  constexpr int N = 2048, NP = 32;
+  extern __shared__ __align__(128) float smem[];
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + DB_WARPS * DB_REGION);
+  uint32_t* smf = reinterpret_cast<uint32_t*>(bars + 2 * DB_WARPS);  // sign masks, fragment order
+
+  const int slot = threadIdx.x >> 5;
+  const int l = threadIdx.x & 31;
+  const int g = l >> 2, c = l & 3;
+  float* region = smem + slot * DB_REGION;
+  uint64_t* bar = bars + 2 * slot;
+  const bool has_signs = a.signmask != nullptr;
+
+  const int64_t units = a.M * a.chunks;
+  const int64_t stride = (int64_t)gridDim.x * DB_WARPS;
+  int64_t u = (int64_t)blockIdx.x * DB_WARPS + slot;
+  const int64_t drow = stride / a.chunks;
+  const int dchunk = (int)(stride - drow * a.chunks);
+  int64_t row = u / a.chunks;
+  int chunk = (int)(u - row * a.chunks);
+  auto src_of = [&](int64_t r, int ch) -> const void* {
+    return static_cast<const uint8_t*>(a.A) + ((int64_t)r * a.lda + (int64_t)ch * N) * 2;
+  };
+  auto advance = [&](int64_t& r, int& ch) {
+    r += drow;
+    ch += dchunk;
+    if (ch >= a.chunks) { ch -= a.chunks; ++r; }
+  };
+  // cursor of the unit whose copy is issued next (two units ahead of the current one)
+  int64_t lrow = row;
+  int lchunk = chunk;
+  advance(lrow, lchunk);
+
+  if (l == 0) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_addr(bar)) : "memory");
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_addr(bar + 1)) : "memory");
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (has_signs) {
+    for (int idx = threadIdx.x; idx < a.K / 2; idx += DB_THREADS) {
+      const int ch = idx >> 10, i = (idx >> 7) & 7, ln = (idx >> 2) & 31, r = idx & 3;
+      const int off = ch * N + 8 * (ln >> 2) + 2 * (ln & 3) + 256 * i + ((r & 1) << 7) + ((r & 2) << 5);
+      smf[idx] = a.signmask[off >> 1];
+    }
+  }
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  // (testing hook: slot 0 of CTA 0 issues neither first copy, so nothing is in flight when it gives up)
+  if (l == 0 && !(a.skip_first && blockIdx.x == 0 && slot == 0)) {
+    if (u < units) stage_issue(bar, region, src_of(row, chunk), N * 2);
+    if (u + stride < units) stage_issue(bar + 1, region + 2048, src_of(lrow, lchunk), N * 2);
+  }
+  advance(lrow, lchunk);
+  __syncthreads();
+
+  uint32_t hb[2][2];
+#pragma unroll
+  for (int q = 0; q < 2; ++q) {
+    const int o = 8 * q + g;
+    hb[q][0] = h16_bf16(2 * c, o) | (h16_bf16(2 * c + 1, o) << 16);
+    hb[q][1] = h16_bf16(2 * c + 8, o) | (h16_bf16(2 * c + 9, o) << 16);
+  }
+  const uint32_t lrow_b = (uint32_t)(8 * (l & 7) + ((l >> 3) & 1) * 128 + ((l >> 4) & 1) * 64) * 2;
+  const uint32_t rbase = smem_addr(region);
+  const int abase = 2 * c + 8 * g;
+  uint32_t par = 0;            // bit b: phase parity of staging buffer b
+  int b = 0;
+
+  for (; u < units; u += stride) {
+    const int cbase = chunk * N;
+    float2 xp[NP];
+    if (!stage_wait(bar + b, (par >> b) & 1u, a.wait_ns)) break;
+    par ^= 1u << b;
+    const uint32_t sbase = rbase + (uint32_t)b * 8192u;      // staged bf16 chunk (S0 or S1)
+    float* win = region + b * 1024;                          // transpose window (S0+X or X+S1)
+
+    const uint4* sm4 = reinterpret_cast<const uint4*>(smf + (cbase >> 1)) + l;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      uint32_t af[4];
+      ldsm_x4(sbase + lrow_b + i * 512, af);
+      if (has_signs) {
+        const uint4 m = sm4[i * 32];
+        af[0] ^= m.x; af[1] ^= m.y; af[2] ^= m.z; af[3] ^= m.w;
+      }
+      mma_h16(xp[4 * i + 0], xp[4 * i + 2], af, hb[0][0], hb[0][1]);
+      mma_h16(xp[4 * i + 1], xp[4 * i + 3], af, hb[1][0], hb[1][1]);
+    }
+#pragma unroll
+    for (int bb = 1; bb < 5; ++bb) stage_pairs<NP>(xp, bb);
+
+    __syncwarp();   // every lane's ldmatrix reads of the staged chunk are done
+#pragma unroll
+    for (int p = 0; p < NP; ++p)
+      *reinterpret_cast<float2*>(win + ((abase ^ ((p & 7) << 2)) + 64 * p)) = xp[p];
+    __syncwarp();
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      const float4 q = *reinterpret_cast<const float4*>(win + 64 * l + ((4 * j) ^ ((l & 7) << 2)));
+      xp[2 * j] = make_float2(q.x, q.y);
+      xp[2 * j + 1] = make_float2(q.z, q.w);
+    }
+    // the window is read back: the staging buffer of this chunk takes the copy two units ahead
+    if (u + 2 * stride < units) {
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      __syncwarp();
+      if (l == 0) stage_issue(bar + b, region + b * 2048, src_of(lrow, lchunk), N * 2);
+    }
+    advance(lrow, lchunk);
+#pragma unroll
+    for (int bb = 2; bb < 5; ++bb) stage_pairs<NP>(xp, bb);
+    const int64_t cur_row = row;
+    advance(row, chunk);
+    b ^= 1;
+    quantise_store<11, BITS, GT, 64, 32>(a, xp, cur_row, cbase + 64 * l, l);
+  }
+}
+
 size_t mma_smem_bytes(int K) {
   return (size_t)MMA_SLOTS * MMA_SSTRIDE * 4 + (size_t)MMA_SLOTS * 8 + (size_t)(K / 2) * 4;
 }
@@ -837,8 +988,48 @@ bool tc_enabled() {
   return on;
 }
 
+// Double-buffered staging for the tensor-core kernel (ROT_B200_DB=0 selects the single-buffer one).
+bool db_enabled() {
+  static const bool on = [] {
+    const char* e = std::getenv("ROT_B200_DB");
+    return !(e && e[0] == '0');
+  }();
+  return on;
+}
+
+template <int BITS, int GT>
+rot_status launch_mma_db(const Args& a, cudaStream_t s) {
+  const size_t smem = db_smem_bytes(a.K);
+  auto kern = fwht_mma_db_kernel<BITS, GT>;
+  static int configured[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !configured[dev]) {
+    ROT_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024));
+    configured[dev] = 1;
+  }
+  const int64_t units = a.M * a.chunks;
+  int64_t grid = (units + DB_WARPS - 1) / DB_WARPS;
+  const int64_t cap = (int64_t)sm_count();
+  if (grid > cap) grid = cap;
+  if (grid < 1) return ROT_OK;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3(DB_THREADS);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl_enabled() ? 1 : 0;
+  ROT_CUDA_TRY(cudaLaunchKernelEx(&cfg, kern, a));
+  return ROT_OK;
+}
+
 template <int BITS, int GT>
 rot_status launch_mma(const Args& a, cudaStream_t s) {
+  if (db_enabled() && db_smem_bytes(a.K) <= 227 * 1024) return launch_mma_db<BITS, GT>(a, s);
   const size_t smem = mma_smem_bytes(a.K);
   if (smem > 227 * 1024) return set_error(ROT_EUNSUPPORTED, "fused rotation: sign table too large for shared memory");
   auto kern = fwht_mma_kernel<BITS, GT>;
@@ -963,12 +1154,15 @@ rot_status fwht_quant(const rot_plan_s* p, const void* A, int a_dtype, int64_t M
   a.ngroups = p->K / G;
   {
     const double nd = 1.0 / std::sqrt((double)(1 << p->chunk_log2));
-    a.cdiv = (float)(nd / (bits == 4 ? 7.0 : 1.0));
+    a.cdiv = (float)(nd / (bits == 8 ? 127.0 : bits == 4 ? 7.0 : 1.0));
     a.cf = (float)(nd * (1.0 + 0x1p-22));
   }
   const int n = p->chunk_log2;
-  if (a_dtype == ROT_BF16)
+  if (a_dtype == ROT_BF16) {
+    if (bits == 8) return dispatch_logn<true, MODE_QUANT, 8>(n, a, s);
     return bits == 4 ? dispatch_logn<true, MODE_QUANT, 4>(n, a, s) : dispatch_logn<true, MODE_QUANT, 2>(n, a, s);
+  }
+  if (bits == 8) return dispatch_logn<false, MODE_QUANT, 8>(n, a, s);
   return bits == 4 ? dispatch_logn<false, MODE_QUANT, 4>(n, a, s) : dispatch_logn<false, MODE_QUANT, 2>(n, a, s);
 }
 

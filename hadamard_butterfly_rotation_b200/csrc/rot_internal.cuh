@@ -74,15 +74,16 @@ rot_status stages_quant(const rot_plan_s* p, const void* A, int a_dtype, int64_t
 // dequantisation (rot_dequant.cu)
 rot_status dequant_launch(const uint8_t* codes, const uint16_t* scales, int64_t M, int K, int bits,
                           int G, float* out, cudaStream_t s);
-// W4A4 linear (w4a4_linear.cu)
+// W4A4 / W4A8 linear (w4a4_linear.cu); a8: Aq holds int8 codes [M, K] instead of packed int4
 // split-K accumulation: `scratch` (scratch_floats floats) if non-null, else a stream-ordered
 // temporary; only used for bf16 output on the split path
 constexpr int64_t W4A4_NOALLOC_SCRATCH_FLOATS = int64_t(1) << 20;
 rot_status w4a4_launch(const uint8_t* Aq, const uint16_t* As, const uint8_t* Wq,
                        const uint16_t* Ws, int64_t M, int64_t N, int64_t K, int G, void* C,
                        int c_dtype, int32_t* partials, cudaStream_t s, float* scratch = nullptr,
-                       int64_t scratch_floats = 0);
+                       int64_t scratch_floats = 0, bool a8 = false, bool pdl = false);
 rot_status w4a4_noalloc_scratch(float** out);
+rot_status f32_to_bf16_launch(const float* src, void* dst, int64_t n, cudaStream_t s);
 struct W4A4TilePlan {
   int64_t tiles_m, tiles_n, units, grid;
   int splits, kb_per_split;
@@ -136,6 +137,17 @@ __device__ __forceinline__ uint16_t group_scale(float m_z, float c_div, float c_
   asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(s));
   *f = (s > 0.0f && s <= 65504.0f) ? r * c_f : 0.0f;
   return (uint16_t)hb;
+}
+
+// Per bit width: qmax = 2^(bits-1) - 1, the rounding constant 2^23 + qmax + 1 (its low bits
+// hold the offset code qmax + 1 + q after an fma), and the XOR that turns packed offset codes
+// (qmax + 1 + q, the high bit of each field set for q >= 0) into two's complement fields.
+__host__ __device__ constexpr float qmax_of_bits(int bits) { return bits == 8 ? 127.0f : bits == 4 ? 7.0f : 1.0f; }
+__host__ __device__ constexpr float magic_of_bits(int bits) {
+  return bits == 8 ? 8388736.0f : bits == 4 ? 8388616.0f : 8388610.0f;
+}
+__host__ __device__ constexpr uint32_t offset_xor_of_bits(int bits) {
+  return bits == 8 ? 0x80808080u : bits == 4 ? 0x88888888u : 0xAAAAAAAAu;
 }
 
 // Offset code u = qmax + 1 + rne(v) in the low bits of the result (magic-number rounding);

@@ -8,6 +8,7 @@
 // Sylvester-Hadamard stages over the leading digits are, per contiguous chunk of
 // 2^n coordinates, a signed Walsh-Hadamard transform [HARP abstract: the processor
 // initialises to the RHT]; those run on the fused butterfly kernel.
+#include <algorithm>
 #include <atomic>
 #include <cmath>
 #include <cstring>
@@ -265,6 +266,165 @@ extern "C" rot_status rot_harp_givens_blocks(const double* theta, int64_t n, flo
     out[4 * i + 1] = (float)((c + s) * h);
     out[4 * i + 2] = (float)((s + c) * h);
     out[4 * i + 3] = (float)((s - c) * h);
+  }
+  return ROT_OK;
+}
+
+// Cayley map Q = (I + S)^{-1} (I - S) of the skew-symmetric S with strictly upper entries
+// params (row-major order), times the base mixer G: B = Q G [HARP gist.science summary, 2.2:
+// B = Q(theta) G, Q a Cayley map for b > 2]. I + S is never singular (the eigenvalues of S are
+// imaginary); Gaussian elimination with partial pivoting in double.
+extern "C" rot_status rot_harp_cayley_block(const double* params, int b, const float* mixer, float* out) {
+  if (b < 2 || !out || (!params && b > 1)) return set_error(ROT_EINVAL, "rot_harp_cayley_block: bad arguments");
+  std::vector<double> A((size_t)b * b, 0.0), X((size_t)b * b, 0.0);
+  int k = 0;
+  for (int i = 0; i < b; ++i) {
+    A[i * b + i] = 1.0;
+    X[i * b + i] = 1.0;
+  }
+  for (int i = 0; i < b; ++i)
+    for (int j = i + 1; j < b; ++j, ++k) {
+      A[i * b + j] += params[k];    // I + S
+      A[j * b + i] -= params[k];
+      X[i * b + j] -= params[k];    // I - S
+      X[j * b + i] += params[k];
+    }
+  for (int c = 0; c < b; ++c) {
+    int piv = c;
+    for (int r = c + 1; r < b; ++r)
+      if (std::fabs(A[r * b + c]) > std::fabs(A[piv * b + c])) piv = r;
+    if (A[piv * b + c] == 0.0) return set_error(ROT_EINVAL, "rot_harp_cayley_block: singular I + S");
+    if (piv != c)
+      for (int j = 0; j < b; ++j) {
+        std::swap(A[c * b + j], A[piv * b + j]);
+        std::swap(X[c * b + j], X[piv * b + j]);
+      }
+    for (int r = 0; r < b; ++r) {
+      if (r == c) continue;
+      const double f = A[r * b + c] / A[c * b + c];
+      if (f == 0.0) continue;
+      for (int j = 0; j < b; ++j) {
+        A[r * b + j] -= f * A[c * b + j];
+        X[r * b + j] -= f * X[c * b + j];
+      }
+    }
+  }
+  for (int r = 0; r < b; ++r)
+    for (int j = 0; j < b; ++j) X[r * b + j] /= A[r * b + r];
+  // B = Q G, G = mixer (row-major b x b) or the base mixer
+  std::vector<double> G((size_t)b * b, 0.0);
+  if (mixer) {
+    for (int i = 0; i < b * b; ++i) G[i] = mixer[i];
+  } else if (is_pow2(b)) {
+    const double h = 1.0 / std::sqrt((double)b);
+    for (int r = 0; r < b; ++r)
+      for (int c = 0; c < b; ++c) G[r * b + c] = sylv(r, c) * h;
+  } else {
+    for (int r = 0; r < b; ++r) G[r * b + r] = 1.0;
+  }
+  for (int r = 0; r < b; ++r)
+    for (int c = 0; c < b; ++c) {
+      double acc = 0.0;
+      for (int j = 0; j < b; ++j) acc += X[r * b + j] * G[j * b + c];
+      out[r * b + c] = (float)acc;
+    }
+  return ROT_OK;
+}
+
+namespace rotb {
+namespace {
+
+// Givens blocks of a stage from its int8 codes, on the device: theta = code * scale,
+// B = R(theta) H_2 / sqrt(2) [HARP gist.science summary, 2.2 (Givens for b = 2) and 2.4 (int8
+// parameter storage)]. One thread per block.
+__global__ void givens_expand_kernel(const int8_t* __restrict__ codes, float scale, int64_t n,
+                                     float* __restrict__ out) {
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+    const float th = (float)codes[i] * scale;
+    float sn, cs;
+    sincosf(th, &sn, &cs);
+    const float h = 0.70710678118654752f;
+    float4 v;
+    v.x = (cs - sn) * h;
+    v.y = (cs + sn) * h;
+    v.z = (sn + cs) * h;
+    v.w = (sn - cs) * h;
+    reinterpret_cast<float4*>(out)[i] = v;
+  }
+}
+
+}  // namespace
+}  // namespace rotb
+
+extern "C" rot_status rot_plan_create_q8(rot_plan_t* out, int K, int n_stages, const int* radices,
+                                         const int8_t* const* codes, const float* scales,
+                                         const int64_t* n_blocks, const float* const* mixers,
+                                         const int32_t* const* perms, const int8_t* signs) {
+  if (!out) return set_error(ROT_EINVAL, "rot_plan_create_q8: out is NULL");
+  *out = nullptr;
+  if (K < 1 || n_stages < 1 || n_stages > 64 || !radices)
+    return set_error(ROT_EINVAL, "rot_plan_create_q8: need K >= 1, 1 <= n_stages <= 64, radices");
+  for (int t = 0; t < n_stages; ++t)
+    if (radices[t] < 2 || K % radices[t] != 0) return set_error(ROT_EINVAL, "rot_plan_create_q8: bad radix");
+  std::vector<std::vector<float>> host(n_stages);
+  std::vector<const float*> params(n_stages, nullptr);
+  std::vector<int64_t> nb(n_stages, 0);
+  std::vector<int> expand(n_stages, 0);   // Givens stages built on the device after plan creation
+  for (int t = 0; t < n_stages; ++t) {
+    const int b = radices[t];
+    const int8_t* q = codes ? codes[t] : nullptr;
+    const float* mix = mixers ? mixers[t] : nullptr;
+    if (b == 2 && mix) return set_error(ROT_EINVAL, "rot_plan_create_q8: a radix-2 stage takes no mixer");
+    if (!q) {   // theta = 0: the block is the mixer
+      if (mix) {
+        host[t].assign(mix, mix + (size_t)b * b);
+        params[t] = host[t].data();
+        nb[t] = 1;
+      }
+      continue;
+    }
+    if (!scales || !n_blocks || (n_blocks[t] != 1 && n_blocks[t] != K / b))
+      return set_error(ROT_EINVAL, "rot_plan_create_q8: a stage with codes needs a scale and n_blocks 1 or K/b");
+    const int64_t n = n_blocks[t];
+    const int npb = b == 2 ? 1 : b * (b - 1) / 2;   // codes per block
+    bool any = false;
+    for (int64_t i = 0; i < n * npb && !any; ++i) any = q[i] != 0;
+    if (!any && !mix) continue;                      // all zero: the base mixer
+    nb[t] = n;
+    host[t].assign((size_t)n * b * b, 0.0f);
+    params[t] = host[t].data();
+    if (b == 2) {   // placeholder blocks, replaced on the device by the expansion kernel
+      expand[t] = 1;
+      continue;
+    }
+    std::vector<double> th(npb);
+    for (int64_t c = 0; c < n; ++c) {
+      for (int k = 0; k < npb; ++k) th[k] = (double)q[c * npb + k] * (double)scales[t];
+      rot_status st = rot_harp_cayley_block(th.data(), b, mix, host[t].data() + (size_t)c * b * b);
+      if (st) return st;
+    }
+  }
+  rot_status st = rot_plan_create(out, K, n_stages, radices, params.data(), nb.data(), perms, signs);
+  if (st) return st;
+  for (int t = 0; t < n_stages; ++t) {
+    if (!expand[t]) continue;
+    Stage& S = (*out)->stages[t];
+    const int64_t n = nb[t];
+    int8_t* dq = nullptr;
+    cudaError_t e = cudaMalloc(&dq, (size_t)n);
+    if (e == cudaSuccess) e = cudaMemcpy(dq, codes[t], (size_t)n, cudaMemcpyHostToDevice);
+    if (e == cudaSuccess) {
+      const int64_t grid = std::min<int64_t>((n + 255) / 256, 4096);
+      givens_expand_kernel<<<(unsigned)grid, 256>>>(dq, scales[t], n, S.d_blocks);
+      e = cudaGetLastError();
+      if (e == cudaSuccess) e = cudaDeviceSynchronize();
+    }
+    if (dq) cudaFree(dq);
+    if (e != cudaSuccess) {
+      rot_plan_destroy(*out);
+      *out = nullptr;
+      return cuda_error(e, "rot_plan_create_q8: expanding Givens blocks");
+    }
   }
   return ROT_OK;
 }

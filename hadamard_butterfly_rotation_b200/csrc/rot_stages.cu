@@ -131,8 +131,8 @@ __global__ void __launch_bounds__(THREADS) stages_kernel(const Args a) {
       for (int i = threadIdx.x; i < K; i += THREADS) dst[i] = cur[i];
     } else {
       // one warp per group: absmax by warp reduction, then one lane per 32-bit code word
-      const float qmax = a.bits == 4 ? 7.0f : 1.0f;
-      const float magic = a.bits == 4 ? 8388616.0f : 8388610.0f;
+      const float qmax = qmax_of_bits(a.bits);
+      const float magic = magic_of_bits(a.bits);
       const int cpw = 32 / a.bits;
       const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
       const int ngr = K / a.G;
@@ -143,7 +143,7 @@ __global__ void __launch_bounds__(THREADS) stages_kernel(const Args a) {
         for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
         float f;
         bool slow;
-        const uint16_t s16 = group_scale(m, a.bits == 4 ? 1.0f / 7.0f : 1.0f, 1.0f + 0x1p-22f, &f, &slow);
+        const uint16_t s16 = group_scale(m, 1.0f / qmax, 1.0f + 0x1p-22f, &f, &slow);
         if (lane == 0) a.scales[row * ngr + g] = s16;
         uint32_t* cw = reinterpret_cast<uint32_t*>(a.codes + row * (int64_t)(K / cpw) * 4) +
                        (int64_t)g * a.G / cpw;
@@ -154,7 +154,7 @@ __global__ void __launch_bounds__(THREADS) stages_kernel(const Args a) {
                                     : code_magic(gx[w * cpw + j], f, magic);
             word |= (u & ((1u << a.bits) - 1u)) << (a.bits * j);
           }
-          cw[w] = word ^ (a.bits == 4 ? 0x88888888u : 0xAAAAAAAAu);
+          cw[w] = word ^ offset_xor_of_bits(a.bits);
         }
       }
     }
@@ -344,11 +344,11 @@ __global__ void __launch_bounds__(MR_THREADS, 1) stages_rows_kernel(const MrArgs
       } else {
         // one warp per group; lane l takes 4 consecutive values per 128-value slice (one
         // 16-byte load), neighbouring lanes' code bits are merged with shuffles
-        const float qmax = a.bits == 4 ? 7.0f : 1.0f;
-        const float magic = a.bits == 4 ? 8388616.0f : 8388610.0f;
+        const float qmax = qmax_of_bits(a.bits);
+        const float magic = magic_of_bits(a.bits);
         const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
         const int ngr = K / a.G;
-        const int lpw = a.bits == 4 ? 2 : 4;   // lanes per 32-bit code word
+        const int lpw = a.bits / 2;            // lanes per 32-bit code word (4 codes per lane)
         for (int g = warp; g < ngr; g += MR_THREADS / 32) {
           const float* gx = xr + (int64_t)g * a.G;
           float m = 0.0f;
@@ -359,7 +359,7 @@ __global__ void __launch_bounds__(MR_THREADS, 1) stages_rows_kernel(const MrArgs
           for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
           float f;
           bool slow;
-          const uint16_t s16 = group_scale(m, a.bits == 4 ? 1.0f / 7.0f : 1.0f, 1.0f + 0x1p-22f, &f, &slow);
+          const uint16_t s16 = group_scale(m, 1.0f / qmax, 1.0f + 0x1p-22f, &f, &slow);
           if (lane == 0) a.scales[row * ngr + g] = s16;
           uint32_t* cw = reinterpret_cast<uint32_t*>(a.codes + row * (int64_t)(K * a.bits / 8)) +
                          (int64_t)g * a.G * a.bits / 32;
@@ -379,7 +379,7 @@ __global__ void __launch_bounds__(MR_THREADS, 1) stages_rows_kernel(const MrArgs
             uint32_t word = part << (4 * a.bits * (lane % lpw));
             for (int o = 1; o < lpw; o <<= 1) word |= __shfl_down_sync(0xffffffffu, word, o);
             if (lane % lpw == 0 && i < a.G)
-              cw[(i0 + 4 * lane) * a.bits / 32] = word ^ (a.bits == 4 ? 0x88888888u : 0xAAAAAAAAu);
+              cw[(i0 + 4 * lane) * a.bits / 32] = word ^ offset_xor_of_bits(a.bits);
           }
         }
       }

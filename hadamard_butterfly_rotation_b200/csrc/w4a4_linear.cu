@@ -65,8 +65,6 @@ constexpr int LOADER_WARP = N_EPI / 32;  // warp 8
 constexpr int N_UNP = 192;               // unpacker threads (warps 9-14)
 constexpr int N_UNP_WARPS = N_UNP / 32;
 constexpr int THREADS = N_EPI + 32 + N_UNP + 32;
-constexpr int N_CHUNKS = (BM + BN) * (KB / 32);                  // 16-byte packed chunks / stage
-constexpr int UNP_ITERS = (N_CHUNKS + N_UNP - 1) / N_UNP;        // per unpacker thread (last one partial)
 constexpr int EPI_COLS = BN / 2;         // columns per epilogue warp
 constexpr int MMA_WARP = (N_EPI + 32 + N_UNP) / 32;
 constexpr int LAUNCH_REGS = 128;         // 65536 / THREADS
@@ -81,16 +79,38 @@ constexpr uint32_t BIAS_BITS = 0x4B400000u;  // 1.5 * 2^23
 constexpr float BIAS_F = 12582912.0f;
 constexpr unsigned long long WAIT_NS = 2000000000ull;
 
-// smem layout (offsets from a 1024-byte aligned base)
-constexpr int OFF_STAGES = 0;
-constexpr int OFF_PSTAGES = STAGES * STAGE_BYTES;
-constexpr int OFF_SLOTS = OFF_PSTAGES + PSTAGES * PSTAGE_BYTES;  // per epilogue warp: sW/256 of its columns
-constexpr int OFF_BARS = OFF_SLOTS + N_EPI_WARPS * EPI_COLS * 4;
+// Shared-memory layout (offsets from a 1024-byte aligned base) of the two variants:
+//   A8 = false (W4A4): a packed stage holds the packed A and W tiles of one K-block (16 KB), and
+//                      the int8 ring stage holds the unpacked A and W tiles (32 KB);
+//   A8 = true  (W4A8): a packed stage holds the int8 A tile, landed by TMA in the MMA's 128-byte
+//                      swizzled K-major layout (16 KB), and the packed W tile (8 KB); the int8 ring
+//                      stage holds only the unpacked W tile (16 KB).
+// The int8 operands hold UNIT_A * qA and UNIT_W * qW (unpacking leaves 16 * q), so the int32
+// accumulators hold UNIT * P, UNIT = 256 (W4A4) or 16 (W4A8).
 constexpr int N_BARS = 2 * STAGES + 2 * PSTAGES + 2 * NACC;
-constexpr int OFF_TMEM = OFF_BARS + N_BARS * 8;
-constexpr int SMEM_BYTES = OFF_TMEM + 16 + 1024;          // + alignment slack
-static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
-static_assert(OFF_PSTAGES % 1024 == 0 && PSTAGE_BYTES % 1024 == 0, "TMA destinations stay 128-byte aligned");
+template <bool A8>
+struct Lay {
+  static constexpr int A_PBYTES = A8 ? BM * KB : BM * PROW_BYTES;   // A part of a packed stage
+  static constexpr int W_PBYTES = BN * PROW_BYTES;
+  static constexpr int PSTAGE = A_PBYTES + W_PBYTES;
+  static constexpr int STAGE = A8 ? B_STAGE_BYTES : STAGE_BYTES;    // int8 ring stage
+  static constexpr int B_OFF = A8 ? 0 : A_STAGE_BYTES;              // W tile within an int8 stage
+  static constexpr int ROWS_UNP = A8 ? BN : BM + BN;                // rows the unpackers expand
+  static constexpr int N_CHUNKS = ROWS_UNP * (KB / 32);             // 16-byte packed chunks / stage
+  static constexpr int UNP_ITERS = (N_CHUNKS + N_UNP - 1) / N_UNP;  // per unpacker thread (last partial)
+  static constexpr int SRC_OFF = A8 ? A_PBYTES : 0;                 // first unpacked row in a packed stage
+  static constexpr int OFF_STAGES = 0;
+  static constexpr int OFF_PSTAGES = STAGES * STAGE;
+  static constexpr int OFF_SLOTS = OFF_PSTAGES + PSTAGES * PSTAGE;  // per epilogue warp: sW/UNIT of its columns
+  static constexpr int OFF_BARS = OFF_SLOTS + N_EPI_WARPS * EPI_COLS * 4;
+  static constexpr int OFF_TMEM = OFF_BARS + N_BARS * 8;
+  static constexpr int SMEM = OFF_TMEM + 16 + 1024;                 // + alignment slack
+  static constexpr float UNIT = A8 ? 16.0f : 256.0f;
+  static constexpr int PEMPTY_ARRIVALS = N_UNP_WARPS + (A8 ? 1 : 0);  // + the MMA's commit (A8)
+  static_assert(SMEM <= 227 * 1024, "shared memory");
+  static_assert(OFF_PSTAGES % 1024 == 0 && PSTAGE % 1024 == 0 && A_PBYTES % 1024 == 0,
+                "TMA destinations and the swizzled A tile stay 1024-byte aligned");
+};
 
 __device__ int g_w4a4_error = 0;
 
@@ -281,20 +301,21 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* tmap, 
       : "memory");
 }
 
-template <bool PARTIALS>
+template <bool PARTIALS, bool A8>
 __global__ void __launch_bounds__(THREADS, 1) w4a4_kernel(const __grid_constant__ Params p) {
+  using L = Lay<A8>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BARS);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::OFF_BARS);
   uint64_t* full = bars;                 // [STAGES]  unpackers -> MMA (one arrival per unpacker warp)
   uint64_t* empty = full + STAGES;       // [STAGES]  MMA commit -> unpackers
   uint64_t* pfull = empty + STAGES;      // [PSTAGES] TMA bytes -> unpackers
-  uint64_t* pempty = pfull + PSTAGES;    // [PSTAGES] unpackers -> loader
+  uint64_t* pempty = pfull + PSTAGES;    // [PSTAGES] unpackers (and, A8, the MMA commit) -> loader
   uint64_t* tfull = pempty + PSTAGES;    // [NACC]    MMA commit -> epilogue
   uint64_t* tempty = tfull + NACC;       // [NACC]    epilogue warps -> MMA
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_TMEM);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + OFF_TMEM + 8);
-  float* slots = reinterpret_cast<float*>(smem + OFF_SLOTS);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_TMEM);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::OFF_TMEM + 8);
+  float* slots = reinterpret_cast<float*>(smem + L::OFF_SLOTS);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -307,7 +328,7 @@ __global__ void __launch_bounds__(THREADS, 1) w4a4_kernel(const __grid_constant_
     }
     for (int s = 0; s < PSTAGES; ++s) {
       mbar_init(&pfull[s], 1);
-      mbar_init(&pempty[s], N_UNP_WARPS);
+      mbar_init(&pempty[s], L::PEMPTY_ARRIVALS);
     }
     for (int b = 0; b < NACC; ++b) {
       mbar_init(&tfull[b], 1);
@@ -326,6 +347,11 @@ __global__ void __launch_bounds__(THREADS, 1) w4a4_kernel(const __grid_constant_
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // Under programmatic dependent launch the set-up above may overlap the previous kernel in the
+  // stream (e.g. the rotation that writes Aq and As); every global access comes after this wait
+  // (a no-op for an ordinary launch). Dependents may start their own set-up at once.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   if (warp < N_EPI_WARPS) {
     // ======================= epilogue
@@ -410,8 +436,8 @@ __global__ void __launch_bounds__(THREADS, 1) w4a4_kernel(const __grid_constant_
             q0w0 = __ldg(nw0); q0w1 = __ldg(nw1); q0a = __ldg(na);
           }
           __syncwarp();                 // every lane has read the previous group's column scales
-          wsc[lane] = __half2float(__ushort_as_half(rw0)) * (1.0f / 256.0f);
-          wsc[lane + 32] = __half2float(__ushort_as_half(rw1)) * (1.0f / 256.0f);
+          wsc[lane] = __half2float(__ushort_as_half(rw0)) * (1.0f / L::UNIT);
+          wsc[lane + 32] = __half2float(__ushort_as_half(rw1)) * (1.0f / L::UNIT);
           sa = __half2float(__ushort_as_half(ra));
           __syncwarp();
         }
@@ -452,7 +478,7 @@ __global__ void __launch_bounds__(THREADS, 1) w4a4_kernel(const __grid_constant_
             for (int j = 0; j < 64; ++j) {
               const int n = w.n0 + wg * EPI_COLS + j;
               const uint32_t v = j < 32 ? r0[j] : r1[j - 32];
-              if (n < p.N) p.P[((int64_t)m * p.N + n) * NG + g] = ((int32_t)v) / 256;
+              if (n < p.N) p.P[((int64_t)m * p.N + n) * NG + g] = ((int32_t)v) / (int32_t)L::UNIT;
             }
           }
         }
@@ -516,12 +542,13 @@ __global__ void __launch_bounds__(THREADS, 1) w4a4_kernel(const __grid_constant_
           break;
         }
         if (lane == 0) {
-          uint8_t* pst = smem + OFF_PSTAGES + ps * PSTAGE_BYTES;
+          uint8_t* pst = smem + L::OFF_PSTAGES + ps * L::PSTAGE;
           const int kb = w.kb0 + j;
-          mbar_arrive_expect_tx(&pfull[ps], (uint32_t)PSTAGE_BYTES);
-          // x = kb * 64 bytes: a multiple of 16, as a tiled TMA requires of the inner coordinate
-          tma_load_2d(pst, &p.tmA, kb * PROW_BYTES, w.m0, &pfull[ps]);
-          tma_load_2d(pst + BM * PROW_BYTES, &p.tmW, kb * PROW_BYTES, w.n0, &pfull[ps]);
+          mbar_arrive_expect_tx(&pfull[ps], (uint32_t)L::PSTAGE);
+          // x = kb * 128 (int8 A) or kb * 64 bytes: a multiple of 16, as a tiled TMA requires of the
+          // inner coordinate; the int8 A box lands 128-byte swizzled (the MMA's operand layout)
+          tma_load_2d(pst, &p.tmA, kb * (A8 ? KB : PROW_BYTES), w.m0, &pfull[ps]);
+          tma_load_2d(pst + L::A_PBYTES, &p.tmW, kb * PROW_BYTES, w.n0, &pfull[ps]);
         }
         __syncwarp();
       }
@@ -536,7 +563,8 @@ __global__ void __launch_bounds__(THREADS, 1) w4a4_kernel(const __grid_constant_
     // 128-byte rows (row r at byte 128*r of the stage).
     const int c = ut & 3, r0 = ut >> 2, r7 = r0 & 7;
     const int lo_off = ((2 * c) ^ r7) << 4, hi_off = ((2 * c + 1) ^ r7) << 4;
-    const bool tail = ut + N_UNP * (UNP_ITERS - 1) < N_CHUNKS;   // this thread has a last chunk
+    constexpr int UNP_ITERS = L::UNP_ITERS;
+    const bool tail = ut + N_UNP * (UNP_ITERS - 1) < L::N_CHUNKS;   // this thread has a last chunk
     int it = 0;
     bool ok = true;
     for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x) {
@@ -548,8 +576,8 @@ __global__ void __launch_bounds__(THREADS, 1) w4a4_kernel(const __grid_constant_
           ok = false;
           break;
         }
-        const uint8_t* src = smem + OFF_PSTAGES + ps * PSTAGE_BYTES + ut * 16;
-        uint8_t* dst = smem + OFF_STAGES + s * STAGE_BYTES + r0 * 128;
+        const uint8_t* src = smem + L::OFF_PSTAGES + ps * L::PSTAGE + L::SRC_OFF + ut * 16;
+        uint8_t* dst = smem + L::OFF_STAGES + s * L::STAGE + r0 * 128;
         // all loads first, then the stores: the shared-memory latency is paid once per stage
         uint4 v[UNP_ITERS];
 #pragma unroll
@@ -563,8 +591,19 @@ __global__ void __launch_bounds__(THREADS, 1) w4a4_kernel(const __grid_constant_
             const uint4 hi = make_uint4(v[i].x & 0xF0F0F0F0u, v[i].y & 0xF0F0F0F0u, v[i].z & 0xF0F0F0F0u,
                                         v[i].w & 0xF0F0F0F0u);
             uint8_t* rowp = dst + i * (N_UNP / 4) * 128;
-            *reinterpret_cast<uint4*>(rowp + lo_off) = lo;
-            *reinterpret_cast<uint4*>(rowp + hi_off) = hi;
+            if constexpr (A8) {
+              // natural K order (the int8 A tile is not permuted): interleave even / odd codes
+              *reinterpret_cast<uint4*>(rowp + lo_off) =
+                  make_uint4(prmt(lo.x, hi.x, 0x5140u), prmt(lo.x, hi.x, 0x7362u), prmt(lo.y, hi.y, 0x5140u),
+                             prmt(lo.y, hi.y, 0x7362u));
+              *reinterpret_cast<uint4*>(rowp + hi_off) =
+                  make_uint4(prmt(lo.z, hi.z, 0x5140u), prmt(lo.z, hi.z, 0x7362u), prmt(lo.w, hi.w, 0x5140u),
+                             prmt(lo.w, hi.w, 0x7362u));
+            } else {
+              // even codes of the 32-code chunk, then odd codes (the same K order for A and W)
+              *reinterpret_cast<uint4*>(rowp + lo_off) = lo;
+              *reinterpret_cast<uint4*>(rowp + hi_off) = hi;
+            }
           }
         }
         fence_proxy_async();
@@ -578,10 +617,13 @@ __global__ void __launch_bounds__(THREADS, 1) w4a4_kernel(const __grid_constant_
   } else {
     // ======================= MMA issue (the whole warp runs the loop; elect.sync issues)
     asm volatile("setmaxnreg.dec.sync.aligned.u32 80;");  // same value as the rest of its warpgroup
-    // descriptors of stage 0; stage s and k-step k4 add (s * STAGE_BYTES + 32 * k4) >> 4 to the
-    // start-address field (no carry: shared addresses stay below 2^18)
-    const uint32_t sbase = smem_u32(smem + OFF_STAGES);
-    const uint64_t dA0 = make_desc(sbase), dB0 = make_desc(sbase + A_STAGE_BYTES);
+    // descriptors of stage 0; stage s and k-step k4 add (s * stage bytes + 32 * k4) >> 4 to the
+    // start-address field (no carry: shared addresses stay below 2^18). W4A4: A and W in the
+    // int8 stage s; W4A8: A in the packed stage ps (landed by TMA), W in the int8 stage s.
+    const uint32_t sbase = smem_u32(smem + L::OFF_STAGES);
+    const uint64_t dA0 = A8 ? make_desc(smem_u32(smem + L::OFF_PSTAGES)) : make_desc(sbase);
+    const uint64_t dB0 = make_desc(sbase + L::B_OFF);
+    int ps = 0, pph = 0;                    // packed stage of the K-block (A8: A's stage), its parity
     const int gsteps = p.G / 32;            // k-steps per group
     int s = 0, sph = 0;                     // int8 stage and its phase parity
     int b = 0, tph = 0;                     // accumulator and its phase parity
@@ -591,13 +633,15 @@ __global__ void __launch_bounds__(THREADS, 1) w4a4_kernel(const __grid_constant_
     for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x) {
       const Unit w = unit_of(p, u);         // K range group-aligned: kg == 0 here
       for (int j = 0; j < w.nkb; ++j) {
-        if (!bar_wait(&full[s], sph, abort_flag, p.wait_ns)) {
+        if (!bar_wait(&full[s], sph, abort_flag, p.wait_ns) ||
+            (A8 && !bar_wait(&pfull[ps], pph, abort_flag, p.wait_ns))) {   // A8: the A tile has landed
           ok = false;
           break;
         }
         tc_fence_after();
         const int nk = min(4, w.ks - 4 * j);
-        const uint64_t so = (uint64_t)((s * STAGE_BYTES) >> 4);
+        const uint64_t soA = (uint64_t)(((A8 ? ps * L::PSTAGE : s * L::STAGE)) >> 4);
+        const uint64_t soB = (uint64_t)((s * L::STAGE) >> 4);
 #pragma unroll
         for (int k4 = 0; k4 < 4; ++k4) {
           if (k4 < nk) {
@@ -608,7 +652,7 @@ __global__ void __launch_bounds__(THREADS, 1) w4a4_kernel(const __grid_constant_
               }
               tc_fence_after();
             }
-            umma_i8(tmem + b * BN, dA0 + so + 2 * k4, dB0 + so + 2 * k4, kg != 0 ? 1u : 0u);
+            umma_i8(tmem + b * BN, dA0 + soA + 2 * k4, dB0 + soB + 2 * k4, kg != 0 ? 1u : 0u);
             if (++kg == gsteps) {
               umma_commit(&tfull[b]);
               kg = 0;
@@ -621,10 +665,15 @@ __global__ void __launch_bounds__(THREADS, 1) w4a4_kernel(const __grid_constant_
         }
         if (!ok) break;
         umma_commit(&empty[s]);
+        if (A8) umma_commit(&pempty[ps]);   // the A tile of this packed stage is consumed
         ++nblk;
         if (++s == STAGES) {
           s = 0;
           sph ^= 1;
+        }
+        if (++ps == PSTAGES) {
+          ps = 0;
+          pph ^= 1;
         }
       }
     }
@@ -632,6 +681,10 @@ __global__ void __launch_bounds__(THREADS, 1) w4a4_kernel(const __grid_constant_
     if (ok && nblk > 0) {
       const int last = s == 0 ? STAGES - 1 : s - 1;
       bar_wait(&empty[last], s == 0 ? sph ^ 1 : sph, abort_flag, p.wait_ns);
+      if (A8) {
+        const int plast = ps == 0 ? PSTAGES - 1 : ps - 1;
+        bar_wait(&pempty[plast], ps == 0 ? pph ^ 1 : pph, abort_flag, p.wait_ns);
+      }
     }
   }
 
@@ -681,8 +734,14 @@ struct DecParams {
   int groups_per_split;
 };
 
-template <int MT>
+// A8 (W4A8): the activation codes are int8 [M, K] in natural order; per span each lane loads the
+// 32 int8 codes of its rows that meet its 16-byte weight piece and splits them into even / odd
+// codes (byte permutes), the same order as the unpacked weights; products are 16 * qA * qW.
+template <int MT, bool A8>
 __global__ void __launch_bounds__(DEC_THREADS) w4a4_decode_kernel(const DecParams p) {
+  constexpr float UNIT = A8 ? 16.0f : 256.0f;
+  asm volatile("griddepcontrol.wait;" ::: "memory");   // see w4a4_kernel (programmatic launch)
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int warp = threadIdx.x >> 5, l = threadIdx.x & 31;
   const int g = l >> 2, c = l & 3;
   const int nt = blockIdx.x * (DEC_THREADS / 32) + warp;   // n-tile of 8 weight rows
@@ -718,28 +777,53 @@ __global__ void __launch_bounds__(DEC_THREADS) w4a4_decode_kernel(const DecParam
 #pragma unroll
       for (int t = 0; t < MT; ++t) {
         const int m_lo = t * 16 + g, m_hi = m_lo + 8;
-        uint4 alo = make_uint4(0u, 0u, 0u, 0u), ahi = make_uint4(0u, 0u, 0u, 0u);
-        if (m_lo < p.M) alo = __ldg(reinterpret_cast<const uint4*>(p.Aq + (int64_t)m_lo * ldp + (int64_t)span * 64 + 16 * c));
-        if (m_hi < p.M) ahi = __ldg(reinterpret_cast<const uint4*>(p.Aq + (int64_t)m_hi * ldp + (int64_t)span * 64 + 16 * c));
-        const uint32_t al[4] = {alo.x, alo.y, alo.z, alo.w}, ah[4] = {ahi.x, ahi.y, ahi.z, ahi.w};
+        if constexpr (A8) {
+          // int8 codes 128 * span + 32 c .. + 31 of rows m_lo / m_hi (two 16-byte loads each)
+          const int64_t lda8 = p.K;
+          uint4 l0 = make_uint4(0u, 0u, 0u, 0u), l1 = l0, h0 = l0, h1 = l0;
+          if (m_lo < p.M) {
+            const uint4* q = reinterpret_cast<const uint4*>(p.Aq + (int64_t)m_lo * lda8 + (int64_t)span * 128 + 32 * c);
+            l0 = __ldg(q);
+            l1 = __ldg(q + 1);
+          }
+          if (m_hi < p.M) {
+            const uint4* q = reinterpret_cast<const uint4*>(p.Aq + (int64_t)m_hi * lda8 + (int64_t)span * 128 + 32 * c);
+            h0 = __ldg(q);
+            h1 = __ldg(q + 1);
+          }
+          const uint32_t al[8] = {l0.x, l0.y, l0.z, l0.w, l1.x, l1.y, l1.z, l1.w};
+          const uint32_t ah[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
 #pragma unroll
-        for (int s4 = 0; s4 < 4; ++s4) {
-          // A rows g / g + 8: even codes (low nibbles, as 16*q) then odd codes (high nibbles)
-          const uint32_t a[4] = {(al[s4] << 4) & 0xF0F0F0F0u, (ah[s4] << 4) & 0xF0F0F0F0u, al[s4] & 0xF0F0F0F0u,
-                                 ah[s4] & 0xF0F0F0F0u};
-          mma_s8_16832(d[t], a, (ww[s4] << 4) & 0xF0F0F0F0u, ww[s4] & 0xF0F0F0F0u);
+          for (int s4 = 0; s4 < 4; ++s4) {
+            // codes 8 s4 .. 8 s4 + 7 of the lane's 32: even ones, then odd ones
+            const uint32_t a[4] = {prmt(al[2 * s4], al[2 * s4 + 1], 0x6420u), prmt(ah[2 * s4], ah[2 * s4 + 1], 0x6420u),
+                                   prmt(al[2 * s4], al[2 * s4 + 1], 0x7531u), prmt(ah[2 * s4], ah[2 * s4 + 1], 0x7531u)};
+            mma_s8_16832(d[t], a, (ww[s4] << 4) & 0xF0F0F0F0u, ww[s4] & 0xF0F0F0F0u);
+          }
+        } else {
+          uint4 alo = make_uint4(0u, 0u, 0u, 0u), ahi = make_uint4(0u, 0u, 0u, 0u);
+          if (m_lo < p.M) alo = __ldg(reinterpret_cast<const uint4*>(p.Aq + (int64_t)m_lo * ldp + (int64_t)span * 64 + 16 * c));
+          if (m_hi < p.M) ahi = __ldg(reinterpret_cast<const uint4*>(p.Aq + (int64_t)m_hi * ldp + (int64_t)span * 64 + 16 * c));
+          const uint32_t al[4] = {alo.x, alo.y, alo.z, alo.w}, ah[4] = {ahi.x, ahi.y, ahi.z, ahi.w};
+#pragma unroll
+          for (int s4 = 0; s4 < 4; ++s4) {
+            // A rows g / g + 8: even codes (low nibbles, as 16*q) then odd codes (high nibbles)
+            const uint32_t a[4] = {(al[s4] << 4) & 0xF0F0F0F0u, (ah[s4] << 4) & 0xF0F0F0F0u, al[s4] & 0xF0F0F0F0u,
+                                   ah[s4] & 0xF0F0F0F0u};
+            mma_s8_16832(d[t], a, (ww[s4] << 4) & 0xF0F0F0F0u, ww[s4] & 0xF0F0F0F0u);
+          }
         }
       }
     }
     // group scales: D[row][col] with rows m (tokens) and cols n0 + 2c (+1)
-    const float sw0 = __half2float(__ushort_as_half(p.Ws[(int64_t)(n0 + 2 * c) * NG + gg])) * (1.0f / 256.0f);
-    const float sw1 = __half2float(__ushort_as_half(p.Ws[(int64_t)(n0 + 2 * c + 1) * NG + gg])) * (1.0f / 256.0f);
+    const float sw0 = __half2float(__ushort_as_half(p.Ws[(int64_t)(n0 + 2 * c) * NG + gg])) * (1.0f / UNIT);
+    const float sw1 = __half2float(__ushort_as_half(p.Ws[(int64_t)(n0 + 2 * c + 1) * NG + gg])) * (1.0f / UNIT);
 #pragma unroll
     for (int t = 0; t < MT; ++t) {
       const int m_lo = t * 16 + g, m_hi = m_lo + 8;
       const float sa0 = m_lo < p.M ? __half2float(__ushort_as_half(p.As[(int64_t)m_lo * NG + gg])) : 0.0f;
       const float sa1 = m_hi < p.M ? __half2float(__ushort_as_half(p.As[(int64_t)m_hi * NG + gg])) : 0.0f;
-      // exact int32 partials (|256 P| < 2^22) convert exactly; P*sW then acc += (P*sW)*sA
+      // exact int32 partials (|UNIT P| < 2^22) convert exactly; P*sW then acc += (P*sW)*sA
       acc[t][0] = fmaf((float)d[t][0] * sw0, sa0, acc[t][0]);
       acc[t][1] = fmaf((float)d[t][1] * sw1, sa0, acc[t][1]);
       acc[t][2] = fmaf((float)d[t][2] * sw0, sa1, acc[t][2]);
@@ -811,9 +895,28 @@ rot_status w4a4_tile_plan_compute(int64_t M, int64_t N, int64_t K, int G, int sm
   return ROT_OK;
 }
 
+// Launch a kernel, with programmatic stream serialization when pdl is set (its prologue may then
+// overlap the previous kernel; the kernels wait with griddepcontrol.wait before any global access).
+template <typename P>
+cudaError_t launch_maybe_pdl(void (*kern)(const P), dim3 grid, dim3 block, size_t smem, cudaStream_t s, bool pdl,
+                             const P& prm) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, prm);
+  return e != cudaSuccess ? e : cudaGetLastError();
+}
+
 rot_status w4a4_launch(const uint8_t* Aq, const uint16_t* As, const uint8_t* Wq, const uint16_t* Ws, int64_t M,
                        int64_t N, int64_t K, int G, void* C, int c_dtype, int32_t* partials, cudaStream_t s,
-                       float* scratch, int64_t scratch_floats) {
+                       float* scratch, int64_t scratch_floats, bool a8, bool pdl) {
   if (G > 256) return set_error(ROT_EUNSUPPORTED, "w4a4_linear: G > 256 is not supported");
   if (M > (1ll << 30) || N > (1ll << 30) || K > (1ll << 30)) return set_error(ROT_EUNSUPPORTED, "w4a4_linear: size too large");
   // fp32 accumulation target for K-split launches: C itself (fp32), the caller's scratch, or a
@@ -871,11 +974,12 @@ rot_status w4a4_launch(const uint8_t* Aq, const uint16_t* As, const uint8_t* Wq,
     }
     const dim3 grid((unsigned)((ntiles + DEC_THREADS / 32 - 1) / (DEC_THREADS / 32)), (unsigned)splits);
     const int mt = (int)((M + 15) / 16);
-    if (mt == 1) w4a4_decode_kernel<1><<<grid, DEC_THREADS, 0, s>>>(d);
-    else if (mt == 2) w4a4_decode_kernel<2><<<grid, DEC_THREADS, 0, s>>>(d);
-    else if (mt == 3) w4a4_decode_kernel<3><<<grid, DEC_THREADS, 0, s>>>(d);
-    else w4a4_decode_kernel<4><<<grid, DEC_THREADS, 0, s>>>(d);
-    ROT_CUDA_TRY(cudaGetLastError());
+    void (*dk)(const DecParams) = nullptr;
+    if (a8) dk = mt == 1 ? w4a4_decode_kernel<1, true> : mt == 2 ? w4a4_decode_kernel<2, true>
+                 : mt == 3 ? w4a4_decode_kernel<3, true> : w4a4_decode_kernel<4, true>;
+    else dk = mt == 1 ? w4a4_decode_kernel<1, false> : mt == 2 ? w4a4_decode_kernel<2, false>
+              : mt == 3 ? w4a4_decode_kernel<3, false> : w4a4_decode_kernel<4, false>;
+    ROT_CUDA_TRY(launch_maybe_pdl(dk, grid, dim3(DEC_THREADS), 0, s, pdl && splits == 1, d));
     return splits > 1 ? finish_acc(d.Cacc) : ROT_OK;
   }
   static int configured[64] = {0};
@@ -884,13 +988,15 @@ rot_status w4a4_launch(const uint8_t* Aq, const uint16_t* As, const uint8_t* Wq,
   if (dev < 64 && !configured[dev]) {
     // The setmaxnreg split is only valid for the register count it was sized for: refuse
     // to launch otherwise (an over-subscribed split would wait for registers forever).
-    for (int v = 0; v < 2; ++v) {
-      const void* k = v ? (const void*)w4a4_kernel<true> : (const void*)w4a4_kernel<false>;
+    const void* ks[4] = {(const void*)w4a4_kernel<false, false>, (const void*)w4a4_kernel<true, false>,
+                         (const void*)w4a4_kernel<false, true>, (const void*)w4a4_kernel<true, true>};
+    for (int v = 0; v < 4; ++v) {
       cudaFuncAttributes fa;
-      ROT_CUDA_TRY(cudaFuncGetAttributes(&fa, k));
+      ROT_CUDA_TRY(cudaFuncGetAttributes(&fa, ks[v]));
       if (fa.numRegs != LAUNCH_REGS)
         return set_error(ROT_EUNSUPPORTED, "w4a4_linear: kernel built with an unexpected register count");
-      ROT_CUDA_TRY(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES));
+      ROT_CUDA_TRY(cudaFuncSetAttribute(ks[v], cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        v < 2 ? Lay<false>::SMEM : Lay<true>::SMEM));
     }
     configured[dev] = 1;
   }
@@ -908,12 +1014,15 @@ rot_status w4a4_launch(const uint8_t* Aq, const uint16_t* As, const uint8_t* Wq,
     const cuuint64_t ldp = (cuuint64_t)(K / 2);
     const cuuint32_t estr[2] = {1, 1};
     {
-      const cuuint64_t dims[2] = {ldp, (cuuint64_t)(M > 0 ? M : 1)};
-      const cuuint64_t strides[1] = {ldp};
-      const cuuint32_t box[2] = {(cuuint32_t)PROW_BYTES, (cuuint32_t)BM};
+      // W4A4: packed A [M, K/2], box {64 bytes, BM rows}; W4A8: int8 A [M, K], box {128 bytes,
+      // BM rows}, 128-byte swizzled into the MMA's K-major operand layout
+      const cuuint64_t lda = a8 ? (cuuint64_t)K : ldp;
+      const cuuint64_t dims[2] = {lda, (cuuint64_t)(M > 0 ? M : 1)};
+      const cuuint64_t strides[1] = {lda};
+      const cuuint32_t box[2] = {(cuuint32_t)(a8 ? KB : PROW_BYTES), (cuuint32_t)BM};
       if (encode(&p.tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(Aq), dims, strides, box, estr,
-                 CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
-                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+                 CU_TENSOR_MAP_INTERLEAVE_NONE, a8 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                 CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
         return set_error(ROT_EINVAL, "w4a4_linear: tensor map for Aq rejected");
     }
     {
@@ -955,10 +1064,22 @@ rot_status w4a4_launch(const uint8_t* Aq, const uint16_t* As, const uint8_t* Wq,
   }
   // persistent: one CTA per SM (the shared-memory footprint admits no second one)
   const unsigned grid = (unsigned)tp.grid;
-  if (partials) w4a4_kernel<true><<<grid, THREADS, SMEM_BYTES, s>>>(p);
-  else w4a4_kernel<false><<<grid, THREADS, SMEM_BYTES, s>>>(p);
-  ROT_CUDA_TRY(cudaGetLastError());
+  void (*tk)(const Params) = a8 ? (partials ? w4a4_kernel<true, true> : w4a4_kernel<false, true>)
+                                : (partials ? w4a4_kernel<true, false> : w4a4_kernel<false, false>);
+  // (after a split-K memset the launch is an ordinary one: the dependency is not a kernel)
+  ROT_CUDA_TRY(launch_maybe_pdl(tk, dim3(grid), dim3(THREADS), a8 ? Lay<true>::SMEM : Lay<false>::SMEM, s,
+                                pdl && p.splits == 1, p));
   return p.splits > 1 ? finish_acc(p.Cacc) : ROT_OK;
+}
+
+rot_status f32_to_bf16_launch(const float* src, void* dst, int64_t n, cudaStream_t s) {
+  if (n % 4 != 0) return set_error(ROT_EINVAL, "f32_to_bf16: n must be a multiple of 4");
+  const int64_t n4 = n / 4;
+  if (n4 == 0) return ROT_OK;
+  const int64_t blocks = std::min<int64_t>((n4 + 255) / 256, (int64_t)sm_count() * 8);
+  f32_to_bf16_kernel<<<(unsigned)blocks, 256, 0, s>>>(src, static_cast<__nv_bfloat16*>(dst), n4);
+  ROT_CUDA_TRY(cudaGetLastError());
+  return ROT_OK;
 }
 
 rot_status w4a4_noalloc_scratch(float** out) {

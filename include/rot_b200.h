@@ -35,6 +35,7 @@
  *       activations  A      [M, lda]  bf16 or fp32
  *       codes        uint8  [M, K*bits/8]  int4: byte j = q[2j] | q[2j+1] << 4
  *                                          int2: byte j holds q[4j+i] in bits 2i..2i+1
+ *                                          int8: byte j = q[j]
  *                           (two's complement, symmetric levels -qmax..qmax,
  *                            qmax = 2^(bits-1) - 1)
  *       scales       uint16 [M, K/G]  IEEE binary16 bit patterns, one per (row, group)
@@ -107,7 +108,7 @@ rot_status rot_apply(const void* A, int a_dtype, int64_t M, int64_t lda, rot_pla
 
 /* Fused rotate + quantise + pack, one HBM pass [HARP abstract; Hadamard-Int4-Accuracy
  * wiki, Method]: codes [M, K*bits/8], scales [M, K/G] (binary16 bits).
- * bits in {2, 4}; G must divide K and be a multiple of 8 (int4) or 16 (int2).
+ * bits in {2, 4, 8}; G must divide K and be a multiple of 16 (int2), 8 (int4) or 4 (int8).
  * Errors: ROT_EINVAL for a bad G / bits / pointer / leading dimension. */
 rot_status rot_quant(const void* A, int a_dtype, int64_t M, int64_t lda, rot_plan_t plan,
                      int bits, int G, uint8_t* codes, uint16_t* scales, void* stream);
@@ -147,6 +148,56 @@ rot_status w4a4_linear_noalloc(const uint8_t* Aq, const uint16_t* As, const uint
                                const uint16_t* Ws, int64_t M, int64_t N, int64_t K, int G, void* C,
                                int c_dtype, void* stream);
 
+/* W4A4 linear with a two-sided processor [HARP abstract: a two-sided orthogonal processor;
+ * HARP gist.science summary, sections 1 and 3]. With an input-side plan T (size K) and an
+ * output-side plan U (size N), the weights are prepared offline as B~ = T B U^T (the rows of B,
+ * length N, through U; then the columns through T; quantised as the rows of B~^T), so that
+ * (A T^T) B~ = A B U^T: every output row comes out as c~ = U c. This call runs w4a4_linear on
+ * (Aq, As) and (Wq, Ws) = the quantised rows of B~^T and then returns each row to c = U^T c~
+ * with the rotation kernels (in place on fp32; for bf16 output on a stream-ordered fp32
+ * temporary of M * N floats, converted afterwards).
+ *   out_plan  the output-side plan U on the current device, out_plan K == N
+ * Other arguments, layouts and constraints as for w4a4_linear. */
+rot_status w4a4_linear_rot(const uint8_t* Aq, const uint16_t* As, const uint8_t* Wq, const uint16_t* Ws,
+                           int64_t M, int64_t N, int64_t K, int G, rot_plan_t out_plan, void* C,
+                           int c_dtype, void* stream);
+
+/* The online path in one call: rot_quant of the activations (int4, group G) into a caller
+ * workspace, then w4a4_linear against the prepared weights [Hadamard-Int4-Accuracy wiki,
+ * Hypothesis: A.B = (A.Q)(Q.B) with both operands quantised; HARP gist.science summary 2.4: stage
+ * kernels fused to keep the overhead low]. The linear is launched with programmatic dependent
+ * launch: its set-up (barriers, tensor-memory allocation) overlaps the rotation's tail and it
+ * reads the packed codes once the rotation has completed, while they are still in L2 at
+ * prefill sizes (M * K / 2 bytes: 4 MB for A[2048, 4096]).
+ *   A, a_dtype, M, lda, plan   as for rot_quant (plan K = the linear's K)
+ *   Wq, Ws, N, G, C, c_dtype   as for w4a4_linear
+ *   workspace                  caller-owned device memory, 16-byte aligned, of at least
+ *                              w4a4_linear_act_workspace(M, K, G) bytes: the packed codes
+ *                              [M, K/2] then (16-byte aligned) the scales [M, K/G]; they keep
+ *                              the rotated codes after the call.
+ * Errors: as rot_quant and w4a4_linear; ROT_EINVAL for a missing or short workspace. */
+rot_status w4a4_linear_act_workspace(int64_t M, int64_t K, int G, size_t* bytes);
+rot_status w4a4_linear_act(const void* A, int a_dtype, int64_t M, int64_t lda, rot_plan_t plan,
+                           const uint8_t* Wq, const uint16_t* Ws, int64_t N, int G, void* C, int c_dtype,
+                           void* workspace, size_t workspace_bytes, void* stream);
+
+/* W4A8 linear: int8 activations, int4 weights [Hadamard-Int4-Accuracy wiki, Method
+ * (matmul_q_err with abits = 8, bbits = 4) and Results ("W4A8 (act8/wt4)", a diagnostic that
+ * isolates which operand's int4 hurts); fact 3: int8 activations absorb the outliers]:
+ *   C[m, n] = sum_g float(As[m, g]) * float(Ws[n, g]) * P[m, n, g],
+ *   P[m, n, g] = sum_{k in group g} qA[m, k] * qW[n, k]   (exact int32)
+ * Aq: int8 [M, K] (rot_quant with bits = 8: one two's-complement code per byte, natural order),
+ * As: binary16 [M, K/G]; Wq, Ws, C and every constraint as for w4a4_linear. The same kernels run
+ * with the int8 activation tile loaded as is (tcgen05 kind::i8; mma.sync s8 for decode-sized M)
+ * and only the weights unpacked. */
+rot_status w4a8_linear(const int8_t* Aq, const uint16_t* As, const uint8_t* Wq, const uint16_t* Ws,
+                       int64_t M, int64_t N, int64_t K, int G, void* C, int c_dtype, void* stream);
+
+/* The exact int32 group partial sums P[m, n, g] of the W4A8 contraction (int8 Aq [M, K]),
+ * written to P: int32 [M, N, K/G]. For checking only. */
+rot_status w4a8_group_partials(const int8_t* Aq, const uint8_t* Wq, int64_t M, int64_t N, int64_t K,
+                               int G, int32_t* P, void* stream);
+
 /* Host only (no device work): the work list the tcgen05 tile kernel of w4a4_linear uses for a
  * shape (M > 64 or G % 128 != 0), given the device's SM count. out: int64 [6] =
  * {tiles_m, tiles_n, splits, kb_per_split, units, grid}: 128 x 128 output tiles; K split into
@@ -169,6 +220,34 @@ rot_status w4a4_group_partials(const uint8_t* Aq, const uint8_t* Wq, int64_t M, 
  *     (Householder QR in double), out holds b * b floats. */
 rot_status rot_harp_givens_blocks(const double* theta, int64_t n, float* out);
 rot_status rot_harp_qr_block(const double* g, int b, float* out);
+
+/* rot_harp_cayley_block: B = Q(theta) G for one b x b block (b >= 2), Q(theta) = (I + S)^{-1}
+ *   (I - S) the Cayley map of the skew-symmetric S whose strictly upper entries are params
+ *   (b(b-1)/2 doubles, row-major order: S[i][j] = params[k] for i < j, S[j][i] = -params[k]),
+ *   G = mixer (b x b row-major fp32) or, when mixer is NULL, the base mixer (H_b / sqrt(b) for a
+ *   power of two, else the identity). Q(0) = I, so B(0) = G [HARP gist.science summary, 2.2:
+ *   Cayley map for b_t > 2]. out: b * b floats. Host only, double precision. */
+rot_status rot_harp_cayley_block(const double* params, int b, const float* mixer, float* out);
+
+/* Build a plan from HARP parameters stored in int8 [HARP gist.science summary, 2.4 (storage in
+ * int8) and 4 (2.00 -> 2.05 bits per parameter)]: stage t's parameters are
+ * theta = codes[t][i] * scales[t] (one fp32 scale per stage).
+ *   codes[t]   NULL (theta = 0: the block is the stage's mixer) or host int8:
+ *              b_t == 2: n_blocks[t] Givens angles, B = R(theta) H_2 / sqrt(2);
+ *              b_t >  2: n_blocks[t] * b(b-1)/2 Cayley parameters per block (rot_harp_cayley_block
+ *              order), B = Q(theta) G_b
+ *   scales     host fp32[n_stages] (read for stages with codes)
+ *   n_blocks   host int64[n_stages]: 1 or K / b_t for stages with codes
+ *   mixers     NULL or host array of n_stages pointers: NULL (base mixer) or a b x b fp32 G_b
+ *              (e.g. the QR fallback, rot_harp_qr_block); radix-2 stages take none
+ *   perms, signs as for rot_plan_create.
+ * The Givens blocks are computed on the device from the int8 codes when the plan is loaded
+ * (sincosf in fp32); Cayley blocks are built on the host in double. The kernels then read the
+ * expanded fp32 blocks, so rot_apply / rot_quant cost the same as with an fp32 plan.
+ * Errors: as rot_plan_create; ROT_EINVAL for a missing scale / n_blocks or a radix-2 mixer. */
+rot_status rot_plan_create_q8(rot_plan_t* out, int K, int n_stages, const int* radices,
+                              const int8_t* const* codes, const float* scales, const int64_t* n_blocks,
+                              const float* const* mixers, const int32_t* const* perms, const int8_t* signs);
 
 /* Synchronise the current device and report device-side errors recorded by bounded
  * waits (ROT_ETIMEOUT) since the last call; clears the record. */

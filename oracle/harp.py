@@ -60,6 +60,56 @@ def qr_block(gauss: np.ndarray) -> np.ndarray:
     return Q * d[None, :]
 
 
+def cayley(params: np.ndarray, b: int) -> np.ndarray:
+    """Cayley map of a b x b skew-symmetric matrix S built from its b(b-1)/2 strictly upper
+    entries (row-major order: S[i, j] = p_k for i < j, S[j, i] = -p_k):
+    Q(S) = (I + S)^{-1} (I - S)  (= (I - S)(I + S)^{-1}; the two factors commute).
+
+    Source: HARP gist.science summary, section 2.2: Q_{t,c}(theta) is a learnable orthogonal
+    matrix, a Cayley map for b_t > 2, with Q(0) = I. Reading: the standard Cayley transform of a
+    skew-symmetric matrix (orthogonal with determinant +1); the page does not fix the sign
+    convention or the parameter order.
+    """
+    p = np.asarray(params, dtype=np.float64).reshape(-1)
+    if p.size != b * (b - 1) // 2:
+        raise ValueError("a b x b Cayley block takes b(b-1)/2 parameters")
+    S = np.zeros((b, b))
+    iu = np.triu_indices(b, 1)
+    S[iu] = p
+    S -= S.T
+    eye = np.eye(b)
+    return np.linalg.solve(eye + S, eye - S)
+
+
+def cayley_blocks(params: np.ndarray, b: int, mixer: np.ndarray | None = None) -> np.ndarray:
+    """B = Q(theta) G_b for each parameter row (HARP summary, section 2.2: B = Q(theta) G,
+    G the base mixer: normalised Sylvester-Hadamard for powers of two, else the given fallback
+    mixer, e.g. the QR of a fixed Gaussian). params: [n, b(b-1)/2] -> [n, b, b]."""
+    G = base_mixer(b) if mixer is None else np.asarray(mixer, dtype=np.float64)
+    P = np.asarray(params, dtype=np.float64).reshape(-1, b * (b - 1) // 2)
+    return np.stack([cayley(p, b) @ G for p in P])
+
+
+def quant_params_int8(theta: np.ndarray):
+    """Store a stage's parameters in int8 (HARP gist.science summary, section 2.4: the
+    parameters can be stored in int8 with minimal effect; section 4: 2.00 -> 2.05 bits per
+    parameter). Reading: one symmetric absmax scale per stage, s = fp32(max|theta| / 127),
+    codes q = clamp(round_half_away(theta / s), -127, 127); s = 0 gives q = 0.
+    Returns (codes int8, scale float32)."""
+    th = np.asarray(theta, dtype=np.float64)
+    s = np.float32(np.max(np.abs(th)) / 127.0) if th.size else np.float32(0.0)
+    if s == 0:
+        return np.zeros(th.shape, dtype=np.int8), np.float32(0.0)
+    v = th / np.float64(s)
+    q = np.clip(np.sign(v) * np.floor(np.abs(v) + 0.5), -127, 127)
+    return q.astype(np.int8), s
+
+
+def dequant_params_int8(codes: np.ndarray, scale) -> np.ndarray:
+    """theta = q * s in fp64 (s the stored fp32 scale)."""
+    return np.asarray(codes, dtype=np.float64) * np.float64(np.float32(scale))
+
+
 @dataclass
 class HarpSpec:
     K: int
@@ -106,6 +156,24 @@ def spec_from_draws(draws, signs: np.ndarray | None, variant: str) -> HarpSpec:
             raise ValueError(variant)
     perms = list(draws.perms) if variant == "random" else [None] * len(radices)
     return HarpSpec(K, radices, blocks, perms, signs)
+
+
+def spec_from_q8(draws, signs: np.ndarray | None) -> HarpSpec:
+    """A processor stored with int8 parameters (``workloads.harp_q8_draws``): per stage
+    theta = code * scale (dequant_params_int8); Givens blocks for b = 2, Cayley blocks
+    Q(theta) G_b for b > 2 with G_b the Sylvester-Hadamard mixer (powers of two) or the QR
+    fallback of the drawn Gaussian; the drawn permutations between stages."""
+    radices = list(draws.radices)
+    K = int(np.prod(radices))
+    blocks = []
+    for t, b in enumerate(radices):
+        th = dequant_params_int8(draws.codes[t], draws.scales[t])
+        if b == 2:
+            blocks.append(givens_blocks(th))
+        else:
+            mix = None if draws.mixer_gaussians[t] is None else qr_block(draws.mixer_gaussians[t])
+            blocks.append(cayley_blocks(th, b, mix))
+    return HarpSpec(K, radices, blocks, list(draws.perms), signs)
 
 
 def _stage_blocks(spec: HarpSpec, t: int) -> np.ndarray:

@@ -36,6 +36,29 @@ def w4a4_reference(qa: np.ndarray, sa16: np.ndarray, qw: np.ndarray, sw16: np.nd
     return np.einsum("mg,ng,mng->mn", sa, sw, P)
 
 
+def w4a8_reference(qa8: np.ndarray, sa16: np.ndarray, qw: np.ndarray, sw16: np.ndarray, G: int) -> np.ndarray:
+    """The W4A8 linear (int8 activation codes, int4 weight codes; the wiki's "W4A8 (act8/wt4)"
+    row): the same definition, C[m, n] = sum_g float(sa[m,g]) * float(sw[n,g]) * P[m,n,g] with
+    exact int64 group sums of the int8 x int4 products, in fp64."""
+    return w4a4_reference(qa8, sa16, qw, sw16, G)
+
+
+def two_sided_weights(B: np.ndarray, rot_in, rot_out) -> np.ndarray:
+    """Offline weight preparation of a two-sided processor (HARP abstract: a two-sided orthogonal
+    processor). With the input-side operator T (``rot_in``: rows x -> T x, size K) and the
+    output-side operator U (``rot_out``: rows x -> U x, size N), B~ = T B U^T; returned as the rows
+    of B~^T [N, K] (what is quantised): the rows of B (length N) go through U, then the columns
+    of B U^T (length K) through T."""
+    BU = rot_out(np.asarray(B, dtype=np.float64))        # rows of B -> U b: B U^T  [K, N]
+    return rot_in(np.ascontiguousarray(BU.T))            # columns of B U^T -> T col: (T B U^T)^T
+
+
+def unrotate_output(Ct: np.ndarray, rot_out_inv) -> np.ndarray:
+    """Rows c~ = U c of the two-sided linear's output back to c = U^T c~ (``rot_out_inv``: rows
+    x -> U^T x)."""
+    return rot_out_inv(np.asarray(Ct, dtype=np.float64))
+
+
 def _quant_dequant_rows(X: np.ndarray, bits: int, G: int) -> np.ndarray:
     q, s = Q.quantize(X, bits, G)
     return Q.dequantize(q, s, G).astype(np.float64)

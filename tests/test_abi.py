@@ -185,3 +185,30 @@ def test_test_inject_rejects_unknown_faults(lib):
     with pytest.raises(lib.RotError):
         lib.test_inject(0, -1)
     lib.test_inject(lib.ROT_TEST_NONE, 0)
+
+
+@pytest.mark.parametrize("b", [2, 3, 5, 8, 43])
+def test_cayley_block_matches_oracle(lib, b):
+    g = W.rng(b + 100)
+    p = g.standard_normal(b * (b - 1) // 2) * 0.4
+    mix = None if b in (2, 8) else Hp.qr_block(g.standard_normal((b, b))).astype(np.float32)
+    got = lib.harp_cayley_block(p, b, mix).astype(np.float64)
+    ref = Hp.cayley_blocks(p[None], b, None if mix is None else mix.astype(np.float64))[0]
+    assert np.max(np.abs(got - ref)) < 2e-6
+    assert np.max(np.abs(got @ got.T - np.eye(b))) < 2e-6
+
+
+def test_plan_q8_rejects_bad_arguments_without_a_device(lib):
+    import ctypes as C
+    h = C.c_void_p()
+    rad = (C.c_int * 2)(2, 3)
+    codes = (C.c_int8 * 3)(1, 2, 3)
+    cp = (C.POINTER(C.c_int8) * 2)(C.cast(codes, C.POINTER(C.c_int8)), C.POINTER(C.c_int8)())
+    # a stage with codes but no scales / n_blocks
+    st = lib._lib.rot_plan_create_q8(C.byref(h), 6, 2, rad, cp, None, None, None, None, None)
+    assert st == lib.ROT_EINVAL
+    # a radix-2 stage given a mixer
+    mix = (C.c_float * 4)(1, 0, 0, 1)
+    mp = (C.POINTER(C.c_float) * 2)(C.cast(mix, C.POINTER(C.c_float)), C.POINTER(C.c_float)())
+    st = lib._lib.rot_plan_create_q8(C.byref(h), 6, 2, rad, None, None, None, mp, None, None)
+    assert st == lib.ROT_EINVAL and "mixer" in lib.last_error()

@@ -114,3 +114,36 @@ def test_w4a4_end_to_end_rotated_pipeline(lib, M):
     qw0, sw0 = Q.quantize(Wt, bits, G)
     err_plain = np.linalg.norm(L.w4a4_reference(qa0, sa0, qw0, sw0, G) - exact) / np.linalg.norm(exact)
     assert err_rot < 0.8 * err_plain
+
+
+@pytest.mark.parametrize("name", ["q_proj_prefill", "q_proj_decode", "up_proj_prefill"])
+@pytest.mark.parametrize("out", ["f32", "bf16"])
+def test_w4a4_linear_act_full_size(lib, name, out):
+    """The one-call online path (rotate + quantise the bf16 activations into a workspace, then the
+    linear, launched as a programmatic dependent): the workspace codes and scales against the
+    oracle on sampled rows, and C against the oracle linear on those codes."""
+    import torch
+    from parity import POISON, Guarded
+    wl = W.make_workload(name)
+    bits, G = wl.quant[0]
+    plan = lib.Plan.rht(wl.K, wl.signs)
+    Wq, Ws = guarded_quant(lib, to_device(np.ascontiguousarray(wl.W.T), False), plan, bits, G)
+    N = Wq.shape[0]
+    nbytes = lib.w4a4_linear_act_workspace(wl.M, wl.K, G)
+    ws = Guarded((nbytes,), torch.uint8, POISON["codes4"])
+    dt = torch.float32 if out == "f32" else torch.bfloat16
+    C = Guarded((wl.M, N), dt, POISON["f32" if out == "f32" else "bf16"])
+    lib.w4a4_linear_act(to_device(wl.A, True), plan, Wq, Ws, G, out=C.t, workspace=ws.t)
+    C.check()
+    ws.check()
+    lib.check_device()
+    cbytes = -(-wl.M * wl.K // 2 // 16) * 16
+    codes = ws.t[:wl.M * wl.K // 2].view(wl.M, wl.K // 2)
+    scales = ws.t[cbytes:cbytes + wl.M * (wl.K // G) * 2].view(torch.float16).view(wl.M, wl.K // G)
+    rows = sample_rows(wl.M, 16)
+    idx = rows.tolist()
+    assert_codes_match(codes[idx].cpu().numpy(), scales[idx].cpu().numpy(), Hd.rht_apply(wl.A[rows], wl.signs),
+                       bits, G, what="w4a4_linear_act workspace")
+    qa, sa = Q.unpack(codes[idx].cpu().numpy(), 4, wl.K), scales[idx].cpu().numpy()
+    C_ref = L.w4a4_reference(qa, sa, Q.unpack(Wq.cpu().numpy(), 4, wl.K), Ws.cpu().numpy(), G)
+    assert_linear_close(C.t[idx].float().cpu().numpy(), C_ref, tol=1e-4 if out == "f32" else 2 ** -8)

@@ -439,3 +439,78 @@ def test_plain_cpu_baseline_edge_cases():
     assert not ((Q.unpack(codes, 4, K) != q_ref) & ~cflag).any()
     # a constant row puts all its energy in coordinate 0 (no signs): group 0's scale overflows to inf
     assert np.isinf(scales[2, 0].astype(np.float32)) and (Q.unpack(codes, 4, K)[2] == 0).all()
+
+
+# ----------------------------------------------------------------------------- Cayley blocks, int8 parameters
+
+def test_cayley_b2_is_the_rotation_by_twice_the_arctangent():
+    """Closed form: for S = [[0, t], [-t, 0]], (I + S)^{-1}(I - S) = [[1 - t^2, -2t], [2t, 1 - t^2]] / (1 + t^2),
+    the rotation by 2 atan(t) (a textbook identity of the Cayley transform)."""
+    for t in (0.0, 0.3, -1.7, 5.0):
+        Q = Hp.cayley(np.array([t]), 2)
+        phi = 2.0 * np.arctan(t)
+        R = np.array([[np.cos(phi), -np.sin(phi)], [np.sin(phi), np.cos(phi)]])
+        assert np.max(np.abs(Q - R)) < 1e-14
+
+
+@pytest.mark.parametrize("b", [3, 5, 8, 43])
+def test_cayley_orthogonal_det_one_and_inverse(b):
+    g = W.rng(b)
+    p = g.standard_normal(b * (b - 1) // 2) * 0.7
+    Q = Hp.cayley(p, b)
+    assert np.max(np.abs(Q @ Q.T - np.eye(b))) < 1e-12
+    assert abs(np.linalg.det(Q) - 1.0) < 1e-10
+    # the inverse map S = (I - Q)(I + Q)^{-1} gives back the skew-symmetric matrix
+    S = (np.eye(b) - Q) @ np.linalg.inv(np.eye(b) + Q)
+    iu = np.triu_indices(b, 1)
+    assert np.max(np.abs(S + S.T)) < 1e-10 and np.max(np.abs(S[iu] - p)) < 1e-10
+    assert np.array_equal(Hp.cayley(np.zeros_like(p), b), np.eye(b))   # Q(0) = I
+
+
+def test_cayley_blocks_at_zero_are_the_base_mixer():
+    """B(0) = G_b (summary 2.2): Sylvester-Hadamard for b = 8, the given fallback for b = 5."""
+    assert np.max(np.abs(Hp.cayley_blocks(np.zeros((1, 28)), 8)[0] - Hd.sylvester(8) / np.sqrt(8))) < 1e-15
+    G5 = Hp.qr_block(W.rng(1).standard_normal((5, 5)))
+    assert np.array_equal(Hp.cayley_blocks(np.zeros((2, 10)), 5, G5)[1], G5)
+
+
+def test_int8_parameter_storage():
+    th = np.array([0.0, 1.0, -2.54, 2.54, 0.01, -1.27])
+    q, s = Hp.quant_params_int8(th)
+    assert s == np.float32(2.54 / 127)
+    assert q.dtype == np.int8 and q[2] == -127 and q[3] == 127 and q[0] == 0
+    back = Hp.dequant_params_int8(q, s)
+    assert np.all(np.abs(back - th) <= float(s) / 2 + 1e-12)
+    # a tie rounds away from zero: theta = 2.5 s exactly
+    s0 = np.float32(0.5)
+    q2, _ = Hp.quant_params_int8(np.array([63.5, 2.5 * float(s0), -1.25]))   # scale 0.5
+    assert list(q2) == [127, 3, -3]
+    z, sz = Hp.quant_params_int8(np.zeros(5))
+    assert sz == 0 and not z.any()
+
+
+# ----------------------------------------------------------------------------- two-sided processor
+
+def test_two_sided_exact_equivalence():
+    """(A T^T)(T B U^T) U = A B in fp64 to 1e-12, with T an RHT of size K and U a random HARP
+    processor of size N (mixed radix with permutations), both applied through the oracle."""
+    K, N = 256, 96
+    g = W.rng(21)
+    A = g.standard_normal((7, K))
+    B = g.standard_normal((K, N))
+    sT = W.signs(g, K)
+    radU = [2, 3, 2, 2, 2, 2]
+    spec = Hp.HarpSpec(N, radU, [np.stack([Hp.qr_block(g.standard_normal((b, b))) for _ in range(N // b)])
+                                 for b in radU], [g.permutation(N).astype(np.int32), None, None, None, None, None],
+                       (1 - 2 * g.integers(0, 2, N)).astype(np.int8))
+    rot_in = lambda X: Hd.rht_apply(X, sT)
+    rot_out = lambda X: Hp.harp_apply(X, spec)
+    rot_out_inv = lambda X: Hp.harp_apply(X, spec, inverse=True)
+    Bt = L.two_sided_weights(B, rot_in, rot_out)           # rows of (T B U^T)^T
+    Ct = rot_in(A) @ Bt.T                                  # (A T^T)(T B U^T) = A B U^T
+    C = L.unrotate_output(Ct, rot_out_inv)
+    ref = A @ B
+    assert np.linalg.norm(C - ref) / np.linalg.norm(ref) < 1e-12
+    # each output row of the rotated product is U c (the output side is really rotated)
+    assert np.linalg.norm(Ct - rot_out(ref)) / np.linalg.norm(ref) < 1e-12
+    assert np.linalg.norm(Ct - ref) / np.linalg.norm(ref) > 0.1

@@ -41,6 +41,8 @@ __all__ = [
     "weights",
     "HarpDraws",
     "harp_draws",
+    "HarpQ8Draws",
+    "harp_q8_draws",
     "to_bf16_exact",
     "WORKLOADS",
     "Workload",
@@ -129,6 +131,42 @@ def harp_draws(seed: int, radices: list[int], *, per_block_gaussian: bool = Fals
             d.perms.append(g.permutation(K).astype(np.int32))
         else:
             d.perms.append(None)
+    return d
+
+
+@dataclass
+class HarpQ8Draws:
+    """Raw random numbers of a HARP processor stored with int8 parameters: per stage int8 codes
+    and an fp32 scale (theta = code * scale); Givens stages (b = 2) hold one code per block, the
+    other stages b(b-1)/2 Cayley codes per block and, for a non-power-of-two radix, a Gaussian
+    b x b matrix whose QR factor is the fallback base mixer. No block is built here."""
+
+    radices: list[int]
+    codes: list[np.ndarray] = field(default_factory=list)           # [n_blocks] or [n_blocks, b(b-1)/2] int8
+    scales: list[float] = field(default_factory=list)
+    mixer_gaussians: list[np.ndarray | None] = field(default_factory=list)
+    perms: list[np.ndarray | None] = field(default_factory=list)
+
+
+def harp_q8_draws(seed: int, radices: list[int], *, per_block: bool = True, with_perms: bool = True,
+                  cayley_range: float = 0.3) -> HarpQ8Draws:
+    """Seeded int8-stored HARP parameters: codes uniform in [-127, 127]; Givens scale pi / 127
+    (angles over [-pi, pi]), Cayley scale cayley_range / 127."""
+    K = int(np.prod(radices))
+    g = rng(seed)
+    d = HarpQ8Draws(list(radices))
+    for b in radices:
+        n = K // b if per_block else 1
+        if b == 2:
+            d.codes.append(g.integers(-127, 128, n).astype(np.int8))
+            d.scales.append(float(np.float32(np.pi / 127)))
+            d.mixer_gaussians.append(None)
+        else:
+            d.codes.append(g.integers(-127, 128, (n, b * (b - 1) // 2)).astype(np.int8))
+            d.scales.append(float(np.float32(cayley_range / 127)))
+            d.mixer_gaussians.append(None if (b & (b - 1)) == 0 else g.standard_normal((b, b)))
+    for t in range(len(radices)):
+        d.perms.append(g.permutation(K).astype(np.int32) if (with_perms and t < len(radices) - 1) else None)
     return d
 
 
