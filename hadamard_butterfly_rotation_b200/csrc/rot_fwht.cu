@@ -631,9 +631,12 @@ __global__ void __launch_bounds__(Cfg<LOGN>::THREADS, 1) fwht_kernel(const Args 
 //   phase B after a transpose through shared memory (XOR-swizzled 16-byte chunks, no bank
 //           conflicts either way) lane l holds the contiguous coordinates 64 l .. 64 l + 63:
 //           butterflies over e3..e5, then group quantisation and packing as in fwht_kernel.
-constexpr int MMA_THREADS = 640;               // 20 warps, one chunk each
-constexpr int MMA_SLOTS = MMA_THREADS / 32;
-static_assert(MMA_SLOTS % 2 == 0, "the sign table after the slot barriers must stay 16-byte aligned");
+#ifndef ROT_MMA_WARPS
+#define ROT_MMA_WARPS 20
+#endif
+constexpr int MMA_SLOTS = ROT_MMA_WARPS;          // warps per CTA, one chunk each
+constexpr int MMA_THREADS = MMA_SLOTS * 32;
+constexpr int MMA_BARS = (MMA_SLOTS + 1) & ~1;    // even: the sign table after them stays 16-byte aligned
 constexpr int MMA_SSTRIDE = 2048 + 4;          // floats per slot buffer
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
@@ -664,7 +667,7 @@ __global__ void __launch_bounds__(MMA_THREADS, 1) fwht_mma_kernel(const Args a) 
   extern __shared__ __align__(128) float smem[];
   float* sbuf = smem;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + MMA_SLOTS * MMA_SSTRIDE);
-  uint32_t* smf = reinterpret_cast<uint32_t*>(bars + MMA_SLOTS);  // sign masks, fragment order
+  uint32_t* smf = reinterpret_cast<uint32_t*>(bars + MMA_BARS);   // sign masks, fragment order
 
   const int slot = threadIdx.x >> 5;
   const int l = threadIdx.x & 31;
@@ -911,7 +914,7 @@ __global__ void __launch_bounds__(DB_THREADS, 1) fwht_mma_db_kernel(const Args a
 }
 
 size_t mma_smem_bytes(int K) {
-  return (size_t)MMA_SLOTS * MMA_SSTRIDE * 4 + (size_t)MMA_SLOTS * 8 + (size_t)(K / 2) * 4;
+  return (size_t)MMA_SLOTS * MMA_SSTRIDE * 4 + (size_t)MMA_BARS * 8 + (size_t)(K / 2) * 4;
 }
 
 // Programmatic dependent launch (the kernel's prologue may overlap the previous kernel in

@@ -58,7 +58,6 @@ constexpr int A_STAGE_BYTES = BM * KB;   // unpacked int8
 constexpr int B_STAGE_BYTES = BN * KB;
 constexpr int STAGE_BYTES = A_STAGE_BYTES + B_STAGE_BYTES;
 constexpr int PROW_BYTES = KB / 2;       // packed bytes of one row in one K-block
-constexpr int PSTAGE_BYTES = (BM + BN) * PROW_BYTES;
 constexpr int N_EPI = 256;               // epilogue threads (2 warpgroups)
 constexpr int N_EPI_WARPS = N_EPI / 32;
 constexpr int LOADER_WARP = N_EPI / 32;  // warp 8

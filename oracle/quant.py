@@ -124,8 +124,10 @@ def _fp16_midpoint_distance(x: np.ndarray) -> np.ndarray:
 def boundary_flags(y: np.ndarray, bits: int, G: int, eps: float = 1e-5):
     """Elements whose decision lies within ``eps`` of a rounding boundary.
 
-    * code flag: with the oracle's scale s, v = y / s (fp64) lies within eps of a
-      half-integer (the rounding boundary of round-to-nearest);
+    * code flag: with the oracle's scale s, v = y / s (fp64) lies within eps * max(1, |v|) of a
+      half-integer (the rounding boundary of round-to-nearest): the window is relative to the
+      pre-rounding value, as the rotated values it is computed from are known to 1e-5 relative
+      (absolute 1e-5 below |v| = 1; up to 7.5e-5 for int4 and 1.3e-3 for int8 codes);
     * scale flag: absmax/qmax (fp64) lies within eps (relative) of a binary16
       rounding midpoint, so an fp32 computation of the scale may round the other
       way; every code of such a group is flagged.
@@ -143,7 +145,7 @@ def boundary_flags(y: np.ndarray, bits: int, G: int, eps: float = 1e-5):
         v = np.abs(g) / s[..., None]
     v = np.where((s == 0)[..., None], 0.0, v)
     frac = v - np.floor(v)
-    code_flag = np.abs(frac - 0.5) < eps
+    code_flag = np.abs(frac - 0.5) < eps * np.maximum(1.0, v)
     group_flag = _fp16_midpoint_distance(m / qm) < eps
     code_flag |= group_flag[..., None]
     return code_flag.reshape(M, K), group_flag
