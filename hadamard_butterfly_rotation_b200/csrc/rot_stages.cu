@@ -348,7 +348,7 @@ __global__ void __launch_bounds__(MR_THREADS, 1) stages_rows_kernel(const MrArgs
         const float magic = magic_of_bits(a.bits);
         const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
         const int ngr = K / a.G;
-        const int lpw = a.bits / 2;            // lanes per 32-bit code word (4 codes per lane)
+        const int lpw = 8 / a.bits;            // lanes per 32-bit code word (4 codes per lane)
         for (int g = warp; g < ngr; g += MR_THREADS / 32) {
           const float* gx = xr + (int64_t)g * a.G;
           float m = 0.0f;
