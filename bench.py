@@ -532,6 +532,7 @@ def run_extra(hbr, W, dev, stream, peaks):
                                "frac_int8_spec": round(ops / t / 1e12 / INT8_DENSE_SPEC_TOPS, 4),
                                "frac_int8_measured": round(ops / t / 1e12 / int8_peak, 4) if int8_peak else None,
                                "GB/s": round(wbytes / t / 1e9, 1)}
+    out.update(run_extra_next(hbr, W, dev, hbm, int8_peak))
     out["int8_peak_measured_TOPS"] = round(int8_peak, 1) if int8_peak else None
     # roofline of the prefill linear: int8 dense peak = the measured bf16 burst peak x 2 (the
     # nominal int8 : bf16 dense ratio, 4.5 : 2.25 PFLOP/s)
@@ -545,6 +546,66 @@ def run_extra(hbr, W, dev, stream, peaks):
             "peak_source": "measured bf16 burst (MEASURED_PEAKS.json bf16_tflops) x 2, the nominal int8:bf16 ratio",
             "same_run_torch_int_mm_TOPS": out["int8_peak_measured_TOPS"],
             "spec_dense_int8_TOPS": INT8_DENSE_SPEC_TOPS}
+    return out
+
+
+def run_extra_next(hbr, W, dev, hbm, int8_peak):
+    """Timings of the paths beyond the headline: the W4A8 linear, the two-sided linear, the
+    one-call online path, int8-stored and per-block HARP processors, and K = 5120."""
+    import torch
+    out = {}
+    for name in ("q_proj_prefill", "q_proj_decode"):
+        wl = W.make_workload(name)
+        bits, G = wl.quant[0]
+        plan = hbr.Plan.rht(wl.K, wl.signs)
+        dA = torch.from_numpy(wl.A).to(torch.bfloat16).to(dev)
+        Wq, Ws = hbr.rot_quant(torch.from_numpy(np.ascontiguousarray(wl.W.T)).to(dev), plan, bits, G)
+        N = Wq.shape[0]
+        C = torch.empty((wl.M, N), dtype=torch.bfloat16, device=dev)
+        n = 50 if wl.M > 16 else 200
+        ops = 2.0 * wl.M * N * wl.K
+        # W4A8: int8 activation codes
+        A8, S8 = hbr.rot_quant(dA, plan, 8, G)
+        A8i = A8.view(torch.int8)
+        t = _graph_time(lambda i: hbr.w4a8_linear(A8i, S8, Wq, Ws, G, out=C), n, 10)
+        out[f"w4a8_{name}"] = {"us": round(t * 1e6, 2), "TOPS": round(ops / t / 1e12, 1),
+                               "frac_int8_measured": round(ops / t / 1e12 / int8_peak, 4) if int8_peak else None}
+        # one call: rotate + quantise the bf16 activations, then the linear
+        ws = torch.empty(hbr.w4a4_linear_act_workspace(wl.M, wl.K, G), dtype=torch.uint8, device=dev)
+        t = _graph_time(lambda i: hbr.w4a4_linear_act(dA, plan, Wq, Ws, G, out=C, workspace=ws), n, 10)
+        A4, S4 = hbr.rot_quant(dA, plan, 4, G)
+
+        def sep(i):
+            hbr.rot_quant(dA, plan, 4, G, codes=A4, scales=S4)
+            hbr.w4a4_linear(A4, S4, Wq, Ws, G, out=C)
+        t2 = _graph_time(sep, n, 10)
+        out[f"act_path_{name}"] = {"us": round(t * 1e6, 2), "separate_calls_us": round(t2 * 1e6, 2)}
+        # two-sided: the output rows returned through an RHT of size N
+        U = hbr.Plan.rht(N, W.signs(W.rng(77), N))
+        t = _graph_time(lambda i: hbr.w4a4_linear_rot(A4, S4, Wq, Ws, G, U, out=C), n, 10)
+        out[f"two_sided_{name}"] = {"us": round(t * 1e6, 2)}
+    # HARP K = 11008 with int8-stored parameters (256 Cayley blocks of radix 43), the fp32
+    # per-block QR variant, and 5120 = (8, 8, 8, 5, 2)
+    wl = W.make_workload("harp11008")
+    dA = torch.from_numpy(wl.A).to(torch.bfloat16).to(dev)
+    codes = torch.empty((wl.M, wl.K // 2), dtype=torch.uint8, device=dev)
+    scales = torch.empty((wl.M, wl.K // 128), dtype=torch.float16, device=dev)
+    plans = {"harp11008_q8_cayley_per_block": hbr.harp_q8_plan(W.harp_q8_draws(4, wl.extra["radices"]), wl.signs),
+             "harp11008_random_per_block_qr": hbr.harp_plan(W.harp_draws(2, wl.extra["radices"], per_block_gaussian=True),
+                                                            wl.signs, "random")}
+    for key, plan in plans.items():
+        t = _graph_time(lambda i: hbr.rot_quant(dA, plan, 4, 128, codes=codes, scales=scales), 10, 5)
+        b = algorithmic_bytes(wl.M, wl.K, 4, 128)
+        out[f"{key}_int4_G128"] = {"us": round(t * 1e6, 2), "GB/s": round(b / t / 1e9, 1)}
+    K = 5120
+    g = W.rng(10)
+    A = torch.from_numpy(W.activations(g, 4096, K, outlier_frac=0.01, outlier_scale=20.0)).to(torch.bfloat16).to(dev)
+    plan = hbr.harp_q8_plan(W.harp_q8_draws(9, [8, 8, 8, 5, 2]), W.signs(g, K))
+    codes = torch.empty((4096, K // 2), dtype=torch.uint8, device=dev)
+    scales = torch.empty((4096, K // 128), dtype=torch.float16, device=dev)
+    t = _graph_time(lambda i: hbr.rot_quant(A, plan, 4, 128, codes=codes, scales=scales), 10, 5)
+    b = algorithmic_bytes(4096, K, 4, 128)
+    out["harp5120_q8_A4096_int4_G128"] = {"us": round(t * 1e6, 2), "GB/s": round(b / t / 1e9, 1)}
     return out
 
 
