@@ -225,13 +225,15 @@ __device__ __forceinline__ void stage_pairs(float2 (&xp)[NP], int b) {
 
 // Quantise the E values a thread holds (coordinates c0 .. c0+E-1 of one row) and store
 // packed codes and scales. GT > 0: compile-time group size; GT == 0: runtime a.G.
-template <int LOGN, int BITS, int GT, int E, int TPC>
-__device__ __forceinline__ void quantise_store(const Args& a, const float2 (&xp)[E / 2], int64_t row, int c0, int t) {
+// srow: the scales of the row (or of the chunk: any base whose group 0 starts at coordinate 0 of
+// c0's frame); dst: this thread's first code word; c0: its first coordinate in that frame.
+template <int BITS, int GT, int E, int TPC>
+__device__ __forceinline__ void quantise_store_at(const Args& a, const float2 (&xp)[E / 2], uint16_t* srow,
+                                                  uint32_t* dst, int c0, int t) {
   constexpr float QMAX = qmax_of_bits(BITS);
   constexpr float MAGIC = magic_of_bits(BITS);  // 2^23 + qmax + 1
   constexpr int CPW = 32 / BITS;   // codes per 32-bit word
   constexpr int NWD = E / CPW;     // words per thread
-  uint16_t* srow = a.scales + row * a.ngroups;
   uint32_t words[NWD];
   if constexpr (GT > 0) {
     constexpr int GE = GT <= E ? GT : E;     // elements of one group held by this thread
@@ -378,7 +380,6 @@ __device__ __forceinline__ void quantise_store(const Args& a, const float2 (&xp)
       else words[w] = pack16_int2(*reinterpret_cast<const uint32_t(*)[16]>(tt));
     }
   }
-  uint32_t* dst = reinterpret_cast<uint32_t*>(a.codes + row * (int64_t)(a.K / CPW) * 4) + c0 / CPW;
   if constexpr (NWD >= 4) {
 #pragma unroll
     for (int v = 0; v < NWD / 4; ++v)
@@ -388,6 +389,13 @@ __device__ __forceinline__ void quantise_store(const Args& a, const float2 (&xp)
   } else {
     dst[0] = words[0];
   }
+}
+
+template <int LOGN, int BITS, int GT, int E, int TPC>
+__device__ __forceinline__ void quantise_store(const Args& a, const float2 (&xp)[E / 2], int64_t row, int c0, int t) {
+  constexpr int CPW = 32 / BITS;
+  uint32_t* dst = reinterpret_cast<uint32_t*>(a.codes + row * (int64_t)(a.K / CPW) * 4) + c0 / CPW;
+  quantise_store_at<BITS, GT, E, TPC>(a, xp, a.scales + row * a.ngroups, dst, c0, t);
 }
 
 // Sign masks in shared memory: one word per bf16 pair (bits 15 and 31), or, for the bf16
@@ -637,7 +645,7 @@ __global__ void __launch_bounds__(Cfg<LOGN>::THREADS, 1) fwht_kernel(const Args 
 constexpr int MMA_SLOTS = ROT_MMA_WARPS;          // warps per CTA, one chunk each
 constexpr int MMA_THREADS = MMA_SLOTS * 32;
 constexpr int MMA_BARS = (MMA_SLOTS + 1) & ~1;    // even: the sign table after them stays 16-byte aligned
-constexpr int MMA_SSTRIDE = 2048 + 4;          // floats per slot buffer
+constexpr int MMA_SSTRIDE = 2048 + 64;         // floats per slot buffer (256-byte multiple)
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
@@ -661,18 +669,37 @@ __host__ __device__ constexpr uint32_t h16_bf16(int k, int o) {
   return par ? 0xBF80u : 0x3F80u;
 }
 
+// 32-bit shared-state-space accesses (addresses computed once per lane, offsets folded in)
+__device__ __forceinline__ void sts64(uint32_t addr, float2 v) {
+  asm volatile("st.shared.v2.f32 [%0], {%1, %2};" ::"r"(addr), "f"(v.x), "f"(v.y) : "memory");
+}
+__device__ __forceinline__ float4 lds128f(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr) : "memory");
+  return v;
+}
+__device__ __forceinline__ uint4 lds128u(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr) : "memory");
+  return v;
+}
+
 template <int BITS, int GT>
 __global__ void __launch_bounds__(MMA_THREADS, 1) fwht_mma_kernel(const Args a) {
-  constexpr int N = 2048, E = 64, NP = 32;
+  constexpr int N = 2048, NP = 32;
+  constexpr int CPW = 32 / BITS;
   extern __shared__ __align__(128) float smem[];
-  float* sbuf = smem;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + MMA_SLOTS * MMA_SSTRIDE);
+  // slot buffers start on a 256-byte boundary (the transpose addresses below rely on it)
+  const uint32_t sm_raw = smem_addr(smem);
+  const uint32_t sm0 = (sm_raw + 255u) & ~255u;
+  float* sbase_ptr = smem + (sm0 - sm_raw) / 4;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sbase_ptr + MMA_SLOTS * MMA_SSTRIDE);
   uint32_t* smf = reinterpret_cast<uint32_t*>(bars + MMA_BARS);   // sign masks, fragment order
 
   const int slot = threadIdx.x >> 5;
   const int l = threadIdx.x & 31;
   const int g = l >> 2, c = l & 3;
-  float* buf = sbuf + slot * MMA_SSTRIDE;
+  const uint32_t buf_b = sm0 + (uint32_t)(slot * MMA_SSTRIDE * 4);   // this warp's slot buffer
   uint64_t* bar = bars + slot;
   const bool has_signs = a.signmask != nullptr;
 
@@ -686,6 +713,11 @@ __global__ void __launch_bounds__(MMA_THREADS, 1) fwht_mma_kernel(const Args a) 
   auto src_of = [&](int64_t r, int ch) -> const void* {
     return static_cast<const uint8_t*>(a.A) + ((int64_t)r * a.lda + (int64_t)ch * N) * 2;
   };
+  // outputs of unit u (chunk `chunk` of row `row`) are contiguous in u: codes at u * N * bits / 8
+  // bytes, scales at u * N / G (G divides N); this lane's part advances by a constant per unit
+  uint32_t* cdst = reinterpret_cast<uint32_t*>(a.codes) + u * (N / CPW) + (64 * l) / CPW;
+  uint16_t* sdst = a.scales + u * (N / GT);
+  const int64_t cstep = stride * (N / CPW), sstep = stride * (N / GT);
 
   // prologue on plan memory only (see fwht_kernel): barrier, sign table in fragment order
   if (l == 0) {
@@ -703,7 +735,7 @@ __global__ void __launch_bounds__(MMA_THREADS, 1) fwht_mma_kernel(const Args a) 
   asm volatile("griddepcontrol.wait;" ::: "memory");
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   if (l == 0 && u < units && !(a.skip_first && blockIdx.x == 0 && slot == 0))
-    stage_issue(bar, buf, src_of(row, chunk), N * 2);
+    stage_issue(bar, sbase_ptr + slot * MMA_SSTRIDE, src_of(row, chunk), N * 2);
   __syncthreads();
 
   // B fragments of H_16 for the two MMAs (outputs o3 = 0 / 1): n = g, k = 2c + {0,1} (+8)
@@ -714,11 +746,17 @@ __global__ void __launch_bounds__(MMA_THREADS, 1) fwht_mma_kernel(const Args a) 
     hb[q][0] = h16_bf16(2 * c, o) | (h16_bf16(2 * c + 1, o) << 16);
     hb[q][1] = h16_bf16(2 * c + 8, o) | (h16_bf16(2 * c + 9, o) << 16);
   }
-  // ldmatrix row address of this lane (bytes): matrix l >> 3, row l & 7
-  const uint32_t lrow = (uint32_t)(8 * (l & 7) + ((l >> 3) & 1) * 128 + ((l >> 4) & 1) * 64) * 2;
-  const uint32_t sbase = smem_addr(buf);
-  // phase-A store base (element 2c + 8g of each 64-coordinate block, swizzle added per p)
-  const int abase = 2 * c + 8 * g;
+  // ldmatrix row address of this lane: matrix l >> 3, row l & 7
+  const uint32_t ldsm_b = buf_b + (uint32_t)(8 * (l & 7) + ((l >> 3) & 1) * 128 + ((l >> 4) & 1) * 64) * 2;
+  // transpose, phase-A stores: element 2c + 8g + 64 p (+ e0), 16-byte chunks XOR-swizzled by
+  // (p & 7): byte address (buf_b + 8 (c + 4 g)) ^ ((p & 7) << 4) + 256 p (buf_b is 256-aligned
+  // and 8 (c + 4 g) < 256, so the XOR only touches bits 4..6 of the in-buffer offset)
+  const uint32_t wbase = buf_b + (uint32_t)(4 * (2 * c + 8 * g));
+  // phase-B loads: lane l reads floats 64 l + ((4 j) ^ ((l & 7) << 2)): byte address
+  // ((buf_b + 256 l + 16 (l & 7)) ^ (16 (j & 7))) + 128 (j >> 3)
+  const uint32_t rbase = buf_b + (uint32_t)(256 * l + 16 * (l & 7));
+  const uint32_t sgn_b = smem_addr(smf) + 16u * (uint32_t)l;
+  const uint32_t bar_b = smem_addr(bar);
   uint32_t parity = 0;
 
   for (; u < units; u += stride) {
@@ -728,13 +766,13 @@ __global__ void __launch_bounds__(MMA_THREADS, 1) fwht_mma_kernel(const Args a) 
     parity ^= 1u;
 
     // ---------------- MMA: H_16 over {e0, e1, e2, e6} for the 8 row tiles
-    const uint4* sm4 = reinterpret_cast<const uint4*>(smf + (cbase >> 1)) + l;
+    const uint32_t sg = sgn_b + 2u * (uint32_t)cbase;      // this chunk's sign words (fragment order)
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       uint32_t af[4];
-      ldsm_x4(sbase + lrow + i * 512, af);
+      ldsm_x4(ldsm_b + i * 512, af);
       if (has_signs) {
-        const uint4 m = sm4[i * 32];
+        const uint4 m = lds128u(sg + i * 512);
         af[0] ^= m.x; af[1] ^= m.y; af[2] ^= m.z; af[3] ^= m.w;
       }
       // xp index p = e6 + 2 e7 + 4 (e8..e10): MMA q gives e6 = q; rows g / g + 8 give e7
@@ -745,15 +783,14 @@ __global__ void __launch_bounds__(MMA_THREADS, 1) fwht_mma_kernel(const Args a) 
 #pragma unroll
     for (int b = 1; b < 5; ++b) stage_pairs<NP>(xp, b);
 
-    // ---------------- transpose: element e = abase + 64 p (+ e0), physical e ^ ((p & 7) << 2)
+    // ---------------- transpose through the slot buffer (XOR-swizzled 16-byte chunks)
     __syncwarp();   // every lane's ldmatrix reads of the staged row are done
 #pragma unroll
-    for (int p = 0; p < NP; ++p)
-      *reinterpret_cast<float2*>(buf + ((abase ^ ((p & 7) << 2)) + 64 * p)) = xp[p];
+    for (int p = 0; p < NP; ++p) sts64((wbase ^ (uint32_t)((p & 7) << 4)) + 256u * p, xp[p]);
     __syncwarp();
 #pragma unroll
     for (int j = 0; j < 16; ++j) {
-      const float4 q = *reinterpret_cast<const float4*>(buf + 64 * l + ((4 * j) ^ ((l & 7) << 2)));
+      const float4 q = lds128f((rbase ^ (uint32_t)(16 * (j & 7))) + 128u * (j >> 3));
       xp[2 * j] = make_float2(q.x, q.y);
       xp[2 * j + 1] = make_float2(q.z, q.w);
     }
@@ -764,157 +801,27 @@ __global__ void __launch_bounds__(MMA_THREADS, 1) fwht_mma_kernel(const Args a) 
     if (u + stride < units) {
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       __syncwarp();
-      if (l == 0) stage_issue(bar, buf, src_of(nrow, nchunk), N * 2);
+      if (l == 0) {
+        asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar_b), "r"(N * 2) : "memory");
+        asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                         buf_b),
+                     "l"(src_of(nrow, nchunk)), "r"(N * 2), "r"(bar_b)
+                     : "memory");
+      }
     }
     // ---------------- phase B: e3 .. e5 (pair-index bits 2 .. 4)
 #pragma unroll
     for (int b = 2; b < 5; ++b) stage_pairs<NP>(xp, b);
-    const int64_t cur_row = row;
     row = nrow;
     chunk = nchunk;
-    quantise_store<11, BITS, GT, E, 32>(a, xp, cur_row, cbase + 64 * l, l);
-  }
-}
-
-// ---------------------------------------------------------------- double-buffered variant
-// The same per-chunk work as fwht_mma_kernel, with two staging buffers per warp so that the
-// copy of the chunk two units ahead is in flight while the warp computes the current one and
-// the next. A warp's 12 KB region is [S0 | X | S1] (4 KB each): chunk i is staged in S_(i&1),
-// and its fp32 transpose uses the 8 KB window S_(i&1) + X (S0+X or X+S1, contiguous), so the
-// other staging buffer is never touched while its copy is in flight. The copy into S_(i&1) is
-// issued as soon as the transpose has been read back.
-#ifndef ROT_DB_WARPS
-#define ROT_DB_WARPS 18
-#endif
-constexpr int DB_WARPS = ROT_DB_WARPS;         // chunk slots (warps) per CTA
-constexpr int DB_THREADS = DB_WARPS * 32;
-constexpr int DB_REGION = 3 * 1024;            // floats per warp
-
-size_t db_smem_bytes(int K) {
-  return (size_t)DB_WARPS * DB_REGION * 4 + (size_t)DB_WARPS * 2 * 8 + (size_t)(K / 2) * 4;
-}
-
-template <int BITS, int GT>
-__global__ void __launch_bounds__(DB_THREADS, 1) fwht_mma_db_kernel(const Args a) {
-  constexpr int N = 2048, NP = 32;
-  extern __shared__ __align__(128) float smem[];
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + DB_WARPS * DB_REGION);
-  uint32_t* smf = reinterpret_cast<uint32_t*>(bars + 2 * DB_WARPS);  // sign masks, fragment order
-
-  const int slot = threadIdx.x >> 5;
-  const int l = threadIdx.x & 31;
-  const int g = l >> 2, c = l & 3;
-  float* region = smem + slot * DB_REGION;
-  uint64_t* bar = bars + 2 * slot;
-  const bool has_signs = a.signmask != nullptr;
-
-  const int64_t units = a.M * a.chunks;
-  const int64_t stride = (int64_t)gridDim.x * DB_WARPS;
-  int64_t u = (int64_t)blockIdx.x * DB_WARPS + slot;
-  const int64_t drow = stride / a.chunks;
-  const int dchunk = (int)(stride - drow * a.chunks);
-  int64_t row = u / a.chunks;
-  int chunk = (int)(u - row * a.chunks);
-  auto src_of = [&](int64_t r, int ch) -> const void* {
-    return static_cast<const uint8_t*>(a.A) + ((int64_t)r * a.lda + (int64_t)ch * N) * 2;
-  };
-  auto advance = [&](int64_t& r, int& ch) {
-    r += drow;
-    ch += dchunk;
-    if (ch >= a.chunks) { ch -= a.chunks; ++r; }
-  };
-  // cursor of the unit whose copy is issued next (two units ahead of the current one)
-  int64_t lrow = row;
-  int lchunk = chunk;
-  advance(lrow, lchunk);
-
-  if (l == 0) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_addr(bar)) : "memory");
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_addr(bar + 1)) : "memory");
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-  }
-  if (has_signs) {
-    for (int idx = threadIdx.x; idx < a.K / 2; idx += DB_THREADS) {
-      const int ch = idx >> 10, i = (idx >> 7) & 7, ln = (idx >> 2) & 31, r = idx & 3;
-      const int off = ch * N + 8 * (ln >> 2) + 2 * (ln & 3) + 256 * i + ((r & 1) << 7) + ((r & 2) << 5);
-      smf[idx] = a.signmask[off >> 1];
-    }
-  }
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  // (testing hook: slot 0 of CTA 0 issues neither first copy, so nothing is in flight when it gives up)
-  if (l == 0 && !(a.skip_first && blockIdx.x == 0 && slot == 0)) {
-    if (u < units) stage_issue(bar, region, src_of(row, chunk), N * 2);
-    if (u + stride < units) stage_issue(bar + 1, region + 2048, src_of(lrow, lchunk), N * 2);
-  }
-  advance(lrow, lchunk);
-  __syncthreads();
-
-  uint32_t hb[2][2];
-#pragma unroll
-  for (int q = 0; q < 2; ++q) {
-    const int o = 8 * q + g;
-    hb[q][0] = h16_bf16(2 * c, o) | (h16_bf16(2 * c + 1, o) << 16);
-    hb[q][1] = h16_bf16(2 * c + 8, o) | (h16_bf16(2 * c + 9, o) << 16);
-  }
-  const uint32_t lrow_b = (uint32_t)(8 * (l & 7) + ((l >> 3) & 1) * 128 + ((l >> 4) & 1) * 64) * 2;
-  const uint32_t rbase = smem_addr(region);
-  const int abase = 2 * c + 8 * g;
-  uint32_t par = 0;            // bit b: phase parity of staging buffer b
-  int b = 0;
-
-  for (; u < units; u += stride) {
-    const int cbase = chunk * N;
-    float2 xp[NP];
-    if (!stage_wait(bar + b, (par >> b) & 1u, a.wait_ns)) break;
-    par ^= 1u << b;
-    const uint32_t sbase = rbase + (uint32_t)b * 8192u;      // staged bf16 chunk (S0 or S1)
-    float* win = region + b * 1024;                          // transpose window (S0+X or X+S1)
-
-    const uint4* sm4 = reinterpret_cast<const uint4*>(smf + (cbase >> 1)) + l;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      uint32_t af[4];
-      ldsm_x4(sbase + lrow_b + i * 512, af);
-      if (has_signs) {
-        const uint4 m = sm4[i * 32];
-        af[0] ^= m.x; af[1] ^= m.y; af[2] ^= m.z; af[3] ^= m.w;
-      }
-      mma_h16(xp[4 * i + 0], xp[4 * i + 2], af, hb[0][0], hb[0][1]);
-      mma_h16(xp[4 * i + 1], xp[4 * i + 3], af, hb[1][0], hb[1][1]);
-    }
-#pragma unroll
-    for (int bb = 1; bb < 5; ++bb) stage_pairs<NP>(xp, bb);
-
-    __syncwarp();   // every lane's ldmatrix reads of the staged chunk are done
-#pragma unroll
-    for (int p = 0; p < NP; ++p)
-      *reinterpret_cast<float2*>(win + ((abase ^ ((p & 7) << 2)) + 64 * p)) = xp[p];
-    __syncwarp();
-#pragma unroll
-    for (int j = 0; j < 16; ++j) {
-      const float4 q = *reinterpret_cast<const float4*>(win + 64 * l + ((4 * j) ^ ((l & 7) << 2)));
-      xp[2 * j] = make_float2(q.x, q.y);
-      xp[2 * j + 1] = make_float2(q.z, q.w);
-    }
-    // the window is read back: the staging buffer of this chunk takes the copy two units ahead
-    if (u + 2 * stride < units) {
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      __syncwarp();
-      if (l == 0) stage_issue(bar + b, region + b * 2048, src_of(lrow, lchunk), N * 2);
-    }
-    advance(lrow, lchunk);
-#pragma unroll
-    for (int bb = 2; bb < 5; ++bb) stage_pairs<NP>(xp, bb);
-    const int64_t cur_row = row;
-    advance(row, chunk);
-    b ^= 1;
-    quantise_store<11, BITS, GT, 64, 32>(a, xp, cur_row, cbase + 64 * l, l);
+    quantise_store_at<BITS, GT, 64, 32>(a, xp, sdst, cdst, 64 * l, l);
+    cdst += cstep;
+    sdst += sstep;
   }
 }
 
 size_t mma_smem_bytes(int K) {
-  return (size_t)MMA_SLOTS * MMA_SSTRIDE * 4 + (size_t)MMA_BARS * 8 + (size_t)(K / 2) * 4;
+  return 256 + (size_t)MMA_SLOTS * MMA_SSTRIDE * 4 + (size_t)MMA_BARS * 8 + (size_t)(K / 2) * 4;
 }
 
 // Programmatic dependent launch (the kernel's prologue may overlap the previous kernel in
@@ -991,48 +898,8 @@ bool tc_enabled() {
   return on;
 }
 
-// Double-buffered staging for the tensor-core kernel (ROT_B200_DB=0 selects the single-buffer one).
-bool db_enabled() {
-  static const bool on = [] {
-    const char* e = std::getenv("ROT_B200_DB");
-    return !(e && e[0] == '0');
-  }();
-  return on;
-}
-
-template <int BITS, int GT>
-rot_status launch_mma_db(const Args& a, cudaStream_t s) {
-  const size_t smem = db_smem_bytes(a.K);
-  auto kern = fwht_mma_db_kernel<BITS, GT>;
-  static int configured[64] = {0};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 64 && !configured[dev]) {
-    ROT_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024));
-    configured[dev] = 1;
-  }
-  const int64_t units = a.M * a.chunks;
-  int64_t grid = (units + DB_WARPS - 1) / DB_WARPS;
-  const int64_t cap = (int64_t)sm_count();
-  if (grid > cap) grid = cap;
-  if (grid < 1) return ROT_OK;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)grid);
-  cfg.blockDim = dim3(DB_THREADS);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = pdl_enabled() ? 1 : 0;
-  ROT_CUDA_TRY(cudaLaunchKernelEx(&cfg, kern, a));
-  return ROT_OK;
-}
-
 template <int BITS, int GT>
 rot_status launch_mma(const Args& a, cudaStream_t s) {
-  if (db_enabled() && db_smem_bytes(a.K) <= 227 * 1024) return launch_mma_db<BITS, GT>(a, s);
   const size_t smem = mma_smem_bytes(a.K);
   if (smem > 227 * 1024) return set_error(ROT_EUNSUPPORTED, "fused rotation: sign table too large for shared memory");
   auto kern = fwht_mma_kernel<BITS, GT>;
