@@ -263,6 +263,19 @@ __device__ __forceinline__ void umma_commit(uint64_t* bar) {
 }
 
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+#ifndef ROT_W4A4_TMEM_BIAS
+#define ROT_W4A4_TMEM_BIAS 0
+#endif
+// Store one 32-bit value into 32 consecutive columns of the warp's 32 TMEM lanes (four 8-column
+// stores: a vector operand takes distinct registers, and 8 copies of the constant cost no spill).
+__device__ __forceinline__ void tmem_st32_const(uint32_t taddr, uint32_t v) {
+#pragma unroll
+  for (int q = 0; q < 4; ++q)
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%1,%1,%1,%1,%1,%1,%1};" ::"r"(taddr + 8 * q), "r"(v)
+                 : "memory");
+}
 
 // Ordered shared-memory vector load: kept next to the TMEM load it serves, so the scale loads
 // of all column chunks are not hoisted ahead (which would need a register per loaded value).
@@ -359,7 +372,18 @@ __global__ void __launch_bounds__(THREADS, 1) w4a4_kernel(const __grid_constant_
     const int wg = warp >> 2;                 // column half of the tile
     const int row = qd * 32 + lane;           // TMEM lane = tile row
     const uint32_t lane_addr = tmem + ((uint32_t)(qd * 32) << 16) + wg * EPI_COLS;
-    // all accumulators start free (a group's first MMA overwrites its accumulator)
+#if ROT_W4A4_TMEM_BIAS
+    // every accumulator holds the bit pattern of 1.5 * 2^23 when a group starts: the group's MMAs
+    // accumulate onto it, so its int32 result is the bit pattern of the float 1.5 * 2^23 + UNIT*P
+    for (int b = 0; b < NACC; ++b) {
+      tmem_st32_const(lane_addr + b * BN, BIAS_BITS);
+      tmem_st32_const(lane_addr + b * BN + 32, BIAS_BITS);
+    }
+    tmem_wait_st();
+    tc_fence_before();
+    __syncwarp();
+#endif
+    // all accumulators start free
     if (lane == 0)
       for (int b = 0; b < NACC; ++b) mbar_arrive(&tempty[b]);
 
@@ -448,6 +472,19 @@ __global__ void __launch_bounds__(THREADS, 1) w4a4_kernel(const __grid_constant_
         tmem_ld32(lane_addr + b * BN, r0);
         tmem_ld32(lane_addr + b * BN + 32, r1);
         tmem_wait_ld();
+#if ROT_W4A4_TMEM_BIAS
+        // the partials are in registers: reset the accumulator to the bias and release it for
+        // the group NACC ahead before the arithmetic
+        tmem_st32_const(lane_addr + b * BN, BIAS_BITS);
+        tmem_st32_const(lane_addr + b * BN + 32, BIAS_BITS);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tempty[b]);
+        constexpr uint32_t ADD = 0u;                  // the TMEM value already carries the bias
+#else
+        constexpr uint32_t ADD = BIAS_BITS;
+#endif
         if constexpr (!PARTIALS) {
           const float2 sa2 = make_float2(sa, sa);
           const float2 d2 = make_float2(-BIAS_F * sa, -BIAS_F * sa);   // exact: 3 * 2^22 * binary16
@@ -460,9 +497,8 @@ __global__ void __launch_bounds__(THREADS, 1) w4a4_kernel(const __grid_constant_
               const int c = h * 32 + j;
               const float4 w4 = lds128(scw + c);
               // 256*P + bits(1.5 * 2^23) = bits of the float 1.5 * 2^23 + 256*P
-              const float2 u0 = make_float2(__uint_as_float(rr[j] + BIAS_BITS), __uint_as_float(rr[j + 1] + BIAS_BITS));
-              const float2 u1 =
-                  make_float2(__uint_as_float(rr[j + 2] + BIAS_BITS), __uint_as_float(rr[j + 3] + BIAS_BITS));
+              const float2 u0 = make_float2(__uint_as_float(rr[j] + ADD), __uint_as_float(rr[j + 1] + ADD));
+              const float2 u1 = make_float2(__uint_as_float(rr[j + 2] + ADD), __uint_as_float(rr[j + 3] + ADD));
               // 256*P*sA (the bias cancels inside one rounding), then acc += that * sW/256
               const float2 t0 = __ffma2_rn(u0, sa2, d2);
               const float2 t1 = __ffma2_rn(u1, sa2, d2);
@@ -477,14 +513,16 @@ __global__ void __launch_bounds__(THREADS, 1) w4a4_kernel(const __grid_constant_
             for (int j = 0; j < 64; ++j) {
               const int n = w.n0 + wg * EPI_COLS + j;
               const uint32_t v = j < 32 ? r0[j] : r1[j - 32];
-              if (n < p.N) p.P[((int64_t)m * p.N + n) * NG + g] = ((int32_t)v) / (int32_t)L::UNIT;
+              if (n < p.N) p.P[((int64_t)m * p.N + n) * NG + g] = ((int32_t)(v + ADD - BIAS_BITS)) / (int32_t)L::UNIT;
             }
           }
         }
+#if !ROT_W4A4_TMEM_BIAS
         // the partials are in registers: release the accumulator for the group NACC ahead
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&tempty[b]);
+#endif
       }
       if (PARTIALS || !ok) continue;
       if (row_ok) {
@@ -651,7 +689,8 @@ __global__ void __launch_bounds__(THREADS, 1) w4a4_kernel(const __grid_constant_
               }
               tc_fence_after();
             }
-            umma_i8(tmem + b * BN, dA0 + soA + 2 * k4, dB0 + soB + 2 * k4, kg != 0 ? 1u : 0u);
+            // accumulate onto the bias the epilogue stored (or overwrite at a group's first MMA)
+            umma_i8(tmem + b * BN, dA0 + soA + 2 * k4, dB0 + soB + 2 * k4, (ROT_W4A4_TMEM_BIAS || kg != 0) ? 1u : 0u);
             if (++kg == gsteps) {
               umma_commit(&tfull[b]);
               kg = 0;
