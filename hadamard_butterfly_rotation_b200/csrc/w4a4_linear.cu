@@ -265,18 +265,6 @@ __device__ __forceinline__ void umma_commit(uint64_t* bar) {
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
-#ifndef ROT_W4A4_TMEM_BIAS
-#define ROT_W4A4_TMEM_BIAS 0
-#endif
-// Store one 32-bit value into 32 consecutive columns of the warp's 32 TMEM lanes (four 8-column
-// stores: a vector operand takes distinct registers, and 8 copies of the constant cost no spill).
-__device__ __forceinline__ void tmem_st32_const(uint32_t taddr, uint32_t v) {
-#pragma unroll
-  for (int q = 0; q < 4; ++q)
-    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%1,%1,%1,%1,%1,%1,%1};" ::"r"(taddr + 8 * q), "r"(v)
-                 : "memory");
-}
-
 // Ordered shared-memory vector load: kept next to the TMEM load it serves, so the scale loads
 // of all column chunks are not hoisted ahead (which would need a register per loaded value).
 __device__ __forceinline__ float4 lds128(const float* p) {
@@ -372,18 +360,7 @@ __global__ void __launch_bounds__(THREADS, 1) w4a4_kernel(const __grid_constant_
     const int wg = warp >> 2;                 // column half of the tile
     const int row = qd * 32 + lane;           // TMEM lane = tile row
     const uint32_t lane_addr = tmem + ((uint32_t)(qd * 32) << 16) + wg * EPI_COLS;
-#if ROT_W4A4_TMEM_BIAS
-    // every accumulator holds the bit pattern of 1.5 * 2^23 when a group starts: the group's MMAs
-    // accumulate onto it, so its int32 result is the bit pattern of the float 1.5 * 2^23 + UNIT*P
-    for (int b = 0; b < NACC; ++b) {
-      tmem_st32_const(lane_addr + b * BN, BIAS_BITS);
-      tmem_st32_const(lane_addr + b * BN + 32, BIAS_BITS);
-    }
-    tmem_wait_st();
-    tc_fence_before();
-    __syncwarp();
-#endif
-    // all accumulators start free
+    // all accumulators start free (a group's first MMA overwrites its accumulator)
     if (lane == 0)
       for (int b = 0; b < NACC; ++b) mbar_arrive(&tempty[b]);
 
@@ -468,61 +445,59 @@ __global__ void __launch_bounds__(THREADS, 1) w4a4_kernel(const __grid_constant_
         ok = ok && bar_wait(&tfull[b], (gc / NACC) & 1, abort_flag, p.wait_ns);
         if (!ok) break;
         tc_fence_after();
-        uint32_t r0[32], r1[32];
-        tmem_ld32(lane_addr + b * BN, r0);
-        tmem_ld32(lane_addr + b * BN + 32, r1);
-        tmem_wait_ld();
-#if ROT_W4A4_TMEM_BIAS
-        // the partials are in registers: reset the accumulator to the bias and release it for
-        // the group NACC ahead before the arithmetic
-        tmem_st32_const(lane_addr + b * BN, BIAS_BITS);
-        tmem_st32_const(lane_addr + b * BN + 32, BIAS_BITS);
-        tmem_wait_st();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&tempty[b]);
-        constexpr uint32_t ADD = 0u;                  // the TMEM value already carries the bias
-#else
-        constexpr uint32_t ADD = BIAS_BITS;
-#endif
         if constexpr (!PARTIALS) {
+          // The group in two halves of 32 columns: each half's TMEM load is in flight while the
+          // 8 column-scale vectors of that half are loaded from shared memory, so the arithmetic
+          // waits once per half for both (instead of once per scale vector). The accumulator is
+          // released as soon as the second half is in registers.
           const float2 sa2 = make_float2(sa, sa);
           const float2 d2 = make_float2(-BIAS_F * sa, -BIAS_F * sa);   // exact: 3 * 2^22 * binary16
-          const float* scw = wsc;
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
-            const uint32_t* rr = h ? r1 : r0;
+            uint32_t r[32];
+            float4 w4[8];
+            tmem_ld32(lane_addr + b * BN + 32 * h, r);
 #pragma unroll
-            for (int j = 0; j < 32; j += 4) {
-              const int c = h * 32 + j;
-              const float4 w4 = lds128(scw + c);
+            for (int q = 0; q < 8; ++q) w4[q] = lds128(wsc + 32 * h + 4 * q);
+            tmem_wait_ld();
+            if (h == 1) {
+              // the whole group is in registers: release the accumulator for the group NACC ahead
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(&tempty[b]);
+            }
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+              const int c = 32 * h + 4 * q;
               // 256*P + bits(1.5 * 2^23) = bits of the float 1.5 * 2^23 + 256*P
-              const float2 u0 = make_float2(__uint_as_float(rr[j] + ADD), __uint_as_float(rr[j + 1] + ADD));
-              const float2 u1 = make_float2(__uint_as_float(rr[j + 2] + ADD), __uint_as_float(rr[j + 3] + ADD));
+              const float2 u0 = make_float2(__uint_as_float(r[4 * q] + BIAS_BITS), __uint_as_float(r[4 * q + 1] + BIAS_BITS));
+              const float2 u1 =
+                  make_float2(__uint_as_float(r[4 * q + 2] + BIAS_BITS), __uint_as_float(r[4 * q + 3] + BIAS_BITS));
               // 256*P*sA (the bias cancels inside one rounding), then acc += that * sW/256
               const float2 t0 = __ffma2_rn(u0, sa2, d2);
               const float2 t1 = __ffma2_rn(u1, sa2, d2);
-              acc[c / 2] = __ffma2_rn(t0, make_float2(w4.x, w4.y), acc[c / 2]);
-              acc[c / 2 + 1] = __ffma2_rn(t1, make_float2(w4.z, w4.w), acc[c / 2 + 1]);
+              acc[c / 2] = __ffma2_rn(t0, make_float2(w4[q].x, w4[q].y), acc[c / 2]);
+              acc[c / 2 + 1] = __ffma2_rn(t1, make_float2(w4[q].z, w4[q].w), acc[c / 2 + 1]);
             }
           }
         } else {
+          uint32_t r0[32], r1[32];
+          tmem_ld32(lane_addr + b * BN, r0);
+          tmem_ld32(lane_addr + b * BN + 32, r1);
+          tmem_wait_ld();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&tempty[b]);
           if (row_ok) {
             const int g = w.g0 + gl;
 #pragma unroll
             for (int j = 0; j < 64; ++j) {
               const int n = w.n0 + wg * EPI_COLS + j;
               const uint32_t v = j < 32 ? r0[j] : r1[j - 32];
-              if (n < p.N) p.P[((int64_t)m * p.N + n) * NG + g] = ((int32_t)(v + ADD - BIAS_BITS)) / (int32_t)L::UNIT;
+              if (n < p.N) p.P[((int64_t)m * p.N + n) * NG + g] = ((int32_t)v) / (int32_t)L::UNIT;
             }
           }
         }
-#if !ROT_W4A4_TMEM_BIAS
-        // the partials are in registers: release the accumulator for the group NACC ahead
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&tempty[b]);
-#endif
       }
       if (PARTIALS || !ok) continue;
       if (row_ok) {
@@ -689,8 +664,7 @@ __global__ void __launch_bounds__(THREADS, 1) w4a4_kernel(const __grid_constant_
               }
               tc_fence_after();
             }
-            // accumulate onto the bias the epilogue stored (or overwrite at a group's first MMA)
-            umma_i8(tmem + b * BN, dA0 + soA + 2 * k4, dB0 + soB + 2 * k4, (ROT_W4A4_TMEM_BIAS || kg != 0) ? 1u : 0u);
+            umma_i8(tmem + b * BN, dA0 + soA + 2 * k4, dB0 + soB + 2 * k4, kg != 0 ? 1u : 0u);
             if (++kg == gsteps) {
               umma_commit(&tfull[b]);
               kg = 0;
