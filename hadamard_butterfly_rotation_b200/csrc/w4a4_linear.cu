@@ -744,6 +744,7 @@ struct DecParams {
   int M, N, K, G;
   int c_bf16;
   int groups_per_split;
+  unsigned long long wait_ns;   // staged kernel: bound of the weight-slice wait
 };
 
 // A8 (W4A8): the activation codes are int8 [M, K] in natural order; per span each lane loads the
@@ -862,6 +863,220 @@ __global__ void __launch_bounds__(DEC_THREADS) w4a4_decode_kernel(const DecParam
   }
 }
 
+// Staged decode kernel. A CTA owns NPC n-tiles (8 weight rows each, contiguous in Wq) and splits K
+// into KS slices of whole groups: warp (t, k) computes n-tile t over slice k. Each warp streams its
+// own 8 x slice bytes of weights into shared memory at the start with bulk asynchronous copies (one
+// per row) completing on its own mbarrier, so every SM has its whole share of the weight stream in
+// flight at once; the activation codes (L1/L2-resident) are loaded one span ahead. The K-slices
+// are summed through shared memory and the CTA writes its tile of C directly (no atomics, no
+// second launch). Rows are staged K/2 + 64 bytes apart: the 16-byte reads of a quarter-warp
+// (rows g, g + 1 and pieces 0..3) fall in 8 distinct bank groups.
+__device__ int g_dec_error = 0;
+
+struct StagedDec {
+  int npc, ks;       // n-tiles per CTA, K-slices
+  int pitch;         // bytes between staged weight rows
+};
+
+constexpr int staged_threads(int mt) { return mt >= 3 ? 256 : 512; }   // bound on the CTA (registers)
+
+template <int MT, bool A8>
+__global__ void __launch_bounds__(staged_threads(MT)) w4a4_decode_staged_kernel(const DecParams p, const StagedDec q) {
+  constexpr float UNIT = A8 ? 16.0f : 256.0f;
+  extern __shared__ __align__(128) uint8_t dsm[];
+  asm volatile("griddepcontrol.wait;" ::: "memory");   // see w4a4_kernel (programmatic launch)
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  const int warp = threadIdx.x >> 5, l = threadIdx.x & 31;
+  const int g = l >> 2, c = l & 3;
+  const int tl = warp % q.npc, ks = warp / q.npc;
+  const int n0 = (blockIdx.x * q.npc + tl) * 8;
+  const bool active = n0 < p.N;
+  const int NG = p.K / p.G;
+  const int g0 = (int)((int64_t)NG * ks / q.ks);
+  int g1 = (int)((int64_t)NG * (ks + 1) / q.ks);
+  const int gbytes = p.G / 2;                              // packed bytes of one group of a row
+  uint64_t* bar = reinterpret_cast<uint64_t*>(dsm) + warp;
+  const int nwarps = q.npc * q.ks;
+  uint8_t* wsm = dsm + ((nwarps * 8 + 127) & ~127) + (size_t)tl * 8 * q.pitch;
+  float* red = reinterpret_cast<float*>(dsm + ((nwarps * 8 + 127) & ~127) + (size_t)q.npc * 8 * q.pitch);
+  const int64_t ldp = p.K / 2;
+  float acc[MT][4];
+#pragma unroll
+  for (int t = 0; t < MT; ++t)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) acc[t][i] = 0.0f;
+
+  if (active && g1 > g0) {
+    const uint32_t slice_bytes = (uint32_t)((g1 - g0) * gbytes);
+    if (l == 0) {
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(bar)) : "memory");
+      asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+      mbar_arrive_expect_tx(bar, 8u * slice_bytes);
+    }
+    __syncwarp();
+    if (l < 8)
+      asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                       smem_u32(wsm + (size_t)l * q.pitch + (size_t)g0 * gbytes)),
+                   "l"(p.Wq + (int64_t)(n0 + l) * ldp + (int64_t)g0 * gbytes), "r"(slice_bytes), "r"(smem_u32(bar))
+                   : "memory");
+    // activation codes of the first span, loaded while the weights are in flight
+    const int spans_per_group = p.G / 128;
+    const int abytes = A8 ? 32 : 16;                     // this lane's activation bytes per span and row
+    const int64_t lda = A8 ? p.K : ldp;
+    auto a_load = [&](int span, uint4 (&lo)[MT][2], uint4 (&hi)[MT][2]) {
+#pragma unroll
+      for (int t = 0; t < MT; ++t) {
+        const int m_lo = t * 16 + g, m_hi = m_lo + 8;
+        const int64_t off = (int64_t)span * (A8 ? 128 : 64) + abytes * c;
+        lo[t][0] = lo[t][1] = hi[t][0] = hi[t][1] = make_uint4(0u, 0u, 0u, 0u);
+        if (m_lo < p.M) {
+          const uint4* src = reinterpret_cast<const uint4*>(p.Aq + (int64_t)m_lo * lda + off);
+          lo[t][0] = __ldg(src);
+          if (A8) lo[t][1] = __ldg(src + 1);
+        }
+        if (m_hi < p.M) {
+          const uint4* src = reinterpret_cast<const uint4*>(p.Aq + (int64_t)m_hi * lda + off);
+          hi[t][0] = __ldg(src);
+          if (A8) hi[t][1] = __ldg(src + 1);
+        }
+      }
+    };
+    uint4 alo[MT][2], ahi[MT][2];
+    int span = g0 * spans_per_group;
+    a_load(span, alo, ahi);
+    // group scales, loaded one group ahead: sW of rows n0 + 2c (+1), sA of rows m_lo / m_hi
+    auto s_load = [&](int gg, uint16_t (&w)[2], uint16_t (&a)[MT][2]) {
+      w[0] = p.Ws[(int64_t)(n0 + 2 * c) * NG + gg];
+      w[1] = p.Ws[(int64_t)(n0 + 2 * c + 1) * NG + gg];
+#pragma unroll
+      for (int t = 0; t < MT; ++t) {
+        const int m_lo = t * 16 + g, m_hi = m_lo + 8;
+        a[t][0] = m_lo < p.M ? p.As[(int64_t)m_lo * NG + gg] : (uint16_t)0;
+        a[t][1] = m_hi < p.M ? p.As[(int64_t)m_hi * NG + gg] : (uint16_t)0;
+      }
+    };
+    uint16_t swn[2], san[MT][2];
+    s_load(g0, swn, san);
+    // bounded wait for the warp's weight slice
+    {
+      const uint32_t addr = smem_u32(bar);
+      unsigned long long t0 = 0;
+      bool ok = true;
+      for (uint32_t it = 0;; ++it) {
+        uint32_t done;
+        asm volatile("{\n\t.reg .pred q;\n\tmbarrier.try_wait.parity.shared::cta.b64 q, [%1], 0;\n\t"
+                     "selp.u32 %0, 1, 0, q;\n\t}"
+                     : "=r"(done)
+                     : "r"(addr)
+                     : "memory");
+        if (done) break;
+        if ((it & 63) == 63) {
+          unsigned long long now;
+          asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(now));
+          if (t0 == 0) t0 = now;
+          else if (now - t0 > p.wait_ns) {
+            atomicExch(&g_dec_error, (int)ROT_ETIMEOUT);
+            ok = false;
+            break;
+          }
+        }
+      }
+      if (!__all_sync(0xffffffffu, ok)) g1 = g0;   // gave up: compute nothing (outputs unspecified)
+    }
+    const uint8_t* wlane = wsm + (size_t)g * q.pitch + 16 * c;
+    for (int gg = g0; gg < g1; ++gg) {
+      // this group's scales (loaded a group ahead); the next group's loads overlap the MMAs
+      uint16_t swc[2] = {swn[0], swn[1]}, sac[MT][2];
+#pragma unroll
+      for (int t = 0; t < MT; ++t) { sac[t][0] = san[t][0]; sac[t][1] = san[t][1]; }
+      if (gg + 1 < g1) s_load(gg + 1, swn, san);
+      int d[MT][4];
+#pragma unroll
+      for (int t = 0; t < MT; ++t)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) d[t][i] = 0;
+      for (int sp = 0; sp < spans_per_group; ++sp, ++span) {
+        const uint4 wv = *reinterpret_cast<const uint4*>(wlane + (size_t)span * 64);
+        uint4 clo[MT][2], chi[MT][2];
+#pragma unroll
+        for (int t = 0; t < MT; ++t) {
+          clo[t][0] = alo[t][0]; clo[t][1] = alo[t][1]; chi[t][0] = ahi[t][0]; chi[t][1] = ahi[t][1];
+        }
+        if (span + 1 < g1 * spans_per_group) a_load(span + 1, alo, ahi);   // next span's activations
+        const uint32_t ww[4] = {wv.x, wv.y, wv.z, wv.w};
+#pragma unroll
+        for (int t = 0; t < MT; ++t) {
+          if constexpr (A8) {
+            const uint32_t al[8] = {clo[t][0].x, clo[t][0].y, clo[t][0].z, clo[t][0].w,
+                                    clo[t][1].x, clo[t][1].y, clo[t][1].z, clo[t][1].w};
+            const uint32_t ah[8] = {chi[t][0].x, chi[t][0].y, chi[t][0].z, chi[t][0].w,
+                                    chi[t][1].x, chi[t][1].y, chi[t][1].z, chi[t][1].w};
+#pragma unroll
+            for (int s4 = 0; s4 < 4; ++s4) {
+              const uint32_t a[4] = {prmt(al[2 * s4], al[2 * s4 + 1], 0x6420u), prmt(ah[2 * s4], ah[2 * s4 + 1], 0x6420u),
+                                     prmt(al[2 * s4], al[2 * s4 + 1], 0x7531u), prmt(ah[2 * s4], ah[2 * s4 + 1], 0x7531u)};
+              mma_s8_16832(d[t], a, (ww[s4] << 4) & 0xF0F0F0F0u, ww[s4] & 0xF0F0F0F0u);
+            }
+          } else {
+            const uint32_t al[4] = {clo[t][0].x, clo[t][0].y, clo[t][0].z, clo[t][0].w};
+            const uint32_t ah[4] = {chi[t][0].x, chi[t][0].y, chi[t][0].z, chi[t][0].w};
+#pragma unroll
+            for (int s4 = 0; s4 < 4; ++s4) {
+              const uint32_t a[4] = {(al[s4] << 4) & 0xF0F0F0F0u, (ah[s4] << 4) & 0xF0F0F0F0u, al[s4] & 0xF0F0F0F0u,
+                                     ah[s4] & 0xF0F0F0F0u};
+              mma_s8_16832(d[t], a, (ww[s4] << 4) & 0xF0F0F0F0u, ww[s4] & 0xF0F0F0F0u);
+            }
+          }
+        }
+      }
+      const float sw0 = __half2float(__ushort_as_half(swc[0])) * (1.0f / UNIT);
+      const float sw1 = __half2float(__ushort_as_half(swc[1])) * (1.0f / UNIT);
+#pragma unroll
+      for (int t = 0; t < MT; ++t) {
+        const float sa0 = __half2float(__ushort_as_half(sac[t][0]));
+        const float sa1 = __half2float(__ushort_as_half(sac[t][1]));
+        acc[t][0] = fmaf((float)d[t][0] * sw0, sa0, acc[t][0]);
+        acc[t][1] = fmaf((float)d[t][1] * sw1, sa0, acc[t][1]);
+        acc[t][2] = fmaf((float)d[t][2] * sw0, sa1, acc[t][2]);
+        acc[t][3] = fmaf((float)d[t][3] * sw1, sa1, acc[t][3]);
+      }
+    }
+  }
+  // sum the K-slices: slices 1.. park their partial sums in shared memory, slice 0 adds and stores
+  if (ks > 0) {
+    float* r = red + ((size_t)((ks - 1) * q.npc + tl) * 32 + l) * (4 * MT);
+#pragma unroll
+    for (int t = 0; t < MT; ++t)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) r[4 * t + i] = acc[t][i];
+  }
+  __syncthreads();
+  if (ks > 0 || !active) return;
+  for (int k = 1; k < q.ks; ++k) {
+    const float* r = red + ((size_t)((k - 1) * q.npc + tl) * 32 + l) * (4 * MT);
+#pragma unroll
+    for (int t = 0; t < MT; ++t)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) acc[t][i] += r[4 * t + i];
+  }
+#pragma unroll
+  for (int t = 0; t < MT; ++t) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int m = t * 16 + g + 8 * h;
+      if (m >= p.M) continue;
+      const int n = n0 + 2 * c;
+      const float v0 = acc[t][2 * h], v1 = acc[t][2 * h + 1];
+      if (p.c_bf16) {
+        *reinterpret_cast<__nv_bfloat162*>(static_cast<__nv_bfloat16*>(p.C) + (int64_t)m * p.N + n) =
+            __floats2bfloat162_rn(v0, v1);
+      } else {
+        *reinterpret_cast<float2*>(static_cast<float*>(p.C) + (int64_t)m * p.N + n) = make_float2(v0, v1);
+      }
+    }
+  }
+}
+
 // Split-K factor: only when the output tiles leave most SMs idle (decode-sized M); each
 // split then covers a whole number of groups.
 int split_count(int64_t tiles, int group_units, int sms) {
@@ -959,14 +1174,9 @@ rot_status w4a4_launch(const uint8_t* Aq, const uint16_t* As, const uint8_t* Wq,
     return ROT_OK;
   };
   if (!partials && M <= 16 * DEC_MAXMT && G % 128 == 0) {
-    // decode-sized M: weight-streaming kernel, K split until about 32 warps per SM are busy
-    // (more bytes in flight: 16 warps measured 9.7 us, 32 warps 8.8 us for q_proj at M = 16)
     const int64_t ntiles = N / 8;
     const int NG = (int)(K / G);
-    int64_t want = ((int64_t)sm_count() * 32 + ntiles - 1) / ntiles;
-    const int splits0 = (int)std::max<int64_t>(1, std::min<int64_t>(NG, want));
-    const int gps = (NG + splits0 - 1) / splits0;
-    const int splits = (NG + gps - 1) / gps;
+    const int mt = (int)((M + 15) / 16);
     DecParams d{};
     d.Aq = Aq;
     d.As = As;
@@ -979,13 +1189,67 @@ rot_status w4a4_launch(const uint8_t* Aq, const uint16_t* As, const uint8_t* Wq,
     d.K = (int)K;
     d.G = G;
     d.c_bf16 = c_dtype == ROT_BF16;
+    d.wait_ns = wait_limit_ns(WAIT_NS);
+    // staged weight stream (shared memory, rows K/2 + 64 bytes apart): enough n-tiles per CTA that
+    // every CTA is resident at once (two per SM), K-slices to bring the CTA to about 16 warps
+    const int64_t pitch = K / 2 + 64;
+    const int64_t sms = sm_count();
+    const int max_warps = (mt >= 3 ? 256 : 512) / 32;
+    int npc = (int)std::max<int64_t>(1, (ntiles + 2 * sms - 1) / (2 * sms));
+    int ksl = std::max(1, std::min(NG, max_warps / std::max(1, npc)));
+    auto smem_of = [&](int np, int kk) -> size_t {
+      return (size_t)((np * kk * 8 + 127) & ~127) + (size_t)np * 8 * pitch + (size_t)(kk - 1) * np * 32 * 4 * mt * 4;
+    };
+    while (npc > 1 && smem_of(npc, ksl) > 110 * 1024) {   // keep two CTAs per SM
+      npc = (npc + 1) / 2;
+      ksl = std::max(1, std::min(NG, max_warps / npc));
+    }
+    if (npc * ksl <= max_warps && smem_of(npc, ksl) <= 200 * 1024) {
+      StagedDec q;
+      q.npc = npc;
+      q.ks = ksl;
+      q.pitch = (int)pitch;
+      d.groups_per_split = NG;
+      const size_t smem = smem_of(npc, ksl);
+      void (*dk)(const DecParams, const StagedDec) = nullptr;
+      if (a8) dk = mt == 1 ? w4a4_decode_staged_kernel<1, true> : mt == 2 ? w4a4_decode_staged_kernel<2, true>
+                   : mt == 3 ? w4a4_decode_staged_kernel<3, true> : w4a4_decode_staged_kernel<4, true>;
+      else dk = mt == 1 ? w4a4_decode_staged_kernel<1, false> : mt == 2 ? w4a4_decode_staged_kernel<2, false>
+                : mt == 3 ? w4a4_decode_staged_kernel<3, false> : w4a4_decode_staged_kernel<4, false>;
+      static int dec_configured[64][8] = {};   // per device and (A8, MT) variant: the opt-in limit set once
+      int dev = 0;
+      ROT_CUDA_TRY(cudaGetDevice(&dev));
+      const int var = (a8 ? 4 : 0) + (mt - 1);
+      if (dev >= 64 || !dec_configured[dev][var]) {
+        ROT_CUDA_TRY(cudaFuncSetAttribute(dk, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024));
+        if (dev < 64) dec_configured[dev][var] = 1;
+      }
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3((unsigned)((ntiles + npc - 1) / npc));
+      cfg.blockDim = dim3(32 * npc * ksl);
+      cfg.dynamicSmemBytes = smem;
+      cfg.stream = s;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+      attr[0].val.programmaticStreamSerializationAllowed = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = pdl ? 1 : 0;
+      ROT_CUDA_TRY(cudaLaunchKernelEx(&cfg, dk, d, q));
+      ROT_CUDA_TRY(cudaGetLastError());
+      return ROT_OK;
+    }
+    // very long rows: the weights stream through registers, K split until about 32 warps per SM
+    // are busy (more bytes in flight)
+    int64_t want = ((int64_t)sm_count() * 32 + ntiles - 1) / ntiles;
+    const int splits0 = (int)std::max<int64_t>(1, std::min<int64_t>(NG, want));
+    const int gps = (NG + splits0 - 1) / splits0;
+    const int splits = (NG + gps - 1) / gps;
     d.groups_per_split = gps;
     if (splits > 1) {
       rot_status st = acc_target(&d.Cacc);
       if (st) return st;
     }
     const dim3 grid((unsigned)((ntiles + DEC_THREADS / 32 - 1) / (DEC_THREADS / 32)), (unsigned)splits);
-    const int mt = (int)((M + 15) / 16);
     void (*dk)(const DecParams) = nullptr;
     if (a8) dk = mt == 1 ? w4a4_decode_kernel<1, true> : mt == 2 ? w4a4_decode_kernel<2, true>
                  : mt == 3 ? w4a4_decode_kernel<3, true> : w4a4_decode_kernel<4, true>;
@@ -1105,7 +1369,13 @@ rot_status w4a4_noalloc_scratch(float** out) {
 }
 
 rot_status w4a4_fetch_device_error() {
-  int v = 0;
+  int v = 0, vd = 0;
+  ROT_CUDA_TRY(cudaMemcpyFromSymbol(&vd, g_dec_error, sizeof(int)));
+  if (vd) {
+    int z = 0;
+    ROT_CUDA_TRY(cudaMemcpyToSymbol(g_dec_error, &z, sizeof(int)));
+    return set_error((rot_status)vd, "a bounded wait in the decode-sized w4a4 kernel gave up");
+  }
   ROT_CUDA_TRY(cudaMemcpyFromSymbol(&v, g_w4a4_error, sizeof(int)));
   if (v) {
     int z = 0;

@@ -43,10 +43,15 @@ def _dev_operands(qa, sa, qw, sw):
     return dev(Q.pack(qa, 4)), dev(sa), dev(Q.pack(qw, 4)), dev(sw)
 
 
-@pytest.mark.parametrize("M,N,K,G", [(16, 4096, 4096, 128), (16, 1024, 2048, 256), (5, 640, 1024, 64)])
+@pytest.mark.parametrize("M,N,K,G", [(128, 1024, 4096, 128), (96, 2048, 2048, 256), (5, 640, 1024, 64),
+                                     (16, 4096, 4096, 128)])
 @pytest.mark.parametrize("out", ["bf16", "f32"])
 def test_noalloc_matches_allocating_entry(lib, M, N, K, G, out):
     import torch
+    if M > 64 or G % 128:
+        # these shapes take the tile kernel's split-K path, where the bf16 output needs the buffer
+        sms = torch.cuda.get_device_properties(0).multi_processor_count
+        assert lib.w4a4_tile_plan(M, N, K, G, sms)["splits"] > 1
     qa, sa, qw, sw = _operands(M + N + K, M, N, K, G)
     Aq, As, Wq, Ws = _dev_operands(qa, sa, qw, sw)
     dt = torch.bfloat16 if out == "bf16" else torch.float32
@@ -93,7 +98,9 @@ def test_noalloc_leaves_the_memory_pool_untouched(lib):
     import torch
     if torch.cuda.get_allocator_backend() != "native":
         pytest.skip("torch itself allocates from the stream-ordered pool under this configuration")
-    M, N, K, G = 16, 4096, 4096, 128
+    M, N, K, G = 128, 1024, 4096, 128
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    assert lib.w4a4_tile_plan(M, N, K, G, sms)["splits"] > 1
     qa, sa, qw, sw = _operands(11, M, N, K, G)
     Aq, As, Wq, Ws = _dev_operands(qa, sa, qw, sw)
     out = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
