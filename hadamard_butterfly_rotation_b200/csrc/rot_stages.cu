@@ -181,6 +181,7 @@ constexpr int MR_UG = 24;          // gather indices per thread per batch (K <= 
 struct MrStage {
   const float* blocks;   // radix 2: [n_blocks][4]; radix b: [b][b] (shared)
   const int32_t* perm;   // gather after the stage or nullptr
+  const int32_t* iperm;  // its inverse: a non-identity stage scatters output j to iperm[j]
   int b, stride;
   uint32_t magic;        // ceil(2^32 / stride) for stride >= 2 (stride 1 divides trivially)
   int per_block, identity;
@@ -247,19 +248,26 @@ __global__ void __launch_bounds__(MR_THREADS, 1) stages_rows_kernel(const MrArgs
       const MrStage& S = a.st[t];
       if (!S.identity) {
         const int st = S.stride;
+        // a stage followed by a permutation writes its outputs straight to their permuted places
+        // in the other buffer (x''[P^-1[j]] = x'[j]): no separate gather pass
+        const bool scat = S.perm != nullptr;
+        float* dst = scat ? nxt : cur;
         if (S.b == 2) {
-          // MR_UB blocks per thread per batch: their parameter loads (L2) are all in flight
-          // before the first is used
+          // MR_UB blocks per thread per batch: their parameter (and scatter index) loads from L2
+          // are all in flight before the first is used
           for (int c0 = threadIdx.x; c0 < K / 2; c0 += MR_THREADS * MR_UB) {
             float4 B[MR_UB];
-            int base[MR_UB];
+            int base[MR_UB], o0[MR_UB], o1[MR_UB];
 #pragma unroll
             for (int u = 0; u < MR_UB; ++u) {
               const int c = c0 + u * MR_THREADS;
+              const bool on = c < K / 2;
               const int high = st == 1 ? c : (int)__umulhi((uint32_t)c, S.magic);
               base[u] = (c - high * st) + high * 2 * st;
-              B[u] = c < K / 2 ? __ldg(reinterpret_cast<const float4*>(S.blocks + (S.per_block ? 4 * c : 0)))
-                               : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+              B[u] = on ? __ldg(reinterpret_cast<const float4*>(S.blocks + (S.per_block ? 4 * c : 0)))
+                        : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+              o0[u] = scat && on ? __ldg(S.iperm + base[u]) : base[u];
+              o1[u] = scat && on ? __ldg(S.iperm + base[u] + st) : base[u] + st;
             }
 #pragma unroll
             for (int u = 0; u < MR_UB; ++u) {
@@ -267,8 +275,8 @@ __global__ void __launch_bounds__(MR_THREADS, 1) stages_rows_kernel(const MrArgs
 #pragma unroll
                 for (int r = 0; r < MR_ROWS; ++r) {
                   const float x0 = cur[r * K + base[u]], x1 = cur[r * K + base[u] + st];
-                  cur[r * K + base[u]] = fmaf(B[u].x, x0, B[u].y * x1);
-                  cur[r * K + base[u] + st] = fmaf(B[u].z, x0, B[u].w * x1);
+                  dst[r * K + o0[u]] = fmaf(B[u].x, x0, B[u].y * x1);
+                  dst[r * K + o1[u]] = fmaf(B[u].z, x0, B[u].w * x1);
                 }
               }
             }
@@ -310,7 +318,8 @@ __global__ void __launch_bounds__(MR_THREADS, 1) stages_rows_kernel(const MrArgs
                       a3 = fmaf(w.w, in[4 * k4 + 3], a3);
                     }
                   }
-                  x[base + o * st] = (a0 + a1) + (a2 + a3);
+                  const int oi = base + o * st;
+                  dst[r * K + (scat ? __ldg(S.iperm + oi) : oi)] = (a0 + a1) + (a2 + a3);
                 }
               }
               __syncthreads();
@@ -318,8 +327,11 @@ __global__ void __launch_bounds__(MR_THREADS, 1) stages_rows_kernel(const MrArgs
           }
         }
         __syncthreads();
+        if (scat) {
+          float* tmp = cur; cur = nxt; nxt = tmp;
+        }
       }
-      if (S.perm) {
+      if (S.perm && S.identity) {   // a permutation after an identity stage: plain gather
         for (int i0 = threadIdx.x; i0 < K; i0 += MR_THREADS * MR_UG) {
           int src[MR_UG];
 #pragma unroll
@@ -420,6 +432,7 @@ rot_status launch_rows(const rot_plan_s* p, const Args& a0, size_t smem, cudaStr
     MrStage& d = a.st[t];
     d.blocks = S.d_blocks;
     d.perm = S.d_perm;
+    d.iperm = S.d_iperm;
     d.b = S.b;
     d.stride = S.stride;
     d.magic = S.stride > 1 ? (uint32_t)(((1ull << 32) + (uint64_t)S.stride - 1) / (uint64_t)S.stride) : 0u;

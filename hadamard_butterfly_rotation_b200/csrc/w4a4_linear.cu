@@ -944,19 +944,7 @@ __global__ void __launch_bounds__(staged_threads(MT)) w4a4_decode_staged_kernel(
     uint4 alo[MT][2], ahi[MT][2];
     int span = g0 * spans_per_group;
     a_load(span, alo, ahi);
-    // group scales, loaded one group ahead: sW of rows n0 + 2c (+1), sA of rows m_lo / m_hi
-    auto s_load = [&](int gg, uint16_t (&w)[2], uint16_t (&a)[MT][2]) {
-      w[0] = p.Ws[(int64_t)(n0 + 2 * c) * NG + gg];
-      w[1] = p.Ws[(int64_t)(n0 + 2 * c + 1) * NG + gg];
-#pragma unroll
-      for (int t = 0; t < MT; ++t) {
-        const int m_lo = t * 16 + g, m_hi = m_lo + 8;
-        a[t][0] = m_lo < p.M ? p.As[(int64_t)m_lo * NG + gg] : (uint16_t)0;
-        a[t][1] = m_hi < p.M ? p.As[(int64_t)m_hi * NG + gg] : (uint16_t)0;
-      }
-    };
-    uint16_t swn[2], san[MT][2];
-    s_load(g0, swn, san);
+
     // bounded wait for the warp's weight slice
     {
       const uint32_t addr = smem_u32(bar);
@@ -985,11 +973,6 @@ __global__ void __launch_bounds__(staged_threads(MT)) w4a4_decode_staged_kernel(
     }
     const uint8_t* wlane = wsm + (size_t)g * q.pitch + 16 * c;
     for (int gg = g0; gg < g1; ++gg) {
-      // this group's scales (loaded a group ahead); the next group's loads overlap the MMAs
-      uint16_t swc[2] = {swn[0], swn[1]}, sac[MT][2];
-#pragma unroll
-      for (int t = 0; t < MT; ++t) { sac[t][0] = san[t][0]; sac[t][1] = san[t][1]; }
-      if (gg + 1 < g1) s_load(gg + 1, swn, san);
       int d[MT][4];
 #pragma unroll
       for (int t = 0; t < MT; ++t)
@@ -1029,12 +1012,13 @@ __global__ void __launch_bounds__(staged_threads(MT)) w4a4_decode_staged_kernel(
           }
         }
       }
-      const float sw0 = __half2float(__ushort_as_half(swc[0])) * (1.0f / UNIT);
-      const float sw1 = __half2float(__ushort_as_half(swc[1])) * (1.0f / UNIT);
+      const float sw0 = __half2float(__ushort_as_half(p.Ws[(int64_t)(n0 + 2 * c) * NG + gg])) * (1.0f / UNIT);
+      const float sw1 = __half2float(__ushort_as_half(p.Ws[(int64_t)(n0 + 2 * c + 1) * NG + gg])) * (1.0f / UNIT);
 #pragma unroll
       for (int t = 0; t < MT; ++t) {
-        const float sa0 = __half2float(__ushort_as_half(sac[t][0]));
-        const float sa1 = __half2float(__ushort_as_half(sac[t][1]));
+        const int m_lo = t * 16 + g, m_hi = m_lo + 8;
+        const float sa0 = m_lo < p.M ? __half2float(__ushort_as_half(p.As[(int64_t)m_lo * NG + gg])) : 0.0f;
+        const float sa1 = m_hi < p.M ? __half2float(__ushort_as_half(p.As[(int64_t)m_hi * NG + gg])) : 0.0f;
         acc[t][0] = fmaf((float)d[t][0] * sw0, sa0, acc[t][0]);
         acc[t][1] = fmaf((float)d[t][1] * sw1, sa0, acc[t][1]);
         acc[t][2] = fmaf((float)d[t][2] * sw0, sa1, acc[t][2]);
