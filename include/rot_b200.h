@@ -125,14 +125,15 @@ rot_status rot_dequant(const uint8_t* codes, const uint16_t* scales, int64_t M, 
  * Wq: uint8 [N, K/2], Ws: binary16 [N, K/G] (rows of W^T through the same plan, int4);
  * C:  [M, N] fp32 (c_dtype = ROT_F32) or bf16 (ROT_BF16), row-major, ldc = N.
  * Requires K % G == 0, G % 32 == 0, K % 64 == 0, N % 16 == 0; M >= 0 arbitrary.
- * Decode-sized M (M <= 64 with G % 128 == 0) runs a weight-streaming kernel (mma.sync
- * int8 per 8 weight rows); other shapes run a persistent tcgen05 kernel over 128 x 128
+ * Decode-sized M (M <= 64 with G % 128 == 0) runs a weight-streaming kernel (mma.sync int8 per 8
+ * weight rows; each CTA streams its rows' K-slices into shared memory with bulk copies and sums the
+ * slices itself, so C is written directly). Other shapes run a persistent tcgen05 kernel over 128 x 128
  * output tiles, and shapes whose tiles leave most SMs idle split K into ranges aligned to
- * lcm(G, 128). When K is split, the partial results are added
- * with fp32 atomics: C is zeroed on the stream first (fp32 output), or, for bf16 output, a
- * stream-ordered temporary of M * N floats is allocated (cudaMallocAsync), accumulated,
- * converted into C and freed on the stream. The summation order then varies between runs
- * (fp32 rounding). */
+ * lcm(G, 128); their partial results are added with fp32 atomics: C is zeroed on the stream first
+ * (fp32 output), or, for bf16 output, a stream-ordered temporary of M * N floats is allocated
+ * (cudaMallocAsync), accumulated, converted into C and freed on the stream. The summation order then
+ * varies between runs (fp32 rounding). The kernels wait for the previous kernel in the stream
+ * (griddepcontrol.wait) before touching global memory. */
 rot_status w4a4_linear(const uint8_t* Aq, const uint16_t* As, const uint8_t* Wq,
                        const uint16_t* Ws, int64_t M, int64_t N, int64_t K, int G, void* C,
                        int c_dtype, void* stream);
