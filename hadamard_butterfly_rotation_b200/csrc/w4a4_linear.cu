@@ -864,10 +864,11 @@ __global__ void __launch_bounds__(DEC_THREADS) w4a4_decode_kernel(const DecParam
 }
 
 // Staged decode kernel. A CTA owns NPC n-tiles (8 weight rows each, contiguous in Wq) and splits K
-// into KS slices of whole groups: warp (t, k) computes n-tile t over slice k. Each warp streams its
-// own 8 x slice bytes of weights into shared memory at the start with bulk asynchronous copies (one
-// per row) completing on its own mbarrier, so every SM has its whole share of the weight stream in
-// flight at once; the activation codes (L1/L2-resident) are loaded one span ahead. The K-slices
+// into KS slices of whole groups: warp (t, k) computes n-tile t over slice k. The first warp of each
+// n-tile streams its 8 whole rows into shared memory at the start with one bulk asynchronous copy per
+// row, completing on the n-tile's mbarrier that all its slice warps wait on, so every SM has its whole
+// share of the weight stream in flight at once; the activation codes (L1/L2-resident) are loaded one
+// span ahead. The K-slices
 // are summed through shared memory and the CTA writes its tile of C directly (no atomics, no
 // second launch). Rows are staged K/2 + 64 bytes apart: the 16-byte reads of a quarter-warp
 // (rows g, g + 1 and pieces 0..3) fall in 8 distinct bank groups.
@@ -895,7 +896,7 @@ __global__ void __launch_bounds__(staged_threads(MT)) w4a4_decode_staged_kernel(
   const int g0 = (int)((int64_t)NG * ks / q.ks);
   int g1 = (int)((int64_t)NG * (ks + 1) / q.ks);
   const int gbytes = p.G / 2;                              // packed bytes of one group of a row
-  uint64_t* bar = reinterpret_cast<uint64_t*>(dsm) + warp;
+  uint64_t* bar = reinterpret_cast<uint64_t*>(dsm) + tl;   // one per n-tile
   const int nwarps = q.npc * q.ks;
   uint8_t* wsm = dsm + ((nwarps * 8 + 127) & ~127) + (size_t)tl * 8 * q.pitch;
   float* red = reinterpret_cast<float*>(dsm + ((nwarps * 8 + 127) & ~127) + (size_t)q.npc * 8 * q.pitch);
@@ -906,19 +907,22 @@ __global__ void __launch_bounds__(staged_threads(MT)) w4a4_decode_staged_kernel(
 #pragma unroll
     for (int i = 0; i < 4; ++i) acc[t][i] = 0.0f;
 
-  if (active && g1 > g0) {
-    const uint32_t slice_bytes = (uint32_t)((g1 - g0) * gbytes);
+  if (ks == 0 && active) {
+    // the n-tile's first warp: barrier, then one copy of each whole row (K/2 bytes)
     if (l == 0) {
       asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(bar)) : "memory");
       asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-      mbar_arrive_expect_tx(bar, 8u * slice_bytes);
+      mbar_arrive_expect_tx(bar, (uint32_t)(8 * ldp));
     }
     __syncwarp();
     if (l < 8)
       asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-                       smem_u32(wsm + (size_t)l * q.pitch + (size_t)g0 * gbytes)),
-                   "l"(p.Wq + (int64_t)(n0 + l) * ldp + (int64_t)g0 * gbytes), "r"(slice_bytes), "r"(smem_u32(bar))
+                       smem_u32(wsm + (size_t)l * q.pitch)),
+                   "l"(p.Wq + (int64_t)(n0 + l) * ldp), "r"((uint32_t)ldp), "r"(smem_u32(bar))
                    : "memory");
+  }
+  __syncthreads();   // the n-tile barriers are initialised before any warp waits on them
+  if (active && g1 > g0) {
     // activation codes of the first span, loaded while the weights are in flight
     const int spans_per_group = p.G / 128;
     const int abytes = A8 ? 32 : 16;                     // this lane's activation bytes per span and row
