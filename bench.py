@@ -501,6 +501,18 @@ def _graph_time(fn, n, period, warm=3):
     return e0.elapsed_time(e1) / n / 1e3
 
 
+L2_FLUSH_BYTES = 256_000_000   # twice the 126 MB L2
+
+
+def _rotating(tensors, min_sets=3):
+    """Copies of a step's operands (the first set is the tensors themselves), enough that the sets
+    together exceed twice the L2: replaying them in turn, no step finds its operands in L2 (the
+    layer-by-layer case of a model larger than L2)."""
+    nbytes = sum(t.numel() * t.element_size() for t in tensors)
+    nsets = max(min_sets, -(-L2_FLUSH_BYTES // max(1, nbytes)))
+    return [tuple(tensors)] + [tuple(t.clone() for t in tensors) for _ in range(nsets - 1)]
+
+
 def run_extra(hbr, W, dev, stream, peaks):
     import torch
     out = {}
@@ -540,7 +552,13 @@ def run_extra(hbr, W, dev, stream, peaks):
         N = Wq.shape[0]
         C = torch.empty((wl.M, N), dtype=torch.bfloat16, device=dev)
         n = 50 if wl.M > 16 else 200
-        t = _graph_time(lambda i: hbr.w4a4_linear(Aq, As_, Wq, Ws, G, out=C), n, 10)
+        sets = _rotating((Aq, As_, Wq, Ws, C))
+
+        def lin(i, sets=sets):
+            a, sa, w, sw, c = sets[i % len(sets)]
+            hbr.w4a4_linear(a, sa, w, sw, G, out=c)
+        t = _graph_time(lin, n, len(sets))
+        del sets
         ops = 2.0 * wl.M * N * wl.K
         wbytes = Wq.numel() + Ws.numel() * 2 + Aq.numel() + As_.numel() * 2 + C.numel() * 2
         out[f"w4a4_{name}"] = {"us": round(t * 1e6, 2), "TOPS": round(ops / t / 1e12, 1),
@@ -579,25 +597,42 @@ def run_extra_next(hbr, W, dev, hbm, int8_peak):
         C = torch.empty((wl.M, N), dtype=torch.bfloat16, device=dev)
         n = 50 if wl.M > 16 else 200
         ops = 2.0 * wl.M * N * wl.K
+        # every timing replays rotating operand sets (together above twice the L2)
         # W4A8: int8 activation codes
         A8, S8 = hbr.rot_quant(dA, plan, 8, G)
-        A8i = A8.view(torch.int8)
-        t = _graph_time(lambda i: hbr.w4a8_linear(A8i, S8, Wq, Ws, G, out=C), n, 10)
+        sets = _rotating((A8.view(torch.int8), S8, Wq, Ws, C))
+
+        def w8(i, sets=sets):
+            a, sa, w, sw, c = sets[i % len(sets)]
+            hbr.w4a8_linear(a, sa, w, sw, G, out=c)
+        t = _graph_time(w8, n, len(sets))
+        del sets
         out[f"w4a8_{name}"] = {"us": round(t * 1e6, 2), "TOPS": round(ops / t / 1e12, 1),
                                "frac_int8_measured": round(ops / t / 1e12 / int8_peak, 4) if int8_peak else None}
         # one call: rotate + quantise the bf16 activations, then the linear
         ws = torch.empty(hbr.w4a4_linear_act_workspace(wl.M, wl.K, G), dtype=torch.uint8, device=dev)
-        t = _graph_time(lambda i: hbr.w4a4_linear_act(dA, plan, Wq, Ws, G, out=C, workspace=ws), n, 10)
         A4, S4 = hbr.rot_quant(dA, plan, 4, G)
+        sets = _rotating((dA, A4, S4, Wq, Ws, C, ws))
 
-        def sep(i):
-            hbr.rot_quant(dA, plan, 4, G, codes=A4, scales=S4)
-            hbr.w4a4_linear(A4, S4, Wq, Ws, G, out=C)
-        t2 = _graph_time(sep, n, 10)
+        def act(i, sets=sets):
+            a, _, _, w, sw, c, wsp = sets[i % len(sets)]
+            hbr.w4a4_linear_act(a, plan, w, sw, G, out=c, workspace=wsp)
+
+        def sep(i, sets=sets):
+            a, a4, s4, w, sw, c, _ = sets[i % len(sets)]
+            hbr.rot_quant(a, plan, 4, G, codes=a4, scales=s4)
+            hbr.w4a4_linear(a4, s4, w, sw, G, out=c)
+        t = _graph_time(act, n, len(sets))
+        t2 = _graph_time(sep, n, len(sets))
         out[f"act_path_{name}"] = {"us": round(t * 1e6, 2), "separate_calls_us": round(t2 * 1e6, 2)}
         # two-sided: the output rows returned through an RHT of size N
         U = hbr.Plan.rht(N, W.signs(W.rng(77), N))
-        t = _graph_time(lambda i: hbr.w4a4_linear_rot(A4, S4, Wq, Ws, G, U, out=C), n, 10)
+
+        def two(i, sets=sets):
+            _, a4, s4, w, sw, c, _ = sets[i % len(sets)]
+            hbr.w4a4_linear_rot(a4, s4, w, sw, G, U, out=c)
+        t = _graph_time(two, n, len(sets))
+        del sets
         out[f"two_sided_{name}"] = {"us": round(t * 1e6, 2)}
     # HARP K = 11008 with int8-stored parameters (256 Cayley blocks of radix 43), the fp32
     # per-block QR variant, and 5120 = (8, 8, 8, 5, 2)
@@ -639,7 +674,12 @@ def run_profile(args):
         Aq, As = hbr.rot_quant(torch.from_numpy(wl.A).to(torch.bfloat16).to(dev), plan, bits, G)
         Wq, Ws = hbr.rot_quant(torch.from_numpy(np.ascontiguousarray(wl.W.T)).to(dev), plan, bits, G)
         C = torch.empty((wl.M, Wq.shape[0]), dtype=torch.bfloat16, device=dev)
-        fn = lambda i: hbr.w4a4_linear(Aq, As, Wq, Ws, G, out=C)
+        sets = _rotating((Aq, As, Wq, Ws, C))
+        nsets = len(sets)
+
+        def fn(i):
+            a, sa, w, sw, c = sets[i % nsets]
+            hbr.w4a4_linear(a, sa, w, sw, G, out=c)
         work = 2.0 * wl.M * Wq.shape[0] * wl.K
         unit = "TOPS"
     else:
@@ -664,7 +704,7 @@ def run_profile(args):
                                      scales=outs[i % nsets][1])
         work = algorithmic_bytes(wl.M, wl.K, bits, G)
         unit = "GB/s"
-    t = _graph_time(fn, args.steps, 10 if name.startswith("w4a4") else nsets, warm=args.warmup)
+    t = _graph_time(fn, args.steps, nsets, warm=args.warmup)
     print(json.dumps({"profile": name, "us_per_launch": round(t * 1e6, 3),
                       unit: round(work / t / 1e9 if unit == "GB/s" else work / t / 1e12, 2)}))
     return 0

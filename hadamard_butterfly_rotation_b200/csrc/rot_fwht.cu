@@ -824,15 +824,6 @@ size_t mma_smem_bytes(int K) {
   return 256 + (size_t)MMA_SLOTS * MMA_SSTRIDE * 4 + (size_t)MMA_BARS * 8 + (size_t)(K / 2) * 4;
 }
 
-// Programmatic dependent launch (the kernel's prologue may overlap the previous kernel in
-// the stream); ROT_B200_PDL=0 in the environment turns it off.
-bool pdl_enabled() {
-  static const bool on = [] {
-    const char* e = std::getenv("ROT_B200_PDL");
-    return !(e && e[0] == '0');
-  }();
-  return on;
-}
 
 template <int LOGN>
 size_t fused_smem_bytes(int K, bool dual) {
@@ -882,7 +873,7 @@ rot_status launch_one(const Args& a, cudaStream_t s) {
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = pdl_enabled() ? 1 : 0;
+  cfg.numAttrs = pdl_default() ? 1 : 0;
   ROT_CUDA_TRY(cudaLaunchKernelEx(&cfg, kern, a));
   ROT_CUDA_TRY(cudaGetLastError());
   return ROT_OK;
@@ -924,7 +915,7 @@ rot_status launch_mma(const Args& a, cudaStream_t s) {
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = pdl_enabled() ? 1 : 0;
+  cfg.numAttrs = pdl_default() ? 1 : 0;
   ROT_CUDA_TRY(cudaLaunchKernelEx(&cfg, kern, a));
   return ROT_OK;
 }

@@ -78,6 +78,11 @@ rot_status dequant_launch(const uint8_t* codes, const uint16_t* scales, int64_t 
 // split-K accumulation: `scratch` (scratch_floats floats) if non-null, else a stream-ordered
 // temporary; only used for bf16 output on the split path
 constexpr int64_t W4A4_NOALLOC_SCRATCH_FLOATS = int64_t(1) << 20;
+// Programmatic dependent launch for the library's kernels (a kernel's prologue may overlap the
+// previous kernel in the stream; every kernel orders its global accesses after griddepcontrol.wait,
+// L2 prefetches of constant operands aside); ROT_B200_PDL=0 in the environment turns it off.
+bool pdl_default();
+
 rot_status w4a4_launch(const uint8_t* Aq, const uint16_t* As, const uint8_t* Wq,
                        const uint16_t* Ws, int64_t M, int64_t N, int64_t K, int G, void* C,
                        int c_dtype, int32_t* partials, cudaStream_t s, float* scratch = nullptr,

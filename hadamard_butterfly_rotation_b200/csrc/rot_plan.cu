@@ -8,6 +8,7 @@
 // Sylvester-Hadamard stages over the leading digits are, per contiguous chunk of
 // 2^n coordinates, a signed Walsh-Hadamard transform [HARP abstract: the processor
 // initialises to the RHT]; those run on the fused butterfly kernel.
+#include <cstdlib>
 #include <algorithm>
 #include <atomic>
 #include <cmath>
@@ -57,6 +58,14 @@ bool take_test_fault(int which) {
 unsigned long long wait_limit_ns(unsigned long long dflt) {
   const long long v = g_test_wait_ns.load();
   return v > 0 ? (unsigned long long)v : dflt;
+}
+
+bool pdl_default() {
+  static const bool on = [] {
+    const char* e = std::getenv("ROT_B200_PDL");
+    return !(e && e[0] == '0');
+  }();
+  return on;
 }
 
 static bool is_pow2(int64_t x) { return x >= 1 && (x & (x - 1)) == 0; }

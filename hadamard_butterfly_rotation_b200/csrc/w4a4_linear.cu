@@ -868,39 +868,111 @@ __global__ void __launch_bounds__(DEC_THREADS) w4a4_decode_kernel(const DecParam
 // n-tile streams its 8 whole rows into shared memory at the start with one bulk asynchronous copy per
 // row, completing on the n-tile's mbarrier that all its slice warps wait on, so every SM has its whole
 // share of the weight stream in flight at once; the activation codes (L1/L2-resident) are loaded one
-// span ahead. The K-slices
-// are summed through shared memory and the CTA writes its tile of C directly (no atomics, no
-// second launch). Rows are staged K/2 + 64 bytes apart: the 16-byte reads of a quarter-warp
-// (rows g, g + 1 and pieces 0..3) fall in 8 distinct bank groups.
+// span ahead and the scales per group. The K-slices are summed through shared memory and the CTA
+// writes its tile of C directly (no atomics, no second launch). Rows are staged K/2 + 64 bytes apart:
+// the 16-byte reads of a quarter-warp (rows g, g + 1 and pieces 0..3) fall in 8 distinct bank groups.
 __device__ int g_dec_error = 0;
+
+constexpr int DEC_HDR = 256;   // mbarriers, then the staged weight rows
 
 struct StagedDec {
   int npc, ks;       // n-tiles per CTA, K-slices
   int pitch;         // bytes between staged weight rows
+  int apitch;        // one-tile kernel: bytes between staged activation rows
+  int off_acts, off_sa, off_sw, off_red;   // shared-memory offsets (one-tile kernel: all four)
+  int scale_copy;    // one-tile kernel: the scale rows arrive by bulk copy (16-byte aligned, NG % 8 == 0)
 };
 
 constexpr int staged_threads(int mt) { return mt >= 3 ? 256 : 512; }   // bound on the CTA (registers)
+
+// Bounded wait on phase 0 of a staging mbarrier (one use per launch); false when it gave up.
+__device__ __forceinline__ bool dec_wait(uint64_t* bar, unsigned long long wait_ns) {
+  const uint32_t addr = smem_u32(bar);
+  unsigned long long t0 = 0;
+  for (uint32_t it = 0;; ++it) {
+    uint32_t done;
+    asm volatile("{\n\t.reg .pred q;\n\tmbarrier.try_wait.parity.shared::cta.b64 q, [%1], 0;\n\t"
+                 "selp.u32 %0, 1, 0, q;\n\t}"
+                 : "=r"(done)
+                 : "r"(addr)
+                 : "memory");
+    if (done) return true;
+    if ((it & 63) == 63) {
+      unsigned long long now;
+      asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(now));
+      if (t0 == 0) t0 = now;
+      else if (now - t0 > wait_ns) {
+        atomicExch(&g_dec_error, (int)ROT_ETIMEOUT);
+        return false;
+      }
+    }
+  }
+}
+
+// A fragments (m16n8k32, s8) of the four K = 32 steps of one 128-code span: activation pieces lo
+// (row g) / hi (row g + 8) of this lane. W4A4: 16 packed bytes per row hold the span's codes of this
+// lane's quarter; they become the even codes (times 16, low nibbles moved up) and the odd codes (high
+// nibbles in place) of every 8-code word, the K order the weight fragments use too. W4A8: 32 int8
+// codes per row, split into even / odd codes by byte permutes.
+template <bool A8>
+__device__ __forceinline__ void dec_a_frags(uint32_t (&a)[4][4], const uint4 (&lo)[2], const uint4 (&hi)[2]) {
+  if constexpr (A8) {
+    const uint32_t al[8] = {lo[0].x, lo[0].y, lo[0].z, lo[0].w, lo[1].x, lo[1].y, lo[1].z, lo[1].w};
+    const uint32_t ah[8] = {hi[0].x, hi[0].y, hi[0].z, hi[0].w, hi[1].x, hi[1].y, hi[1].z, hi[1].w};
+#pragma unroll
+    for (int s4 = 0; s4 < 4; ++s4) {
+      a[s4][0] = prmt(al[2 * s4], al[2 * s4 + 1], 0x6420u);
+      a[s4][1] = prmt(ah[2 * s4], ah[2 * s4 + 1], 0x6420u);
+      a[s4][2] = prmt(al[2 * s4], al[2 * s4 + 1], 0x7531u);
+      a[s4][3] = prmt(ah[2 * s4], ah[2 * s4 + 1], 0x7531u);
+    }
+  } else {
+    const uint32_t al[4] = {lo[0].x, lo[0].y, lo[0].z, lo[0].w};
+    const uint32_t ah[4] = {hi[0].x, hi[0].y, hi[0].z, hi[0].w};
+#pragma unroll
+    for (int s4 = 0; s4 < 4; ++s4) {
+      a[s4][0] = (al[s4] << 4) & 0xF0F0F0F0u;
+      a[s4][1] = (ah[s4] << 4) & 0xF0F0F0F0u;
+      a[s4][2] = al[s4] & 0xF0F0F0F0u;
+      a[s4][3] = ah[s4] & 0xF0F0F0F0u;
+    }
+  }
+}
+
+// The four MMAs of one span against weight piece wv (16 packed bytes of row g of an n-tile).
+__device__ __forceinline__ void dec_span_mma(int (&d)[4], const uint32_t (&a)[4][4], uint4 wv) {
+  const uint32_t ww[4] = {wv.x, wv.y, wv.z, wv.w};
+#pragma unroll
+  for (int s4 = 0; s4 < 4; ++s4) mma_s8_16832(d, a[s4], (ww[s4] << 4) & 0xF0F0F0F0u, ww[s4] & 0xF0F0F0F0u);
+}
+
+// L2 prefetch of a weight row ahead of griddepcontrol.wait. L2 is the device's point of coherence,
+// so the prefetch is safe even if the previous kernel in the stream is still writing the row: the
+// shared-memory copies issued after the wait read the current data (from L2 when prefetched).
+__device__ __forceinline__ void l2_prefetch(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
 
 template <int MT, bool A8>
 __global__ void __launch_bounds__(staged_threads(MT)) w4a4_decode_staged_kernel(const DecParams p, const StagedDec q) {
   constexpr float UNIT = A8 ? 16.0f : 256.0f;
   extern __shared__ __align__(128) uint8_t dsm[];
-  asm volatile("griddepcontrol.wait;" ::: "memory");   // see w4a4_kernel (programmatic launch)
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int warp = threadIdx.x >> 5, l = threadIdx.x & 31;
   const int g = l >> 2, c = l & 3;
   const int tl = warp % q.npc, ks = warp / q.npc;
   const int n0 = (blockIdx.x * q.npc + tl) * 8;
   const bool active = n0 < p.N;
+  if (ks == 0 && active && l < 8) l2_prefetch(p.Wq + (int64_t)(n0 + l) * (p.K / 2), (uint32_t)(p.K / 2));
+  asm volatile("griddepcontrol.wait;" ::: "memory");   // see w4a4_kernel (programmatic launch)
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int NG = p.K / p.G;
   const int g0 = (int)((int64_t)NG * ks / q.ks);
   int g1 = (int)((int64_t)NG * (ks + 1) / q.ks);
-  const int gbytes = p.G / 2;                              // packed bytes of one group of a row
-  uint64_t* bar = reinterpret_cast<uint64_t*>(dsm) + tl;   // one per n-tile
-  const int nwarps = q.npc * q.ks;
-  uint8_t* wsm = dsm + ((nwarps * 8 + 127) & ~127) + (size_t)tl * 8 * q.pitch;
-  float* red = reinterpret_cast<float*>(dsm + ((nwarps * 8 + 127) & ~127) + (size_t)q.npc * 8 * q.pitch);
+  uint64_t* bar = reinterpret_cast<uint64_t*>(dsm) + tl;       // one per n-tile
+  uint8_t* wsm = dsm + DEC_HDR + (size_t)tl * 8 * q.pitch;
+  float* red = reinterpret_cast<float*>(dsm + q.off_red);
   const int64_t ldp = p.K / 2;
+  const int64_t arow = A8 ? p.K : ldp;                         // bytes of one activation row
   float acc[MT][4];
 #pragma unroll
   for (int t = 0; t < MT; ++t)
@@ -923,10 +995,10 @@ __global__ void __launch_bounds__(staged_threads(MT)) w4a4_decode_staged_kernel(
   }
   __syncthreads();   // the n-tile barriers are initialised before any warp waits on them
   if (active && g1 > g0) {
-    // activation codes of the first span, loaded while the weights are in flight
     const int spans_per_group = p.G / 128;
+    const uint8_t* wlane = wsm + (size_t)g * q.pitch + 16 * c;
+    // activation codes of the first span, loaded while the weights are in flight
     const int abytes = A8 ? 32 : 16;                     // this lane's activation bytes per span and row
-    const int64_t lda = A8 ? p.K : ldp;
     auto a_load = [&](int span, uint4 (&lo)[MT][2], uint4 (&hi)[MT][2]) {
 #pragma unroll
       for (int t = 0; t < MT; ++t) {
@@ -934,12 +1006,12 @@ __global__ void __launch_bounds__(staged_threads(MT)) w4a4_decode_staged_kernel(
         const int64_t off = (int64_t)span * (A8 ? 128 : 64) + abytes * c;
         lo[t][0] = lo[t][1] = hi[t][0] = hi[t][1] = make_uint4(0u, 0u, 0u, 0u);
         if (m_lo < p.M) {
-          const uint4* src = reinterpret_cast<const uint4*>(p.Aq + (int64_t)m_lo * lda + off);
+          const uint4* src = reinterpret_cast<const uint4*>(p.Aq + (int64_t)m_lo * arow + off);
           lo[t][0] = __ldg(src);
           if (A8) lo[t][1] = __ldg(src + 1);
         }
         if (m_hi < p.M) {
-          const uint4* src = reinterpret_cast<const uint4*>(p.Aq + (int64_t)m_hi * lda + off);
+          const uint4* src = reinterpret_cast<const uint4*>(p.Aq + (int64_t)m_hi * arow + off);
           hi[t][0] = __ldg(src);
           if (A8) hi[t][1] = __ldg(src + 1);
         }
@@ -948,34 +1020,8 @@ __global__ void __launch_bounds__(staged_threads(MT)) w4a4_decode_staged_kernel(
     uint4 alo[MT][2], ahi[MT][2];
     int span = g0 * spans_per_group;
     a_load(span, alo, ahi);
-
     // bounded wait for the warp's weight slice
-    {
-      const uint32_t addr = smem_u32(bar);
-      unsigned long long t0 = 0;
-      bool ok = true;
-      for (uint32_t it = 0;; ++it) {
-        uint32_t done;
-        asm volatile("{\n\t.reg .pred q;\n\tmbarrier.try_wait.parity.shared::cta.b64 q, [%1], 0;\n\t"
-                     "selp.u32 %0, 1, 0, q;\n\t}"
-                     : "=r"(done)
-                     : "r"(addr)
-                     : "memory");
-        if (done) break;
-        if ((it & 63) == 63) {
-          unsigned long long now;
-          asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(now));
-          if (t0 == 0) t0 = now;
-          else if (now - t0 > p.wait_ns) {
-            atomicExch(&g_dec_error, (int)ROT_ETIMEOUT);
-            ok = false;
-            break;
-          }
-        }
-      }
-      if (!__all_sync(0xffffffffu, ok)) g1 = g0;   // gave up: compute nothing (outputs unspecified)
-    }
-    const uint8_t* wlane = wsm + (size_t)g * q.pitch + 16 * c;
+    if (!__all_sync(0xffffffffu, dec_wait(bar, p.wait_ns))) g1 = g0;   // gave up: compute nothing
     for (int gg = g0; gg < g1; ++gg) {
       int d[MT][4];
 #pragma unroll
@@ -990,30 +1036,11 @@ __global__ void __launch_bounds__(staged_threads(MT)) w4a4_decode_staged_kernel(
           clo[t][0] = alo[t][0]; clo[t][1] = alo[t][1]; chi[t][0] = ahi[t][0]; chi[t][1] = ahi[t][1];
         }
         if (span + 1 < g1 * spans_per_group) a_load(span + 1, alo, ahi);   // next span's activations
-        const uint32_t ww[4] = {wv.x, wv.y, wv.z, wv.w};
 #pragma unroll
         for (int t = 0; t < MT; ++t) {
-          if constexpr (A8) {
-            const uint32_t al[8] = {clo[t][0].x, clo[t][0].y, clo[t][0].z, clo[t][0].w,
-                                    clo[t][1].x, clo[t][1].y, clo[t][1].z, clo[t][1].w};
-            const uint32_t ah[8] = {chi[t][0].x, chi[t][0].y, chi[t][0].z, chi[t][0].w,
-                                    chi[t][1].x, chi[t][1].y, chi[t][1].z, chi[t][1].w};
-#pragma unroll
-            for (int s4 = 0; s4 < 4; ++s4) {
-              const uint32_t a[4] = {prmt(al[2 * s4], al[2 * s4 + 1], 0x6420u), prmt(ah[2 * s4], ah[2 * s4 + 1], 0x6420u),
-                                     prmt(al[2 * s4], al[2 * s4 + 1], 0x7531u), prmt(ah[2 * s4], ah[2 * s4 + 1], 0x7531u)};
-              mma_s8_16832(d[t], a, (ww[s4] << 4) & 0xF0F0F0F0u, ww[s4] & 0xF0F0F0F0u);
-            }
-          } else {
-            const uint32_t al[4] = {clo[t][0].x, clo[t][0].y, clo[t][0].z, clo[t][0].w};
-            const uint32_t ah[4] = {chi[t][0].x, chi[t][0].y, chi[t][0].z, chi[t][0].w};
-#pragma unroll
-            for (int s4 = 0; s4 < 4; ++s4) {
-              const uint32_t a[4] = {(al[s4] << 4) & 0xF0F0F0F0u, (ah[s4] << 4) & 0xF0F0F0F0u, al[s4] & 0xF0F0F0F0u,
-                                     ah[s4] & 0xF0F0F0F0u};
-              mma_s8_16832(d[t], a, (ww[s4] << 4) & 0xF0F0F0F0u, ww[s4] & 0xF0F0F0F0u);
-            }
-          }
+          uint32_t a[4][4];
+          dec_a_frags<A8>(a, clo[t], chi[t]);
+          dec_span_mma(d[t], a, wv);
         }
       }
       const float sw0 = __half2float(__ushort_as_half(p.Ws[(int64_t)(n0 + 2 * c) * NG + gg])) * (1.0f / UNIT);
@@ -1061,6 +1088,164 @@ __global__ void __launch_bounds__(staged_threads(MT)) w4a4_decode_staged_kernel(
       } else {
         *reinterpret_cast<float2*>(static_cast<float*>(p.C) + (int64_t)m * p.N + n) = make_float2(v0, v1);
       }
+    }
+  }
+}
+
+// One-tile decode kernel (M <= 16 tokens): everything the group loop reads sits in shared memory.
+// A CTA owns NPC n-tiles; warp 0 issues one bulk copy per weight row of all of them and one per
+// activation row, and (q.scale_copy) one copy each of the CTA's weight-scale rows and of the token
+// scale rows (binary16, contiguous in Ws and As), completing on two mbarriers; without scale copies
+// (unaligned scale tables) the threads load the scales into shared memory instead. Before
+// griddepcontrol.wait the CTA's weight rows are prefetched into L2. Warp w computes ALL n-tiles of
+// the CTA over K-slice w: each span's activation fragments are built once and used by the MMAs of
+// every n-tile. The slices are summed through shared memory, warp t sums n-tile t and writes it.
+// Activation rows are staged arow + 64 (W4A4) or + 16 (W4A8) bytes past a 128-byte multiple apart,
+// so the quarter-warp reads (rows g, g + 1) are conflict-free.
+template <bool A8, int NPC>
+__global__ void __launch_bounds__(512) w4a4_decode_tile1_kernel(const DecParams p, const StagedDec q) {
+  constexpr float UNIT = A8 ? 16.0f : 256.0f;
+  extern __shared__ __align__(128) uint8_t dsm[];
+  const int warp = threadIdx.x >> 5, l = threadIdx.x & 31;
+  const int g = l >> 2, c = l & 3;
+  const int NG = p.K / p.G;
+  const int64_t nrow0 = (int64_t)blockIdx.x * NPC * 8;                 // first weight row of the CTA
+  const int nrows = (int)(p.N - nrow0 < NPC * 8 ? p.N - nrow0 : NPC * 8);   // a multiple of 8
+  const int ntl = nrows / 8;                                           // active n-tiles
+  if (warp == 0 && l < nrows) l2_prefetch(p.Wq + (nrow0 + l) * (p.K / 2), (uint32_t)(p.K / 2));
+  asm volatile("griddepcontrol.wait;" ::: "memory");   // see w4a4_kernel (programmatic launch)
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  uint64_t* wbar = reinterpret_cast<uint64_t*>(dsm);
+  uint64_t* abar = wbar + 1;
+  uint8_t* wsm = dsm + DEC_HDR;
+  uint8_t* asm_ = dsm + q.off_acts;
+  uint16_t* sA = reinterpret_cast<uint16_t*>(dsm + q.off_sa);          // [16][NG] binary16
+  uint16_t* sW = reinterpret_cast<uint16_t*>(dsm + q.off_sw);          // [NPC * 8][NG] binary16
+  float* red = reinterpret_cast<float*>(dsm + q.off_red);
+  const int64_t ldp = p.K / 2;
+  const int64_t arow = A8 ? p.K : ldp;
+  const uint32_t sa_bytes = (uint32_t)(p.M * NG * 2), sw_bytes = (uint32_t)(nrows * NG * 2);
+
+  if (warp == 0) {
+    if (l == 0) {
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(wbar)) : "memory");
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(abar)) : "memory");
+      asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+      mbar_arrive_expect_tx(wbar, (uint32_t)(nrows * ldp) + (q.scale_copy ? sw_bytes : 0u));
+      mbar_arrive_expect_tx(abar, (uint32_t)(p.M * arow) + (q.scale_copy ? sa_bytes : 0u));
+    }
+    __syncwarp();
+    if (l < nrows)   // NPC * 8 <= 16 rows
+      asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                       smem_u32(wsm + (size_t)l * q.pitch)),
+                   "l"(p.Wq + (nrow0 + l) * ldp), "r"((uint32_t)ldp), "r"(smem_u32(wbar))
+                   : "memory");
+    if (l < p.M)     // M <= 16 rows
+      asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                       smem_u32(asm_ + (size_t)l * q.apitch)),
+                   "l"(p.Aq + (int64_t)l * arow), "r"((uint32_t)arow), "r"(smem_u32(abar))
+                   : "memory");
+    if (q.scale_copy && l == 16)
+      asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                       smem_u32(sW)),
+                   "l"(p.Ws + nrow0 * NG), "r"(sw_bytes), "r"(smem_u32(wbar))
+                   : "memory");
+    if (q.scale_copy && l == 17)
+      asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                       smem_u32(sA)),
+                   "l"(p.As), "r"(sa_bytes), "r"(smem_u32(abar))
+                   : "memory");
+  }
+  if (!q.scale_copy) {
+    for (int i = threadIdx.x; i < p.M * NG; i += blockDim.x) sA[i] = p.As[i];
+    for (int i = threadIdx.x; i < nrows * NG; i += blockDim.x) sW[i] = p.Ws[nrow0 * NG + i];
+  }
+  __syncthreads();   // barriers initialised (and, without scale copies, the scales in shared memory)
+
+  float acc[NPC][4];
+#pragma unroll
+  for (int t = 0; t < NPC; ++t)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) acc[t][i] = 0.0f;
+  // K-slice of this warp (warps past q.ks only help to sum and store)
+  const int g0 = warp < q.ks ? (int)((int64_t)NG * warp / q.ks) : 0;
+  int g1 = warp < q.ks ? (int)((int64_t)NG * (warp + 1) / q.ks) : 0;
+  if (g1 > g0) {
+    const bool ok = dec_wait(wbar, p.wait_ns) && dec_wait(abar, p.wait_ns);
+    if (!__all_sync(0xffffffffu, ok)) g1 = g0;   // gave up: compute nothing (outputs unspecified)
+  }
+  const int spans_per_group = p.G / 128;
+  const uint8_t* wlane = wsm + (size_t)g * q.pitch + 16 * c;
+  const uint8_t* alo = asm_ + (size_t)g * q.apitch + (A8 ? 32 : 16) * c;
+  const uint8_t* ahi = alo + (size_t)8 * q.apitch;
+  const bool lo_on = g < p.M, hi_on = g + 8 < p.M;   // token rows past M: scale 0 (rows not staged)
+  int span = g0 * spans_per_group;
+  for (int gg = g0; gg < g1; ++gg) {
+    int d[NPC][4];
+#pragma unroll
+    for (int t = 0; t < NPC; ++t)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) d[t][i] = 0;
+    for (int sp = 0; sp < spans_per_group; ++sp, ++span) {
+      const size_t ao = (size_t)span * (A8 ? 128 : 64);
+      uint4 lo[2], hi[2];
+      lo[0] = *reinterpret_cast<const uint4*>(alo + ao);
+      hi[0] = *reinterpret_cast<const uint4*>(ahi + ao);
+      if constexpr (A8) {
+        lo[1] = *reinterpret_cast<const uint4*>(alo + ao + 16);
+        hi[1] = *reinterpret_cast<const uint4*>(ahi + ao + 16);
+      } else {
+        lo[1] = hi[1] = make_uint4(0u, 0u, 0u, 0u);
+      }
+      uint4 wv[NPC];
+#pragma unroll
+      for (int t = 0; t < NPC; ++t)
+        if (t < ntl) wv[t] = *reinterpret_cast<const uint4*>(wlane + (size_t)t * 8 * q.pitch + (size_t)span * 64);
+      uint32_t a[4][4];
+      dec_a_frags<A8>(a, lo, hi);
+#pragma unroll
+      for (int t = 0; t < NPC; ++t)
+        if (t < ntl) dec_span_mma(d[t], a, wv[t]);
+    }
+    const float sa0 = lo_on ? __half2float(__ushort_as_half(sA[g * NG + gg])) : 0.0f;
+    const float sa1 = hi_on ? __half2float(__ushort_as_half(sA[(g + 8) * NG + gg])) : 0.0f;
+#pragma unroll
+    for (int t = 0; t < NPC; ++t) {
+      if (t < ntl) {
+        const float sw0 = __half2float(__ushort_as_half(sW[(t * 8 + 2 * c) * NG + gg])) * (1.0f / UNIT);
+        const float sw1 = __half2float(__ushort_as_half(sW[(t * 8 + 2 * c + 1) * NG + gg])) * (1.0f / UNIT);
+        acc[t][0] = fmaf((float)d[t][0] * sw0, sa0, acc[t][0]);
+        acc[t][1] = fmaf((float)d[t][1] * sw1, sa0, acc[t][1]);
+        acc[t][2] = fmaf((float)d[t][2] * sw0, sa1, acc[t][2]);
+        acc[t][3] = fmaf((float)d[t][3] * sw1, sa1, acc[t][3]);
+      }
+    }
+  }
+  // every slice parks its partial sums (slice-major); warp t then sums n-tile t and writes it
+  if (warp < q.ks) {
+#pragma unroll
+    for (int t = 0; t < NPC; ++t)
+      *reinterpret_cast<float4*>(red + ((size_t)(warp * NPC + t) * 32 + l) * 4) =
+          make_float4(acc[t][0], acc[t][1], acc[t][2], acc[t][3]);
+  }
+  __syncthreads();
+  if (warp >= ntl) return;
+  float4 v = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+  for (int k = 0; k < q.ks; ++k) {
+    const float4 r = *reinterpret_cast<const float4*>(red + ((size_t)(k * NPC + warp) * 32 + l) * 4);
+    v.x += r.x; v.y += r.y; v.z += r.z; v.w += r.w;
+  }
+  const int64_t n = nrow0 + warp * 8 + 2 * c;
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int m = g + 8 * h;
+    if (m >= p.M) continue;
+    const float v0 = h ? v.z : v.x, v1 = h ? v.w : v.y;
+    if (p.c_bf16) {
+      *reinterpret_cast<__nv_bfloat162*>(static_cast<__nv_bfloat16*>(p.C) + (int64_t)m * p.N + n) =
+          __floats2bfloat162_rn(v0, v1);
+    } else {
+      *reinterpret_cast<float2*>(static_cast<float*>(p.C) + (int64_t)m * p.N + n) = make_float2(v0, v1);
     }
   }
 }
@@ -1132,6 +1317,7 @@ cudaError_t launch_maybe_pdl(void (*kern)(const P), dim3 grid, dim3 block, size_
 rot_status w4a4_launch(const uint8_t* Aq, const uint16_t* As, const uint8_t* Wq, const uint16_t* Ws, int64_t M,
                        int64_t N, int64_t K, int G, void* C, int c_dtype, int32_t* partials, cudaStream_t s,
                        float* scratch, int64_t scratch_floats, bool a8, bool pdl) {
+  pdl = pdl || pdl_default();
   if (G > 256) return set_error(ROT_EUNSUPPORTED, "w4a4_linear: G > 256 is not supported");
   if (M > (1ll << 30) || N > (1ll << 30) || K > (1ll << 30)) return set_error(ROT_EUNSUPPORTED, "w4a4_linear: size too large");
   // fp32 accumulation target for K-split launches: C itself (fp32), the caller's scratch, or a
@@ -1178,43 +1364,23 @@ rot_status w4a4_launch(const uint8_t* Aq, const uint16_t* As, const uint8_t* Wq,
     d.G = G;
     d.c_bf16 = c_dtype == ROT_BF16;
     d.wait_ns = wait_limit_ns(WAIT_NS);
-    // staged weight stream (shared memory, rows K/2 + 64 bytes apart): enough n-tiles per CTA that
-    // every CTA is resident at once (two per SM), K-slices to bring the CTA to about 16 warps
-    const int64_t pitch = K / 2 + 64;
+    const int64_t pitch = K / 2 + 64;   // staged weight rows (conflict-free quarter-warp reads)
     const int64_t sms = sm_count();
-    const int max_warps = (mt >= 3 ? 256 : 512) / 32;
-    int npc = (int)std::max<int64_t>(1, (ntiles + 2 * sms - 1) / (2 * sms));
-    int ksl = std::max(1, std::min(NG, max_warps / std::max(1, npc)));
-    auto smem_of = [&](int np, int kk) -> size_t {
-      return (size_t)((np * kk * 8 + 127) & ~127) + (size_t)np * 8 * pitch + (size_t)(kk - 1) * np * 32 * 4 * mt * 4;
-    };
-    while (npc > 1 && smem_of(npc, ksl) > 110 * 1024) {   // keep two CTAs per SM
-      npc = (npc + 1) / 2;
-      ksl = std::max(1, std::min(NG, max_warps / npc));
-    }
-    if (npc * ksl <= max_warps && smem_of(npc, ksl) <= 200 * 1024) {
-      StagedDec q;
-      q.npc = npc;
-      q.ks = ksl;
-      q.pitch = (int)pitch;
-      d.groups_per_split = NG;
-      const size_t smem = smem_of(npc, ksl);
-      void (*dk)(const DecParams, const StagedDec) = nullptr;
-      if (a8) dk = mt == 1 ? w4a4_decode_staged_kernel<1, true> : mt == 2 ? w4a4_decode_staged_kernel<2, true>
-                   : mt == 3 ? w4a4_decode_staged_kernel<3, true> : w4a4_decode_staged_kernel<4, true>;
-      else dk = mt == 1 ? w4a4_decode_staged_kernel<1, false> : mt == 2 ? w4a4_decode_staged_kernel<2, false>
-                : mt == 3 ? w4a4_decode_staged_kernel<3, false> : w4a4_decode_staged_kernel<4, false>;
-      static int dec_configured[64][8] = {};   // per device and (A8, MT) variant: the opt-in limit set once
+    auto set_limit = [&](const void* fn, int var) -> rot_status {
+      static int dec_configured[64][16] = {};   // per device and variant: the opt-in limit set once
       int dev = 0;
       ROT_CUDA_TRY(cudaGetDevice(&dev));
-      const int var = (a8 ? 4 : 0) + (mt - 1);
       if (dev >= 64 || !dec_configured[dev][var]) {
-        ROT_CUDA_TRY(cudaFuncSetAttribute(dk, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024));
+        ROT_CUDA_TRY(cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024));
         if (dev < 64) dec_configured[dev][var] = 1;
       }
+      return ROT_OK;
+    };
+    auto launch_dec = [&](void (*dk)(const DecParams, const StagedDec), int64_t grid, int threads, size_t smem,
+                          const StagedDec& q) -> rot_status {
       cudaLaunchConfig_t cfg = {};
-      cfg.gridDim = dim3((unsigned)((ntiles + npc - 1) / npc));
-      cfg.blockDim = dim3(32 * npc * ksl);
+      cfg.gridDim = dim3((unsigned)grid);
+      cfg.blockDim = dim3(threads);
       cfg.dynamicSmemBytes = smem;
       cfg.stream = s;
       cudaLaunchAttribute attr[1];
@@ -1225,6 +1391,71 @@ rot_status w4a4_launch(const uint8_t* Aq, const uint16_t* As, const uint8_t* Wq,
       ROT_CUDA_TRY(cudaLaunchKernelEx(&cfg, dk, d, q));
       ROT_CUDA_TRY(cudaGetLastError());
       return ROT_OK;
+    };
+    d.groups_per_split = NG;
+    // one token tile: weights, activation rows and scales all staged in shared memory, 1 or 2
+    // n-tiles per CTA (every CTA resident at once, two per SM), 8 to 16 K-slices
+    if (mt == 1) {
+      const int64_t need = (ntiles + 2 * sms - 1) / (2 * sms);
+      const int npc1 = need <= 1 ? 1 : need <= 2 ? 2 : 0;
+      if (npc1) {
+        const int64_t arow = a8 ? K : K / 2;
+        const int64_t apitch = ((arow + 127) & ~(int64_t)127) + (a8 ? 16 : 64);
+        StagedDec q{};
+        q.npc = npc1;
+        q.pitch = (int)pitch;
+        q.apitch = (int)apitch;
+        const size_t off_acts = DEC_HDR + (size_t)npc1 * 8 * pitch;
+        const size_t off_sa = off_acts + (size_t)16 * apitch;
+        const size_t off_sw = off_sa + (((size_t)16 * NG * 2 + 15) & ~(size_t)15);
+        const size_t off_red = off_sw + (((size_t)npc1 * 8 * NG * 2 + 15) & ~(size_t)15);
+        int kk = std::min(NG, 16);
+        while (kk > 1 && off_red + (size_t)kk * npc1 * 512 > 110 * 1024) kk = (kk + 1) / 2;
+        const size_t smem = off_red + (size_t)kk * npc1 * 512;
+        if (smem <= 110 * 1024 && kk >= std::min(NG, 8)) {   // (too few warps: the other path)
+          q.ks = kk;
+          q.scale_copy = (NG % 8 == 0 && (reinterpret_cast<uintptr_t>(As) & 15) == 0 &&
+                          (reinterpret_cast<uintptr_t>(Ws) & 15) == 0) ? 1 : 0;
+          q.off_acts = (int)off_acts;
+          q.off_sa = (int)off_sa;
+          q.off_sw = (int)off_sw;
+          q.off_red = (int)off_red;
+          void (*dk)(const DecParams, const StagedDec) =
+              a8 ? (npc1 == 1 ? w4a4_decode_tile1_kernel<true, 1> : w4a4_decode_tile1_kernel<true, 2>)
+                 : (npc1 == 1 ? w4a4_decode_tile1_kernel<false, 1> : w4a4_decode_tile1_kernel<false, 2>);
+          rot_status st = set_limit((const void*)dk, 8 + (a8 ? 2 : 0) + (npc1 - 1));
+          if (st) return st;
+          return launch_dec(dk, (ntiles + npc1 - 1) / npc1, 32 * std::max(kk, npc1), smem, q);
+        }
+      }
+    }
+    // staged weight stream: enough n-tiles per CTA that every CTA is resident at once (two per SM),
+    // K-slices to bring the CTA to about 16 warps
+    const int max_warps = (mt >= 3 ? 256 : 512) / 32;
+    int npc = (int)std::max<int64_t>(1, (ntiles + 2 * sms - 1) / (2 * sms));
+    int ksl = std::max(1, std::min(NG, max_warps / std::max(1, npc)));
+    const size_t red_unit = (size_t)32 * 4 * mt * 4;   // one warp's partial sums
+    auto smem_of = [&](int np, int kk) -> size_t {
+      return (size_t)DEC_HDR + (size_t)np * 8 * pitch + (size_t)(kk - 1) * np * red_unit;
+    };
+    while (npc > 1 && smem_of(npc, ksl) > 110 * 1024) {   // keep two CTAs per SM
+      npc = (npc + 1) / 2;
+      ksl = std::max(1, std::min(NG, max_warps / npc));
+    }
+    if (npc * ksl <= max_warps && smem_of(npc, ksl) <= 200 * 1024) {
+      StagedDec q{};
+      q.npc = npc;
+      q.ks = ksl;
+      q.pitch = (int)pitch;
+      q.off_red = (int)(DEC_HDR + (size_t)npc * 8 * pitch);
+      void (*dk)(const DecParams, const StagedDec) = nullptr;
+      if (a8) dk = mt == 1 ? w4a4_decode_staged_kernel<1, true> : mt == 2 ? w4a4_decode_staged_kernel<2, true>
+                   : mt == 3 ? w4a4_decode_staged_kernel<3, true> : w4a4_decode_staged_kernel<4, true>;
+      else dk = mt == 1 ? w4a4_decode_staged_kernel<1, false> : mt == 2 ? w4a4_decode_staged_kernel<2, false>
+                : mt == 3 ? w4a4_decode_staged_kernel<3, false> : w4a4_decode_staged_kernel<4, false>;
+      rot_status st = set_limit((const void*)dk, (a8 ? 4 : 0) + (mt - 1));
+      if (st) return st;
+      return launch_dec(dk, (ntiles + npc - 1) / npc, 32 * npc * ksl, smem_of(npc, ksl), q);
     }
     // very long rows: the weights stream through registers, K split until about 32 warps per SM
     // are busy (more bytes in flight)

@@ -45,7 +45,8 @@ def test_group_partials_exact(lib, M, N, K, G):
                                      (64, 512, 4096, 128), (200, 176, 192, 32), (16, 256, 1024, 256),
                                      (300, 784, 640, 64), (5, 640, 1152, 96), (130, 208, 1344, 192),
                                      (7, 96, 896, 224), (33, 144, 640, 160), (5, 640, 192, 192),
-                                     (7, 96, 448, 224)])
+                                     (7, 96, 448, 224), (1, 128, 1024, 128), (9, 176, 768, 256),
+                                     (16, 48, 2560, 128)])
 @pytest.mark.parametrize("out", ["f32", "bf16"])
 def test_w4a4_linear_small(lib, M, N, K, G, out):
     import torch

@@ -82,7 +82,8 @@ def test_w4a8_group_partials_exact(lib, M, N, K, G):
 
 @pytest.mark.parametrize("M,N,K,G", [(1, 16, 128, 32), (3, 48, 256, 64), (129, 272, 384, 128), (64, 512, 4096, 128),
                                      (200, 176, 192, 32), (16, 256, 1024, 256), (300, 784, 640, 64),
-                                     (5, 640, 1152, 96), (130, 208, 1344, 192)])
+                                     (5, 640, 1152, 96), (130, 208, 1344, 192), (1, 128, 1024, 128),
+                                     (9, 176, 768, 256), (16, 48, 2560, 128)])
 @pytest.mark.parametrize("out", ["f32", "bf16"])
 def test_w4a8_linear_small(lib, M, N, K, G, out):
     import torch
