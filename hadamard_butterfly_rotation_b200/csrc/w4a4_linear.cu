@@ -255,6 +255,25 @@ __device__ __forceinline__ void umma_i8(uint32_t tmem_d, uint64_t da, uint64_t d
       : "memory");
 }
 
+// The same MMA and commit issued by the calling thread alone (inside an elected branch).
+__device__ __forceinline__ void umma_i8_one(uint32_t tmem_d, uint64_t da, uint64_t db, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+      "l"(da), "l"(db), "r"(IDESC), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void umma_commit_one(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+__device__ __forceinline__ bool elect_one() {
+  uint32_t e;
+  asm volatile("{\n\t.reg .pred P;\n\telect.sync _|P, 0xffffffff;\n\tselp.u32 %0, 1, 0, P;\n\t}" : "=r"(e));
+  return e != 0;
+}
+
 __device__ __forceinline__ void umma_commit(uint64_t* bar) {
   asm volatile(
       "{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
@@ -364,29 +383,33 @@ __global__ void __launch_bounds__(THREADS, 1) w4a4_kernel(const __grid_constant_
     if (lane == 0)
       for (int b = 0; b < NACC; ++b) mbar_arrive(&tempty[b]);
 
-    // Group scales: each warp stages sW/256 of its own 64 columns in a private shared-memory
-    // buffer (lane l: columns l and l + 32), ordered by __syncwarp alone, and keeps sA of its
-    // row in a register. The raw binary16 values are loaded two groups ahead into a two-entry
-    // register ring addressed statically by the parity of the group, from addresses clamped
-    // into the matrix (rows >= M and columns >= N are never stored), so every load is
+    // Group scales: each warp stages sW/UNIT of its own EPI_COLS columns in a private
+    // shared-memory buffer (lane l: columns l + 32 j), ordered by __syncwarp alone, and keeps sA
+    // of its row in a register. The raw binary16 values are loaded two groups ahead into a
+    // two-entry register ring addressed statically by the parity of the group, from addresses
+    // clamped into the matrix (rows >= M and columns >= N are never stored), so every load is
     // unconditional and no register is read while its load is in flight.
+    constexpr int CQ = EPI_COLS / 32;         // column vectors per lane
     float* wsc = slots + warp * EPI_COLS;
     int su = blockIdx.x;                      // load cursor: unit and group within it
     int sg = 0, s_ngl = 0;
-    const uint16_t *cw0 = p.Ws, *cw1 = p.Ws, *ca = p.Ws;   // the cursor group's scales (dummy past the end)
+    const uint16_t* cw[CQ];                   // the cursor group's scales (dummy past the end)
+    const uint16_t* ca = p.Ws;
+#pragma unroll
+    for (int j = 0; j < CQ; ++j) cw[j] = p.Ws;
     auto cursor_unit = [&]() {
       if (su < p.units) {
         const Unit w = unit_of(p, su);
         s_ngl = w.ngl;
-        cw0 = p.Ws + (int64_t)min(w.n0 + wg * EPI_COLS + lane, p.N - 1) * NG + w.g0;
-        cw1 = p.Ws + (int64_t)min(w.n0 + wg * EPI_COLS + 32 + lane, p.N - 1) * NG + w.g0;
+#pragma unroll
+        for (int j = 0; j < CQ; ++j) cw[j] = p.Ws + (int64_t)min(w.n0 + wg * EPI_COLS + 32 * j + lane, p.N - 1) * NG + w.g0;
         ca = p.As + (int64_t)min(w.m0 + row, p.M - 1) * NG + w.g0;
       } else {
-        cw0 = cw1 = ca = p.Ws;
+#pragma unroll
+        for (int j = 0; j < CQ; ++j) cw[j] = p.Ws;
+        ca = p.Ws;
       }
     };
-    auto cursor_w = [&](int half) -> const uint16_t* { return half ? cw1 : cw0; };
-    auto cursor_a = [&]() -> const uint16_t* { return ca; };
     auto cursor_step = [&]() {
       if (su < p.units) {
         if (++sg == s_ngl) {
@@ -394,22 +417,24 @@ __global__ void __launch_bounds__(THREADS, 1) w4a4_kernel(const __grid_constant_
           su += gridDim.x;
           cursor_unit();
         } else {
-          ++cw0;
-          ++cw1;
+#pragma unroll
+          for (int j = 0; j < CQ; ++j) ++cw[j];
           ++ca;
         }
       }
     };
-    uint16_t q0w0 = 0, q0w1 = 0, q0a = 0, q1w0 = 0, q1w1 = 0, q1a = 0;   // groups gc (+1), by parity
+    uint16_t q0w[CQ], q1w[CQ], q0a = 0, q1a = 0;   // groups gc (+1), by parity
+#pragma unroll
+    for (int j = 0; j < CQ; ++j) q0w[j] = q1w[j] = 0;
     if (!PARTIALS) {
       cursor_unit();
-      q0w0 = __ldg(cursor_w(0));
-      q0w1 = __ldg(cursor_w(1));
-      q0a = __ldg(cursor_a());
+#pragma unroll
+      for (int j = 0; j < CQ; ++j) q0w[j] = __ldg(cw[j]);
+      q0a = __ldg(ca);
       cursor_step();
-      q1w0 = __ldg(cursor_w(0));
-      q1w1 = __ldg(cursor_w(1));
-      q1a = __ldg(cursor_a());
+#pragma unroll
+      for (int j = 0; j < CQ; ++j) q1w[j] = __ldg(cw[j]);
+      q1a = __ldg(ca);
       cursor_step();
     }
 
@@ -425,19 +450,26 @@ __global__ void __launch_bounds__(THREADS, 1) w4a4_kernel(const __grid_constant_
       for (int gl = 0; gl < w.ngl; ++gl, ++gc) {
         float sa = 0.0f;
         if (!PARTIALS) {
-          const uint16_t *nw0 = cursor_w(0), *nw1 = cursor_w(1), *na = cursor_a();
+          const uint16_t* nw[CQ];
+#pragma unroll
+          for (int j = 0; j < CQ; ++j) nw[j] = cw[j];
+          const uint16_t* na = ca;
           cursor_step();
-          uint16_t rw0, rw1, ra;
+          uint16_t rw[CQ], ra;
           if (gc & 1) {
-            rw0 = q1w0; rw1 = q1w1; ra = q1a;
-            q1w0 = __ldg(nw0); q1w1 = __ldg(nw1); q1a = __ldg(na);
+#pragma unroll
+            for (int j = 0; j < CQ; ++j) { rw[j] = q1w[j]; q1w[j] = __ldg(nw[j]); }
+            ra = q1a;
+            q1a = __ldg(na);
           } else {
-            rw0 = q0w0; rw1 = q0w1; ra = q0a;
-            q0w0 = __ldg(nw0); q0w1 = __ldg(nw1); q0a = __ldg(na);
+#pragma unroll
+            for (int j = 0; j < CQ; ++j) { rw[j] = q0w[j]; q0w[j] = __ldg(nw[j]); }
+            ra = q0a;
+            q0a = __ldg(na);
           }
           __syncwarp();                 // every lane has read the previous group's column scales
-          wsc[lane] = __half2float(__ushort_as_half(rw0)) * (1.0f / L::UNIT);
-          wsc[lane + 32] = __half2float(__ushort_as_half(rw1)) * (1.0f / L::UNIT);
+#pragma unroll
+          for (int j = 0; j < CQ; ++j) wsc[lane + 32 * j] = __half2float(__ushort_as_half(rw[j])) * (1.0f / L::UNIT);
           sa = __half2float(__ushort_as_half(ra));
           __syncwarp();
         }
@@ -446,21 +478,21 @@ __global__ void __launch_bounds__(THREADS, 1) w4a4_kernel(const __grid_constant_
         if (!ok) break;
         tc_fence_after();
         if constexpr (!PARTIALS) {
-          // The group in two halves of 32 columns: each half's TMEM load is in flight while the
-          // 8 column-scale vectors of that half are loaded from shared memory, so the arithmetic
-          // waits once per half for both (instead of once per scale vector). The accumulator is
-          // released as soon as the second half is in registers.
+          // The group in chunks of 32 columns: each chunk's TMEM load is in flight while the 8
+          // column-scale vectors of that chunk are loaded from shared memory, so the arithmetic
+          // waits once per chunk for both (instead of once per scale vector). The accumulator is
+          // released as soon as the last chunk is in registers.
           const float2 sa2 = make_float2(sa, sa);
           const float2 d2 = make_float2(-BIAS_F * sa, -BIAS_F * sa);   // exact: 3 * 2^22 * binary16
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {
+          for (int h = 0; h < CQ; ++h) {
             uint32_t r[32];
             float4 w4[8];
             tmem_ld32(lane_addr + b * BN + 32 * h, r);
 #pragma unroll
             for (int q = 0; q < 8; ++q) w4[q] = lds128(wsc + 32 * h + 4 * q);
             tmem_wait_ld();
-            if (h == 1) {
+            if (h == CQ - 1) {
               // the whole group is in registers: release the accumulator for the group NACC ahead
               tc_fence_before();
               __syncwarp();
@@ -481,20 +513,23 @@ __global__ void __launch_bounds__(THREADS, 1) w4a4_kernel(const __grid_constant_
             }
           }
         } else {
-          uint32_t r0[32], r1[32];
-          tmem_ld32(lane_addr + b * BN, r0);
-          tmem_ld32(lane_addr + b * BN + 32, r1);
-          tmem_wait_ld();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&tempty[b]);
-          if (row_ok) {
-            const int g = w.g0 + gl;
+          const int g = w.g0 + gl;
+#pragma unroll 1
+          for (int h = 0; h < CQ; ++h) {
+            uint32_t r[32];
+            tmem_ld32(lane_addr + b * BN + 32 * h, r);
+            tmem_wait_ld();
+            if (h == CQ - 1) {
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(&tempty[b]);
+            }
+            if (row_ok) {
 #pragma unroll
-            for (int j = 0; j < 64; ++j) {
-              const int n = w.n0 + wg * EPI_COLS + j;
-              const uint32_t v = j < 32 ? r0[j] : r1[j - 32];
-              if (n < p.N) p.P[((int64_t)m * p.N + n) * NG + g] = ((int32_t)v) / (int32_t)L::UNIT;
+              for (int j = 0; j < 32; ++j) {
+                const int n = w.n0 + wg * EPI_COLS + 32 * h + j;
+                if (n < p.N) p.P[((int64_t)m * p.N + n) * NG + g] = ((int32_t)r[j]) / (int32_t)L::UNIT;
+              }
             }
           }
         }
@@ -576,6 +611,7 @@ __global__ void __launch_bounds__(THREADS, 1) w4a4_kernel(const __grid_constant_
     const int c = ut & 3, r0 = ut >> 2, r7 = r0 & 7;
     const int lo_off = ((2 * c) ^ r7) << 4, hi_off = ((2 * c + 1) ^ r7) << 4;
     constexpr int UNP_ITERS = L::UNP_ITERS;
+    constexpr int UNP_BATCH = 4;
     const bool tail = ut + N_UNP * (UNP_ITERS - 1) < L::N_CHUNKS;   // this thread has a last chunk
     int it = 0;
     bool ok = true;
@@ -590,18 +626,24 @@ __global__ void __launch_bounds__(THREADS, 1) w4a4_kernel(const __grid_constant_
         }
         const uint8_t* src = smem + L::OFF_PSTAGES + ps * L::PSTAGE + L::SRC_OFF + ut * 16;
         uint8_t* dst = smem + L::OFF_STAGES + s * L::STAGE + r0 * 128;
-        // all loads first, then the stores: the shared-memory latency is paid once per stage
-        uint4 v[UNP_ITERS];
+        // loads in batches of UNP_BATCH, then their stores: the shared-memory latency is paid
+        // once per batch (a batch's loads fit the role's register budget)
 #pragma unroll
-        for (int i = 0; i < UNP_ITERS; ++i)
-          if (i < UNP_ITERS - 1 || tail) v[i] = *reinterpret_cast<const uint4*>(src + i * N_UNP * 16);
+        for (int i0 = 0; i0 < UNP_ITERS; i0 += UNP_BATCH) {
+        uint4 v[UNP_BATCH];
 #pragma unroll
-        for (int i = 0; i < UNP_ITERS; ++i) {
-          if (i < UNP_ITERS - 1 || tail) {
-            const uint4 lo = make_uint4((v[i].x << 4) & 0xF0F0F0F0u, (v[i].y << 4) & 0xF0F0F0F0u,
-                                        (v[i].z << 4) & 0xF0F0F0F0u, (v[i].w << 4) & 0xF0F0F0F0u);
-            const uint4 hi = make_uint4(v[i].x & 0xF0F0F0F0u, v[i].y & 0xF0F0F0F0u, v[i].z & 0xF0F0F0F0u,
-                                        v[i].w & 0xF0F0F0F0u);
+        for (int i1 = 0; i1 < UNP_BATCH; ++i1) {
+          const int i = i0 + i1;
+          if (i < UNP_ITERS - 1 || (i == UNP_ITERS - 1 && tail)) v[i1] = *reinterpret_cast<const uint4*>(src + i * N_UNP * 16);
+        }
+#pragma unroll
+        for (int i1 = 0; i1 < UNP_BATCH; ++i1) {
+          const int i = i0 + i1;
+          if (i < UNP_ITERS - 1 || (i == UNP_ITERS - 1 && tail)) {
+            const uint4 lo = make_uint4((v[i1].x << 4) & 0xF0F0F0F0u, (v[i1].y << 4) & 0xF0F0F0F0u,
+                                        (v[i1].z << 4) & 0xF0F0F0F0u, (v[i1].w << 4) & 0xF0F0F0F0u);
+            const uint4 hi = make_uint4(v[i1].x & 0xF0F0F0F0u, v[i1].y & 0xF0F0F0F0u, v[i1].z & 0xF0F0F0F0u,
+                                        v[i1].w & 0xF0F0F0F0u);
             uint8_t* rowp = dst + i * (N_UNP / 4) * 128;
             if constexpr (A8) {
               // natural K order (the int8 A tile is not permuted): interleave even / odd codes
@@ -617,6 +659,7 @@ __global__ void __launch_bounds__(THREADS, 1) w4a4_kernel(const __grid_constant_
               *reinterpret_cast<uint4*>(rowp + hi_off) = hi;
             }
           }
+        }
         }
         fence_proxy_async();
         __syncwarp();
@@ -651,9 +694,51 @@ __global__ void __launch_bounds__(THREADS, 1) w4a4_kernel(const __grid_constant_
           break;
         }
         tc_fence_after();
-        const int nk = min(4, w.ks - 4 * j);
         const uint64_t soA = (uint64_t)(((A8 ? ps * L::PSTAGE : s * L::STAGE)) >> 4);
         const uint64_t soB = (uint64_t)((s * L::STAGE) >> 4);
+        if (gsteps % 4 == 0) {
+          // G a multiple of 128: the K-block lies inside one group (and K % 128 == 0, so it has
+          // all 4 k-steps). The accumulator wait comes first (warp-wide), then one elected lane
+          // issues the 4 MMAs and the commits back to back (no per-MMA branches or elections).
+          if (kg == 0) {
+            if (!bar_wait(&tempty[b], tph, abort_flag, p.wait_ns)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+          }
+          const bool last = kg + 4 == gsteps;
+          if (elect_one()) {
+            const uint32_t td = tmem + b * BN;
+            umma_i8_one(td, dA0 + soA, dB0 + soB, kg != 0 ? 1u : 0u);
+            umma_i8_one(td, dA0 + soA + 2, dB0 + soB + 2, 1u);
+            umma_i8_one(td, dA0 + soA + 4, dB0 + soB + 4, 1u);
+            umma_i8_one(td, dA0 + soA + 6, dB0 + soB + 6, 1u);
+            if (last) umma_commit_one(&tfull[b]);
+            umma_commit_one(&empty[s]);
+            if (A8) umma_commit_one(&pempty[ps]);
+          }
+          __syncwarp();
+          kg += 4;
+          if (last) {
+            kg = 0;
+            if (++b == NACC) {
+              b = 0;
+              tph ^= 1;
+            }
+          }
+          ++nblk;
+          if (++s == STAGES) {
+            s = 0;
+            sph ^= 1;
+          }
+          if (++ps == PSTAGES) {
+            ps = 0;
+            pph ^= 1;
+          }
+          continue;
+        }
+        const int nk = min(4, w.ks - 4 * j);
 #pragma unroll
         for (int k4 = 0; k4 < 4; ++k4) {
           if (k4 < nk) {
