@@ -38,6 +38,8 @@ struct Stage {
   bool identity = false;
   bool hadamard = false;  // blocks equal H_b / sqrt(b) (power-of-two b)
   float* d_blocks = nullptr;   // [n_blocks, b, b] fp32 row-major (base mixer materialised)
+  float* d_blocks_pad = nullptr;  // per-block stages of radix 3..48: [n_blocks, b, bp] rows padded
+                                  // to bp = a multiple of 4 floats (zeros), for 16-byte loads
   int32_t* d_perm = nullptr;   // gather after the stage, or nullptr
   int32_t* d_iperm = nullptr;  // inverse permutation (for T^T)
 };

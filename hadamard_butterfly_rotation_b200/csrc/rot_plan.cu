@@ -77,6 +77,7 @@ static void free_plan_memory(rot_plan_s* p) {
   if (p->d_signmask) cudaFree(p->d_signmask);
   for (auto& s : p->stages) {
     if (s.d_blocks) cudaFree(s.d_blocks);
+    if (s.d_blocks_pad) cudaFree(s.d_blocks_pad);
     if (s.d_perm) cudaFree(s.d_perm);
     if (s.d_iperm) cudaFree(s.d_iperm);
   }
@@ -171,6 +172,21 @@ extern "C" rot_status rot_plan_create(rot_plan_t* out, int K, int n_stages, cons
         return set_error(ROT_ENOMEM, "rot_plan_create: cudaMalloc(blocks)");
       }
       cudaMemcpy(st.d_blocks, host.data(), bytes, cudaMemcpyHostToDevice);
+      if (st.n_blocks > 1 && b > 2 && b <= 48) {
+        // padded copy for the multi-row kernel's per-block dense stages
+        const int bp = (b + 3) & ~3;
+        std::vector<float> pad((size_t)st.n_blocks * b * bp, 0.0f);
+        for (int64_t c = 0; c < st.n_blocks; ++c)
+          for (int r = 0; r < b; ++r)
+            for (int k = 0; k < b; ++k) pad[((size_t)c * b + r) * bp + k] = host[((size_t)c * b + r) * b + k];
+        if (cudaMalloc(&st.d_blocks_pad, pad.size() * sizeof(float)) != cudaSuccess) {
+          cudaFree(st.d_blocks);
+          free_plan_memory(p);
+          delete p;
+          return set_error(ROT_ENOMEM, "rot_plan_create: cudaMalloc(padded blocks)");
+        }
+        cudaMemcpy(st.d_blocks_pad, pad.data(), pad.size() * sizeof(float), cudaMemcpyHostToDevice);
+      }
     }
     if (perms && perms[t]) {
       std::vector<int32_t> seen(K, 0), inv(K);

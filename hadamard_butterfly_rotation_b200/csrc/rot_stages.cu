@@ -13,6 +13,7 @@
 // The inverse T^T runs the stages in reverse order with transposed blocks and inverse
 // permutations, and applies the signs last.
 #include <cstdlib>
+#include <type_traits>
 
 #include "rot_internal.cuh"
 
@@ -166,9 +167,10 @@ __global__ void __launch_bounds__(THREADS) stages_kernel(const Args a) {
 // Forward rotation (+ quantisation) of ROWS rows at a time per CTA, so that every stage
 // parameter read from L2 serves ROWS rows. Stages:
 //   radix 2:  in place, one thread per 2 x 2 block (per-block or shared parameters);
-//   radix b:  (3 <= b <= MR_MAXB, one shared block kept in shared memory) each work item
-//             holds the b inputs of one block in registers and produces a range of outputs,
-//             written back in place after a barrier;
+//   radix b:  (3 <= b <= MR_MAXB) each work item holds the b inputs of one block in registers
+//             and produces a range of outputs, written back in place after a barrier; a shared
+//             block is kept in shared memory (read as broadcasts), per-block blocks are read
+//             from a copy with rows padded to a multiple of 4 floats (16-byte loads, L2/L1);
 //   gather:   x''[j] = x'[P[j]] into the second buffer.
 // The block index c = low + high * s of coordinate base = low + high * b * s uses a
 // multiply-high division by s (exact for c < 2^16).
@@ -179,12 +181,13 @@ constexpr int MR_UB = 12;          // 2 x 2 blocks per thread per batch (K/2 <= 
 constexpr int MR_UG = 24;          // gather indices per thread per batch (K <= 12288: one batch)
 
 struct MrStage {
-  const float* blocks;   // radix 2: [n_blocks][4]; radix b: [b][b] (shared)
+  const float* blocks;   // radix 2: [n_blocks][4]; radix b: [b][b] (shared) or [n_blocks][b][bp] (padded)
   const int32_t* perm;   // gather after the stage or nullptr
   const int32_t* iperm;  // its inverse: a non-identity stage scatters output j to iperm[j]
   int b, stride;
   uint32_t magic;        // ceil(2^32 / stride) for stride >= 2 (stride 1 divides trivially)
   int per_block, identity;
+  int sh_off;            // radix b > 2, shared block: its offset (floats) in the shared-memory block area
 };
 
 struct MrArgs {
@@ -195,8 +198,7 @@ struct MrArgs {
   const float* signs;
   int n_stages;
   MrStage st[MAX_STAGES];
-  int dense_b;           // radix of the dense stage (0: none)
-  const float* dense_block;
+  int sh_floats;         // shared-memory block area (floats): the shared dense blocks, rows padded
   float* Y;
   int64_t ldy;
   uint8_t* codes;
@@ -204,17 +206,24 @@ struct MrArgs {
   int G, bits;
 };
 
+// PB: the plan has per-block dense stages (a separate instance, so that plans without them run
+// the shared-block code alone)
+template <bool PB>
 __global__ void __launch_bounds__(MR_THREADS, 1) stages_rows_kernel(const MrArgs a) {
   extern __shared__ __align__(16) float smem[];
   const int K = a.K;
   float* bufA = smem;                          // [MR_ROWS][K]
   float* bufB = smem + MR_ROWS * K;            // [MR_ROWS][K]
-  float* sblk = smem + 2 * MR_ROWS * K;        // dense block, rows padded to a multiple of 4
-  const int bp = (a.dense_b + 3) & ~3;
-  for (int i = threadIdx.x; i < a.dense_b * a.dense_b; i += MR_THREADS)
-    sblk[(i / a.dense_b) * bp + (i % a.dense_b)] = a.dense_block[i];
-  for (int i = threadIdx.x; i < a.dense_b * bp; i += MR_THREADS)
-    if (i % bp >= a.dense_b) sblk[i] = 0.0f;
+  float* sblk = smem + 2 * MR_ROWS * K;        // shared dense blocks, rows padded to a multiple of 4
+  for (int t = 0; t < a.n_stages; ++t) {
+    const MrStage& S = a.st[t];
+    if (S.identity || S.b == 2 || S.per_block) continue;
+    const int b = S.b, bp = (b + 3) & ~3;
+    for (int i = threadIdx.x; i < b * bp; i += MR_THREADS) {
+      const int r = i / bp, k = i - r * bp;
+      sblk[S.sh_off + i] = k < b ? S.blocks[r * b + k] : 0.0f;
+    }
+  }
 
   for (int64_t row0 = (int64_t)blockIdx.x * MR_ROWS; row0 < a.M; row0 += (int64_t)gridDim.x * MR_ROWS) {
     const int nr = (int)(a.M - row0 < MR_ROWS ? a.M - row0 : MR_ROWS);
@@ -286,7 +295,7 @@ __global__ void __launch_bounds__(MR_THREADS, 1) stages_rows_kernel(const MrArgs
           // warp (warps alternate halves), so every shared-memory load of a block row is one
           // broadcast; both halves of a block lie in the same pass (a pass covers 32-block
           // groups times 2 halves), so the in-place writes are safe.
-          const int b = S.b, nb = K / b;
+          const int b = S.b, nb = K / b, bp = (b + 3) & ~3;
           const int nb32 = (nb + 31) & ~31;
           for (int r = 0; r < MR_ROWS; ++r) {
             float* x = cur + r * K;
@@ -305,21 +314,35 @@ __global__ void __launch_bounds__(MR_THREADS, 1) stages_rows_kernel(const MrArgs
               __syncthreads();   // every input of this pass is in registers before any write
               if (on) {
                 const int r0 = h ? (b + 1) / 2 : 0, r1 = h ? b : (b + 1) / 2;
-                for (int o = r0; o < r1; ++o) {
-                  const float4* brow = reinterpret_cast<const float4*>(sblk + o * bp);
-                  float a0 = 0.0f, a1 = 0.0f, a2 = 0.0f, a3 = 0.0f;   // four independent chains
+                // the output rows of this item's block: shared (block rows in shared memory, the
+                // loads broadcasts) or per block (the padded copy, read through L1/L2); the two
+                // forms are separate loops so that the shared one keeps shared-memory loads
+                auto outputs = [&](auto per_block) {
+                  for (int o = r0; o < r1; ++o) {
+                    float a0 = 0.0f, a1 = 0.0f, a2 = 0.0f, a3 = 0.0f;   // four independent chains
 #pragma unroll
-                  for (int k4 = 0; k4 < MR_MAXB / 4; ++k4) {
-                    if (4 * k4 < b) {
-                      const float4 w = brow[k4];
-                      a0 = fmaf(w.x, in[4 * k4], a0);
-                      a1 = fmaf(w.y, in[4 * k4 + 1], a1);
-                      a2 = fmaf(w.z, in[4 * k4 + 2], a2);
-                      a3 = fmaf(w.w, in[4 * k4 + 3], a3);
+                    for (int k4 = 0; k4 < MR_MAXB / 4; ++k4) {
+                      if (4 * k4 < b) {
+                        float4 w;
+                        if constexpr (decltype(per_block)::value)
+                          w = __ldg(reinterpret_cast<const float4*>(S.blocks + ((size_t)c * b + o) * bp) + k4);
+                        else
+                          w = reinterpret_cast<const float4*>(sblk + S.sh_off + o * bp)[k4];
+                        a0 = fmaf(w.x, in[4 * k4], a0);
+                        a1 = fmaf(w.y, in[4 * k4 + 1], a1);
+                        a2 = fmaf(w.z, in[4 * k4 + 2], a2);
+                        a3 = fmaf(w.w, in[4 * k4 + 3], a3);
+                      }
                     }
+                    const int oi = base + o * st;
+                    dst[r * K + (scat ? __ldg(S.iperm + oi) : oi)] = (a0 + a1) + (a2 + a3);
                   }
-                  const int oi = base + o * st;
-                  dst[r * K + (scat ? __ldg(S.iperm + oi) : oi)] = (a0 + a1) + (a2 + a3);
+                };
+                if constexpr (PB) {
+                  if (S.per_block) outputs(std::true_type{});
+                  else outputs(std::false_type{});
+                } else {
+                  outputs(std::false_type{});
                 }
               }
               __syncthreads();
@@ -400,19 +423,21 @@ __global__ void __launch_bounds__(MR_THREADS, 1) stages_rows_kernel(const MrArgs
   }
 }
 
-// The multi-row kernel applies to forward plans whose non-identity stages are radix 2 or one
-// shared dense block of radix 3..MR_MAXB, with K < 2^16 and the two row buffers in shared memory.
+// The multi-row kernel applies to forward plans whose non-identity stages are radix 2 or dense
+// of radix 3..MR_MAXB (shared blocks in shared memory, per-block blocks from their padded copy),
+// with K < 2^16 and the two row buffers in shared memory.
 bool rows_kernel_fits(const rot_plan_s* p, int inverse, size_t* smem_out) {
   if (inverse || p->K >= 65536 || (p->K & 3) || (int)p->stages.size() > MAX_STAGES) return false;
-  int dense = 0;
+  size_t sh = 0;
   for (const Stage& S : p->stages) {
     if (S.identity) continue;
     if (S.b == 2) continue;
-    if (S.b > MR_MAXB || S.n_blocks != 1 || dense) return false;
-    dense = S.b;
+    if (S.b > MR_MAXB) return false;
+    // per-block blocks of small radix: the generic kernel (one row per CTA) is faster
+    if (S.n_blocks != 1 && (!S.d_blocks_pad || S.b < 16)) return false;
+    if (S.n_blocks == 1) sh += (size_t)S.b * ((S.b + 3) & ~3);
   }
-  const int bp = (dense + 3) & ~3;
-  const size_t smem = (size_t)2 * MR_ROWS * p->K * sizeof(float) + (size_t)dense * bp * sizeof(float);
+  const size_t smem = (size_t)2 * MR_ROWS * p->K * sizeof(float) + sh * sizeof(float);
   if (smem > 227 * 1024) return false;
   *smem_out = smem;
   return true;
@@ -438,9 +463,14 @@ rot_status launch_rows(const rot_plan_s* p, const Args& a0, size_t smem, cudaStr
     d.magic = S.stride > 1 ? (uint32_t)(((1ull << 32) + (uint64_t)S.stride - 1) / (uint64_t)S.stride) : 0u;
     d.per_block = S.n_blocks > 1;
     d.identity = S.identity;
+    d.sh_off = 0;
     if (!S.identity && S.b > 2) {
-      a.dense_b = S.b;
-      a.dense_block = S.d_blocks;
+      if (d.per_block) {
+        d.blocks = S.d_blocks_pad;
+      } else {
+        d.sh_off = a.sh_floats;
+        a.sh_floats += S.b * ((S.b + 3) & ~3);
+      }
     }
   }
   a.Y = a0.Y;
@@ -449,17 +479,21 @@ rot_status launch_rows(const rot_plan_s* p, const Args& a0, size_t smem, cudaStr
   a.scales = a0.scales;
   a.G = a0.G;
   a.bits = a0.bits;
-  static int configured[64] = {0};
+  bool pb = false;
+  for (int t = 0; t < a.n_stages; ++t) pb = pb || (!a.st[t].identity && a.st[t].b > 2 && a.st[t].per_block);
+  static int configured[64][2] = {};
   int dev = 0;
   cudaGetDevice(&dev);
-  if (dev < 64 && !configured[dev]) {
-    ROT_CUDA_TRY(cudaFuncSetAttribute(stages_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024));
-    configured[dev] = 1;
+  if (dev < 64 && !configured[dev][pb]) {
+    ROT_CUDA_TRY(cudaFuncSetAttribute(pb ? stages_rows_kernel<true> : stages_rows_kernel<false>,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024));
+    configured[dev][pb] = 1;
   }
   if (a.M == 0) return ROT_OK;
   const int64_t units = (a.M + MR_ROWS - 1) / MR_ROWS;
   const int64_t grid = std::min<int64_t>(units, (int64_t)sm_count());
-  stages_rows_kernel<<<(unsigned)grid, MR_THREADS, smem, s>>>(a);
+  if (pb) stages_rows_kernel<true><<<(unsigned)grid, MR_THREADS, smem, s>>>(a);
+  else stages_rows_kernel<false><<<(unsigned)grid, MR_THREADS, smem, s>>>(a);
   ROT_CUDA_TRY(cudaGetLastError());
   return ROT_OK;
 }
