@@ -13,7 +13,6 @@
 // The inverse T^T runs the stages in reverse order with transposed blocks and inverse
 // permutations, and applies the signs last.
 #include <cstdlib>
-#include <type_traits>
 
 #include "rot_internal.cuh"
 
@@ -297,6 +296,8 @@ __global__ void __launch_bounds__(MR_THREADS, 1) stages_rows_kernel(const MrArgs
           // groups times 2 halves), so the in-place writes are safe.
           const int b = S.b, nb = K / b, bp = (b + 3) & ~3;
           const int nb32 = (nb + 31) & ~31;
+          const float* sbl = sblk + S.sh_off;   // shared block (rows padded to bp floats)
+          const float* pbk = S.blocks;          // per-block: the padded copy
           for (int r = 0; r < MR_ROWS; ++r) {
             float* x = cur + r * K;
             for (int item0 = 0; item0 < 2 * nb32; item0 += MR_THREADS) {
@@ -314,20 +315,15 @@ __global__ void __launch_bounds__(MR_THREADS, 1) stages_rows_kernel(const MrArgs
               __syncthreads();   // every input of this pass is in registers before any write
               if (on) {
                 const int r0 = h ? (b + 1) / 2 : 0, r1 = h ? b : (b + 1) / 2;
-                // the output rows of this item's block: shared (block rows in shared memory, the
-                // loads broadcasts) or per block (the padded copy, read through L1/L2); the two
-                // forms are separate loops so that the shared one keeps shared-memory loads
-                auto outputs = [&](auto per_block) {
+                if (PB && S.per_block) {
+                  // per-block blocks: the padded copy, read through L1/L2
                   for (int o = r0; o < r1; ++o) {
+                    const float4* brow = reinterpret_cast<const float4*>(pbk + ((size_t)c * b + o) * bp);
                     float a0 = 0.0f, a1 = 0.0f, a2 = 0.0f, a3 = 0.0f;   // four independent chains
 #pragma unroll
                     for (int k4 = 0; k4 < MR_MAXB / 4; ++k4) {
                       if (4 * k4 < b) {
-                        float4 w;
-                        if constexpr (decltype(per_block)::value)
-                          w = __ldg(reinterpret_cast<const float4*>(S.blocks + ((size_t)c * b + o) * bp) + k4);
-                        else
-                          w = reinterpret_cast<const float4*>(sblk + S.sh_off + o * bp)[k4];
+                        const float4 w = __ldg(brow + k4);
                         a0 = fmaf(w.x, in[4 * k4], a0);
                         a1 = fmaf(w.y, in[4 * k4 + 1], a1);
                         a2 = fmaf(w.z, in[4 * k4 + 2], a2);
@@ -337,12 +333,24 @@ __global__ void __launch_bounds__(MR_THREADS, 1) stages_rows_kernel(const MrArgs
                     const int oi = base + o * st;
                     dst[r * K + (scat ? __ldg(S.iperm + oi) : oi)] = (a0 + a1) + (a2 + a3);
                   }
-                };
-                if constexpr (PB) {
-                  if (S.per_block) outputs(std::true_type{});
-                  else outputs(std::false_type{});
                 } else {
-                  outputs(std::false_type{});
+                  // one shared block: its rows in shared memory, every load a broadcast
+                  for (int o = r0; o < r1; ++o) {
+                    const float4* brow = reinterpret_cast<const float4*>(sbl + o * bp);
+                    float a0 = 0.0f, a1 = 0.0f, a2 = 0.0f, a3 = 0.0f;   // four independent chains
+#pragma unroll
+                    for (int k4 = 0; k4 < MR_MAXB / 4; ++k4) {
+                      if (4 * k4 < b) {
+                        const float4 w = brow[k4];
+                        a0 = fmaf(w.x, in[4 * k4], a0);
+                        a1 = fmaf(w.y, in[4 * k4 + 1], a1);
+                        a2 = fmaf(w.z, in[4 * k4 + 2], a2);
+                        a3 = fmaf(w.w, in[4 * k4 + 3], a3);
+                      }
+                    }
+                    const int oi = base + o * st;
+                    dst[r * K + (scat ? __ldg(S.iperm + oi) : oi)] = (a0 + a1) + (a2 + a3);
+                  }
                 }
               }
               __syncthreads();
