@@ -23,12 +23,14 @@
  *   - Calls that take a stream are asynchronous on that stream (a cudaStream_t passed as
  *     void*, NULL = legacy default stream) and never synchronise; argument errors are
  *     detected on the host and returned before any launch.
- *   - The fused rotation kernels (rot_apply / rot_quant on RHT-type plans) are launched
- *     with programmatic dependent launch: their prologue (barrier set-up, copying the
- *     plan's sign table) may overlap the tail of the previous kernel in the stream, and
- *     every access to A and to the outputs waits for that kernel to complete. Setting
- *     ROT_B200_PDL=0 in the environment launches them normally. Stream capture into CUDA
- *     graphs is supported (the dependency becomes a programmatic graph edge).
+ *   - The fused rotation kernels (rot_apply / rot_quant on RHT-type plans) and the linear
+ *     kernels are launched with programmatic dependent launch: their prologue (barrier
+ *     set-up, copying the plan's sign table, TMEM allocation, an L2 prefetch of the weight
+ *     rows) may overlap the tail of the previous kernel in the stream, and every other
+ *     global access waits for that kernel to complete (an L2 prefetch is safe: L2 is the
+ *     device's point of coherence). Setting ROT_B200_PDL=0 in the environment launches them
+ *     normally. Stream capture into CUDA graphs is supported (the dependency becomes a
+ *     programmatic graph edge).
  *   - Device pointers must be 16-byte aligned; leading dimensions are in elements and
  *     lda * sizeof(element) must be a multiple of 16 bytes.
  *   - Layouts (row-major):
@@ -126,8 +128,8 @@ rot_status rot_dequant(const uint8_t* codes, const uint16_t* scales, int64_t M, 
  * C:  [M, N] fp32 (c_dtype = ROT_F32) or bf16 (ROT_BF16), row-major, ldc = N.
  * Requires K % G == 0, G % 32 == 0, K % 64 == 0, N % 16 == 0; M >= 0 arbitrary.
  * Decode-sized M (M <= 64 with G % 128 == 0) runs a weight-streaming kernel (mma.sync int8 per 8
- * weight rows; each CTA streams its rows' K-slices into shared memory with bulk copies and sums the
- * slices itself, so C is written directly). Other shapes run a persistent tcgen05 kernel over 128 x 128
+ * weight rows; each CTA streams its rows into shared memory with bulk copies -- for M <= 16 also the
+ * activation rows and the scale rows -- and sums its K-slices itself, so C is written directly). Other shapes run a persistent tcgen05 kernel over 128 x 128
  * output tiles, and shapes whose tiles leave most SMs idle split K into ranges aligned to
  * lcm(G, 128); their partial results are added with fp32 atomics: C is zeroed on the stream first
  * (fp32 output), or, for bf16 output, a stream-ordered temporary of M * N floats is allocated
