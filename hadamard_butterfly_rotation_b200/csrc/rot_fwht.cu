@@ -820,6 +820,93 @@ __global__ void __launch_bounds__(MMA_THREADS, 1) fwht_mma_kernel(const Args a) 
   }
 }
 
+// Few-row kernel for 4096-coordinate chunks (bf16 in, quantised out): one CTA of 256 threads per
+// chunk, 16 values per thread, so a handful of rows (decode) is spread over many SMs instead of one
+// warp per row. The chunk lives in shared memory between three radix-16 passes:
+//   pass 0  thread t holds coordinates 16 t + j (loaded from HBM): butterflies over bits 0..3;
+//   pass 1  thread t holds (t & 15) + 16 j + 256 (t >> 4): bits 4..7;
+//   pass 2  thread t holds t + 256 j: bits 8..11;
+// then thread t reads 16 t + j again and quantises as the other kernels do. Float i is stored at
+// i + (i >> 4) (one pad per 16): every pass's accesses of a warp fall in distinct banks (pass 2:
+// one two-way pair).
+constexpr int SMALL_THREADS = 256;
+constexpr int SMALL_N = 4096;
+constexpr int SMALL_SMEM = (SMALL_N + SMALL_N / 16) * 4;
+
+__device__ __forceinline__ int small_pad(int i) { return i + (i >> 4); }
+
+// 16-point Walsh-Hadamard butterflies on the 16 values of a thread (pairs: bit 0 inside a pair)
+__device__ __forceinline__ void fwht16(float2 (&xp)[8]) {
+#pragma unroll
+  for (int i = 0; i < 8; ++i) xp[i] = make_float2(xp[i].x + xp[i].y, xp[i].x - xp[i].y);
+#pragma unroll
+  for (int b = 0; b < 3; ++b) stage_pairs<8>(xp, b);
+}
+
+template <int BITS, int GT>
+__global__ void __launch_bounds__(SMALL_THREADS) fwht_small_kernel(const Args a) {
+  extern __shared__ __align__(16) float sfl[];
+  const int t = threadIdx.x;
+  const int64_t u = blockIdx.x;               // chunk `chunk` of row `row`
+  const int64_t row = u / a.chunks;
+  const int chunk = (int)(u - row * a.chunks);
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  float2 xp[8];
+  {
+    // 16 bf16 values (two 16-byte loads), signs XORed into the pairs, widened to fp32
+    const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(a.A) +
+                                                      ((int64_t)row * a.lda + (int64_t)chunk * SMALL_N + 16 * t) * 2);
+    const uint4 v0 = src[0], v1 = src[1];
+    uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+    if (a.signmask) {
+      const uint4* sm = reinterpret_cast<const uint4*>(a.signmask + (chunk * SMALL_N + 16 * t) / 2);
+      const uint4 m0 = sm[0], m1 = sm[1];
+      const uint32_t m[8] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
+#pragma unroll
+      for (int i = 0; i < 8; ++i) w[i] ^= m[i];
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) xp[i] = make_float2(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xffff0000u));
+  }
+  // pass 0: bits 0..3
+  fwht16(xp);
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    sfl[small_pad(16 * t + 2 * j)] = xp[j].x;
+    sfl[small_pad(16 * t + 2 * j + 1)] = xp[j].y;
+  }
+  __syncthreads();
+  // pass 1: bits 4..7
+  const int b1 = (t & 15) + 256 * (t >> 4);
+#pragma unroll
+  for (int j = 0; j < 8; ++j) xp[j] = make_float2(sfl[small_pad(b1 + 32 * j)], sfl[small_pad(b1 + 32 * j + 16)]);
+  fwht16(xp);
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    sfl[small_pad(b1 + 32 * j)] = xp[j].x;
+    sfl[small_pad(b1 + 32 * j + 16)] = xp[j].y;
+  }
+  __syncthreads();
+  // pass 2: bits 8..11
+#pragma unroll
+  for (int j = 0; j < 8; ++j) xp[j] = make_float2(sfl[small_pad(t + 512 * j)], sfl[small_pad(t + 512 * j + 256)]);
+  fwht16(xp);
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    sfl[small_pad(t + 512 * j)] = xp[j].x;
+    sfl[small_pad(t + 512 * j + 256)] = xp[j].y;
+  }
+  __syncthreads();
+  // contiguous again: quantise coordinates 16 t .. 16 t + 15 of the chunk
+#pragma unroll
+  for (int j = 0; j < 8; ++j) xp[j] = make_float2(sfl[small_pad(16 * t + 2 * j)], sfl[small_pad(16 * t + 2 * j + 1)]);
+  constexpr int CPW = 32 / BITS;
+  const int c0 = chunk * SMALL_N + 16 * t;                 // coordinate within the row
+  uint32_t* dst = reinterpret_cast<uint32_t*>(a.codes + row * (int64_t)(a.K / CPW) * 4) + c0 / CPW;
+  quantise_store_at<BITS, GT, 16, SMALL_THREADS>(a, xp, a.scales + row * a.ngroups, dst, c0, t);
+}
+
 size_t mma_smem_bytes(int K) {
   return 256 + (size_t)MMA_SLOTS * MMA_SSTRIDE * 4 + (size_t)MMA_BARS * 8 + (size_t)(K / 2) * 4;
 }
@@ -920,8 +1007,49 @@ rot_status launch_mma(const Args& a, cudaStream_t s) {
   return ROT_OK;
 }
 
+// Few rows of 4096-coordinate chunks: one CTA per chunk (ROT_B200_SMALL=0 / 1 in the environment
+// turns the choice off / on for every row count; by default up to SMALL_MAX_UNITS chunks).
+constexpr int64_t SMALL_MAX_UNITS = 512;
+int small_mode() {
+  static const int mode = [] {
+    const char* e = std::getenv("ROT_B200_SMALL");
+    return e ? (e[0] == '0' ? 0 : 1) : -1;
+  }();
+  return mode;
+}
+
+template <int BITS, int GT>
+rot_status launch_small(const Args& a, cudaStream_t s) {
+  const int64_t units = a.M * a.chunks;
+  if (units < 1) return ROT_OK;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)units);
+  cfg.blockDim = dim3(SMALL_THREADS);
+  cfg.dynamicSmemBytes = SMALL_SMEM;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl_default() ? 1 : 0;
+  ROT_CUDA_TRY(cudaLaunchKernelEx(&cfg, fwht_small_kernel<BITS, GT>, a));
+  return ROT_OK;
+}
+
 template <int LOGN, bool BF16, int MODE, int BITS>
 rot_status launch_g(const Args& a, cudaStream_t s) {
+  if constexpr (MODE == MODE_QUANT && BF16 && LOGN == 12) {
+    const int sm = small_mode();
+    // 16-byte row loads (lda a multiple of 8 elements, 16-byte aligned A) and G <= 512 (a group
+    // spans at most one warp of 16-value threads)
+    const bool fits = (a.lda % 8) == 0 && (reinterpret_cast<uintptr_t>(a.A) & 15) == 0 && a.G <= 512 && a.G >= 8;
+    if (fits && (sm == 1 || (sm == -1 && a.M * a.chunks <= SMALL_MAX_UNITS))) {
+      if (a.G == 32) return launch_small<BITS, 32>(a, s);
+      if (a.G == 64) return launch_small<BITS, 64>(a, s);
+      if (a.G == 128) return launch_small<BITS, 128>(a, s);
+      return launch_small<BITS, 0>(a, s);
+    }
+  }
   if constexpr (MODE == MODE_QUANT && BF16 && LOGN == 11) {
     if (tc_enabled() && mma_smem_bytes(a.K) <= 227 * 1024) {
       if (a.G == 32) return launch_mma<BITS, 32>(a, s);

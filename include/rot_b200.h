@@ -264,7 +264,10 @@ rot_status rot_check_device(void);
  *   fault = 0  no fault (only sets the bound)
  *   fault = 1  ROT_TEST_ROTATION_COPY: the next rot_quant / rot_apply launch of the fused
  *              rotation kernel does not issue the first staging copy of CTA 0's first slot;
- *              that slot's waits run out, every other slot completes normally
+ *              that slot's waits run out, every other slot completes normally (the few-row
+ *              kernel for 4096-coordinate chunks -- at most 512 chunks, bf16 in, quantised
+ *              out -- stages nothing and waits on nothing: the fault is consumed and has no
+ *              effect there)
  *   fault = 2  ROT_TEST_W4A4_LOADS: the next launch of the W4A4 tile kernel (M > 64 or
  *              G % 128 != 0) issues no TMA load; every role's waits run out
  * The fault is one-shot (consumed by the next launch of that kernel family on any thread).

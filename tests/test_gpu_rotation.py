@@ -47,8 +47,8 @@ def test_rht_apply_ragged_rows_and_stride(lib, M):
 
 @pytest.mark.parametrize("K,G,bits", [(32, 8, 4), (64, 16, 2), (128, 32, 4), (256, 128, 4), (256, 64, 2),
                                       (512, 256, 4), (1024, 32, 4), (2048, 32, 4), (2048, 128, 4),
-                                      (2048, 2048, 4), (4096, 128, 4), (4096, 64, 2), (8192, 128, 4),
-                                      (8192, 64, 2), (8192, 16, 2)])
+                                      (2048, 2048, 4), (4096, 128, 4), (4096, 64, 2), (4096, 256, 4),
+                                      (4096, 16, 2), (4096, 32, 4), (8192, 128, 4), (8192, 64, 2), (8192, 16, 2)])
 def test_rht_quant(lib, K, G, bits):
     A, s = _acts(67, K, K + G + bits)
     plan = lib.Plan.rht(K, s)
@@ -60,6 +60,21 @@ def test_rht_quant(lib, K, G, bits):
     cflag, gflag = Q.boundary_flags(y, bits, G)
     assert (cflag & ~np.repeat(gflag, G, axis=1)).sum() < 1e-3 * A.size
     assert gflag.sum() <= max(6, 0.06 * gflag.size)
+
+
+@pytest.mark.parametrize("G", [32, 128, 512])
+@pytest.mark.parametrize("M", [1, 7, 600])
+def test_rht_quant_k4096_strided_few_rows(lib, M, G):
+    """K = 4096 bf16 int4 with few rows (one CTA per row) and past the few-row limit of 512 chunks
+    (the one-warp-per-row kernel): rows with a pitch of K + 64 elements, every row against the oracle."""
+    import torch
+    K = 4096
+    A, s = _acts(M, K, 11 * M + G)
+    big = torch.zeros((M, K + 64), dtype=torch.bfloat16, device="cuda")
+    big[:, :K] = to_device(A, True)
+    plan = lib.Plan.rht(K, s)
+    codes, scales = guarded_quant(lib, big[:, :K], plan, 4, G)
+    assert_codes_match(codes, scales, Hd.rht_apply(A, s), 4, G)
 
 
 @pytest.mark.parametrize("G", [32, 64, 128])
