@@ -81,12 +81,13 @@ def load_peaks():
 
 
 def kernel_sources_sha() -> str:
-    """Hash of the fused rotation kernel's device code: rot_fwht.cu up to its host launch code and
-    the device helpers of rot_internal.cuh (host code there does not change the kernel)."""
+    """Hash of the timed rotation kernel's device code: rot_fwht.cu up to the few-row kernel (the
+    helpers, the generic fused kernel and the tensor-core kernel the bench times) and the device
+    helpers of rot_internal.cuh (host code does not change the kernel)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "hadamard_butterfly_rotation_b200", "csrc")
     src = open(os.path.join(csrc, "rot_fwht.cu"), "rb").read()
-    h.update(src[:src.find(b"\nsize_t mma_smem_bytes(")])
+    h.update(src[:src.find(b"\n// Few-row kernel for 4096-coordinate chunks")])
     hdr = open(os.path.join(csrc, "rot_internal.cuh"), "rb").read()
     h.update(hdr[hdr.find(b"device helpers"):])
     return h.hexdigest()[:16]
